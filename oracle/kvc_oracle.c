@@ -1,0 +1,320 @@
+/*
+ * kvc_oracle.c -- plain, slow, float64 CPU oracle for observation-window
+ * token scoring, selection and KV / hidden-state compaction.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or
+ * calls this file; only the tests, the smoke check and the CPU-baseline leg
+ * of the benchmark do.  It shares no code, header, table or helper with the
+ * CUDA library.
+ *
+ * What it follows (citations are to the pages the method is described on):
+ *  - FastKV (gist.science 2502.01068), section 2.A "Token-Selective
+ *    Propagation": at the TSP layer the importance of each context token is
+ *    judged from the attention that a window of recent tokens pays to it, and
+ *    the window tokens themselves always go forward with the selected ones.
+ *  - FastKV, section 2.B "KV retention decoupled": two independent budgets
+ *    (TSP rate, KV retention rate) rank the same scores.
+ *  - FastKV abstract (chatpaper.ai / arXiv 2502.01068): the KV compression is
+ *    GQA-aware, i.e. one retained set per KV head, shared by its query group.
+ *  - StructKV (gist.science 2604.06746), section 2.A: the global in-degree
+ *    centrality C_global is the sum of the per-layer attention contributions;
+ *    section 2.B: per-layer attention entropy, sparsity and variance.
+ * Numeric details the pages leave open are fixed as follows (plainest
+ * reading): contributions are SUMMED over window rows and group heads; the
+ * query head h belongs to KV head floor(h / G); the softmax of window row i
+ * runs over every key at or before its own position (causal inside the
+ * window); pooling is a zero-padded centred moving average over the prefix
+ * (window keys excluded) divided by the kernel size; ties in the ranking go
+ * to the lower position.
+ *
+ * Every floating-point step is float64.  bf16 inputs arrive as raw uint16
+ * bit patterns and are widened exactly.
+ *
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -shared -fPIC.  Defining
+ * ORACLE_MUTANT=n compiles a deliberately wrong variant; the pin tests use
+ * those to show that each plausible mistake is caught.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+
+int oracle_mutant(void) { return ORACLE_MUTANT; }
+
+int oracle_max_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+static double bf16_to_f64(uint16_t bits) {
+  uint32_t u = (uint32_t)bits << 16;
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
+/* KV head that query head h reads (contiguous grouping). */
+static int kv_head_of(int h, int H, int Hkv) {
+#if ORACLE_MUTANT == 3
+  (void)H;
+  return h % Hkv; /* mutant: interleaved grouping */
+#else
+  return h / (H / Hkv);
+#endif
+}
+
+/* s = scale * <q, k> */
+static double logit(const double* q, const double* k, int d, double scale) {
+  double acc = 0.0;
+  for (int c = 0; c < d; ++c) acc += q[c] * k[c];
+#if ORACLE_MUTANT == 2
+  (void)scale;
+  return acc; /* mutant: scale dropped */
+#else
+  return scale * acc;
+#endif
+}
+
+/* Last key that window row i may see: its own position N - w + i. */
+static int64_t last_visible(int64_t N, int w, int i) {
+#if ORACLE_MUTANT == 1
+  (void)w; (void)i;
+  return N - 1; /* mutant: no causal mask inside the window */
+#else
+  return N - w + i;
+#endif
+}
+
+/*
+ * Window attention aggregate of one sequence.
+ *   q : [w][H][d] bf16 bits, element (i, h, c) at q[i*q_si + h*q_sh + c]
+ *   k : [N][Hkv][d] bf16 bits, element (j, g, c) at k[j*k_sn + g*k_sh + c]
+ *   A : [Hkv][N] float64 out, A[g*N + j] =
+ *         sum over query heads h of group g, window rows i with j <= N-w+i,
+ *         of softmax_j( scale * q[i,h] . k[j,g] )
+ * Returns 0 on success, -1 on bad arguments.
+ */
+int oracle_window_scores(const uint16_t* q, int64_t q_si, int64_t q_sh,
+                         const uint16_t* k, int64_t k_sn, int64_t k_sh,
+                         int64_t N, int H, int Hkv, int d, int w, double scale,
+                         double* A) {
+  if (!q || !k || !A || H <= 0 || Hkv <= 0 || H % Hkv || d <= 0 || w < 1 || w > N)
+    return -1;
+  const int G = H / Hkv;
+  const int R = G * w; /* rows per KV head */
+  double* kd = (double*)malloc(sizeof(double) * (size_t)N * d);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)R * d);
+  double* m = (double*)malloc(sizeof(double) * R);
+  double* l = (double*)malloc(sizeof(double) * R);
+  int64_t* last = (int64_t*)malloc(sizeof(int64_t) * R);
+  if (!kd || !qd || !m || !l || !last) {
+    free(kd); free(qd); free(m); free(l); free(last);
+    return -1;
+  }
+  for (int g = 0; g < Hkv; ++g) {
+    /* widen this KV head's keys and its group's window queries */
+    for (int64_t j = 0; j < N; ++j)
+      for (int c = 0; c < d; ++c) kd[j * d + c] = bf16_to_f64(k[j * k_sn + (int64_t)g * k_sh + c]);
+    int r = 0;
+    for (int h = 0; h < H; ++h) {
+      if (kv_head_of(h, H, Hkv) != g) continue;
+      for (int i = 0; i < w; ++i, ++r) {
+        for (int c = 0; c < d; ++c) qd[r * d + c] = bf16_to_f64(q[i * q_si + (int64_t)h * q_sh + c]);
+        last[r] = last_visible(N, w, i);
+      }
+    }
+    /* softmax normaliser of every row: max and sum of exp over visible keys */
+#pragma omp parallel
+    {
+      double* s = (double*)malloc(sizeof(double) * (size_t)N);
+#pragma omp for schedule(dynamic, 1)
+      for (int rr = 0; rr < R; ++rr) {
+        double mx = -INFINITY;
+        for (int64_t j = 0; j <= last[rr]; ++j) {
+          s[j] = logit(qd + rr * d, kd + j * d, d, scale);
+          if (s[j] > mx) mx = s[j];
+        }
+        double sum = 0.0;
+        for (int64_t j = 0; j <= last[rr]; ++j) sum += exp(s[j] - mx);
+        m[rr] = mx;
+        l[rr] = sum;
+      }
+      free(s);
+    }
+    /* A[g, j] = sum over rows of the normalised probability of key j */
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < N; ++j) {
+      double a = 0.0;
+      for (int rr = 0; rr < R; ++rr) {
+        if (j > last[rr]) continue;
+        a += exp(logit(qd + rr * d, kd + j * d, d, scale) - m[rr]) / l[rr];
+      }
+      A[(int64_t)g * N + j] = a;
+    }
+  }
+  free(kd); free(qd); free(m); free(l); free(last);
+  return 0;
+}
+
+/* out[j] = sum_r rows[r*stride + j], r = 0..nrows-1 (TSP aggregate, C_global). */
+void oracle_sum_rows(const double* rows, int nrows, int64_t stride, int64_t n, double* out) {
+  for (int64_t j = 0; j < n; ++j) {
+    double s = 0.0;
+    for (int r = 0; r < nrows; ++r) s += rows[(int64_t)r * stride + j];
+    out[j] = s;
+  }
+}
+
+/*
+ * Zero-padded centred moving average with odd kernel p:
+ *   y[j] = (1/p) * sum_{t=-(p/2)}^{p/2} x[j+t],  x[.] = 0 outside [0, L).
+ */
+int oracle_avg_pool(const double* x, int64_t L, int p, double* y) {
+  if (p < 1 || (p & 1) == 0) return -1;
+  const int half = p / 2;
+  for (int64_t j = 0; j < L; ++j) {
+    double s = 0.0;
+    int cnt = 0;
+    for (int t = -half; t <= half; ++t) {
+      int64_t u = j + t;
+      if (u < 0 || u >= L) continue;
+      s += x[u];
+      ++cnt;
+    }
+#if ORACLE_MUTANT == 4
+    y[j] = s / cnt; /* mutant: divide by the in-range count */
+#else
+    (void)cnt;
+    y[j] = s / p;
+#endif
+  }
+  return 0;
+}
+
+typedef struct {
+  double s;
+  int64_t j;
+} keyed_t;
+
+/* higher score first; equal scores: lower position first */
+static int by_score_then_pos(const void* a, const void* b) {
+  const keyed_t* x = (const keyed_t*)a;
+  const keyed_t* y = (const keyed_t*)b;
+  if (x->s > y->s) return -1;
+  if (x->s < y->s) return 1;
+#if ORACLE_MUTANT == 5
+  return (x->j < y->j) ? 1 : (x->j > y->j) ? -1 : 0; /* mutant: higher position wins ties */
+#else
+  return (x->j < y->j) ? -1 : (x->j > y->j) ? 1 : 0;
+#endif
+}
+
+static int cmp_i32(const void* a, const void* b) {
+  int32_t x = *(const int32_t*)a, y = *(const int32_t*)b;
+  return (x > y) - (x < y);
+}
+
+/*
+ * Top-k that always keeps the window.
+ *   S   : ranking scores of the prefix positions 0..N-w-1 (already pooled)
+ *   k   : budget INCLUDING the w window positions, k >= w
+ *   idx : out, min(k, N) positions in ascending order: the k-w best prefix
+ *         positions (score descending, ties to the lower position) together
+ *         with the window N-w..N-1; if k >= N every position is kept.
+ * Returns the number of indices written, or -1 on bad arguments.
+ */
+int64_t oracle_select_topk(const double* S, int64_t N, int w, int64_t k, int32_t* idx) {
+  if (w < 1 || w > N || k < w) return -1;
+  if (k >= N) {
+    for (int64_t j = 0; j < N; ++j) idx[j] = (int32_t)j;
+    return N;
+  }
+  const int64_t L = N - w;
+  const int64_t kk = k - w;
+  keyed_t* v = (keyed_t*)malloc(sizeof(keyed_t) * (size_t)(L > 0 ? L : 1));
+  if (!v) return -1;
+  for (int64_t j = 0; j < L; ++j) {
+    v[j].s = S[j];
+    v[j].j = j;
+  }
+  qsort(v, (size_t)L, sizeof(keyed_t), by_score_then_pos);
+  int64_t n = 0;
+  for (int64_t t = 0; t < kk; ++t) idx[n++] = (int32_t)v[t].j;
+#if ORACLE_MUTANT == 6
+  for (int t = 0; t < w - 1; ++t) idx[n++] = (int32_t)(L + t); /* mutant: last window token dropped */
+  idx[n++] = (int32_t)v[kk].j;
+#else
+  for (int t = 0; t < w; ++t) idx[n++] = (int32_t)(L + t);
+#endif
+  qsort(idx, (size_t)n, sizeof(int32_t), cmp_i32);
+  free(v);
+  return n;
+}
+
+/*
+ * Row gather (bit copy): out[r*row_elems + c] = src[idx[r]*src_stride + c];
+ * idx[r] == -1 marks a padding row and writes zeros.  Returns the number of
+ * indices outside [-1, nsrc) (those rows are written as zeros too).
+ */
+int64_t oracle_gather_rows(const uint16_t* src, int64_t src_stride, int64_t nsrc, int64_t row_elems,
+                           const int32_t* idx, int64_t n, uint16_t* out) {
+  int64_t bad = 0;
+  for (int64_t r = 0; r < n; ++r) {
+    int64_t j = idx[r];
+    uint16_t* o = out + r * row_elems;
+    if (j < 0 || j >= nsrc) {
+      if (j != -1) ++bad;
+      memset(o, 0, sizeof(uint16_t) * (size_t)row_elems);
+      continue;
+    }
+    memcpy(o, src + j * src_stride, sizeof(uint16_t) * (size_t)row_elems);
+  }
+  return bad;
+}
+
+static int cmp_desc_f64(const void* a, const void* b) {
+  double x = *(const double*)a, y = *(const double*)b;
+  return (x < y) - (x > y);
+}
+
+/*
+ * Per-row attention statistics on a_hat = A / mass_norm (mass_norm = w*G, the
+ * exact total mass of one KV head's aggregate):
+ *   out[0] entropy        -sum a ln a   (0 ln 0 = 0), nats
+ *   out[1] top-1% mass     sum of the ceil(N/100) largest a
+ *   out[2] variance        (1/N) sum (a - mean)^2
+ */
+int oracle_layer_stats(const double* A, int64_t N, double mass_norm, double* out) {
+  if (N < 1 || !(mass_norm > 0)) return -1;
+  double* a = (double*)malloc(sizeof(double) * (size_t)N);
+  if (!a) return -1;
+  double ent = 0.0, sum = 0.0;
+  for (int64_t j = 0; j < N; ++j) {
+    a[j] = A[j] / mass_norm;
+    if (a[j] > 0) ent -= a[j] * log(a[j]);
+    sum += a[j];
+  }
+  const double mean = sum / (double)N;
+  double var = 0.0;
+  for (int64_t j = 0; j < N; ++j) var += (a[j] - mean) * (a[j] - mean);
+  var /= (double)N;
+  qsort(a, (size_t)N, sizeof(double), cmp_desc_f64);
+  const int64_t m = (N + 99) / 100;
+  double top = 0.0;
+  for (int64_t t = 0; t < m; ++t) top += a[t];
+  out[0] = ent;
+  out[1] = top;
+  out[2] = var;
+  free(a);
+  return 0;
+}

@@ -1,0 +1,291 @@
+"""Pins for the float64 oracle: checks against things other than the oracle.
+
+Each pin takes an oracle object and returns None when it holds or a string
+describing the violation.  The same functions run against the real oracle
+(every one must hold) and against deliberately broken builds of it (each
+broken build must violate at least one), which shows that a plausible
+mistake -- a dropped mask, a dropped scale, a wrong head->group map, a wrong
+pooling divisor, a reversed tie-break, a lost window token -- cannot hide.
+
+Sources the pins come from (none of them is the oracle's own code):
+  * closed form: with K = 0 every visible logit is 0, so each window row is
+    uniform over the keys it may see;
+  * a library attention routine: torch's scaled_dot_product_attention in
+    float64 with V = identity returns the attention probabilities;
+  * arbitrary-precision brute force (mpmath) on tiny inputs;
+  * the total mass invariant sum_j A[g, j] = w * G;
+  * scipy's zero-padded uniform filter for the pooling;
+  * the defining order property of a top-k with the lower-position tie-break;
+  * closed forms of entropy / top-1% mass / variance for uniform and one-hot
+    distributions, and scipy.stats.entropy / numpy.var.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+from workloads import f32_to_bf16_bits
+
+
+def _bf16(x):
+    return f32_to_bf16_bits(np.asarray(x, dtype=np.float32))
+
+
+def _rand_qk(rng, N, H, Hkv, d, w, qscale=1.0, kscale=1.0):
+    q = _bf16(rng.standard_normal((w, H, d)) * qscale)
+    k = _bf16(rng.standard_normal((N, Hkv, d)) * kscale)
+    return q, k
+
+
+def _widen(b):
+    return (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# --------------------------------------------------------------------------- #
+# scores
+# --------------------------------------------------------------------------- #
+def closed_form_zero_keys(N, H, Hkv, w):
+    """A for K = 0: row i is uniform over its p_i + 1 visible keys."""
+    G = H // Hkv
+    p = N - w + np.arange(w)          # last visible key of each window row
+    A = np.zeros(N)
+    for i in range(w):
+        A[: p[i] + 1] += 1.0 / (p[i] + 1)
+    return np.tile(G * A, (Hkv, 1))
+
+
+def pin_zero_keys(orc):
+    rng = np.random.default_rng(7)
+    for (N, H, Hkv, d, w) in [(40, 4, 2, 64, 6), (33, 6, 3, 128, 33), (17, 2, 1, 64, 1)]:
+        q = _bf16(rng.standard_normal((w, H, d)))
+        k = np.zeros((N, Hkv, d), dtype=np.uint16)
+        A = orc.window_scores(q, k, H, Hkv, w, 1 / math.sqrt(d))
+        ref = closed_form_zero_keys(N, H, Hkv, w)
+        err = np.max(np.abs(A - ref) / ref)
+        if err > 1e-13:
+            return f"K=0 closed form violated (N={N}, w={w}): rel err {err:.3e}"
+    return None
+
+
+def sdpa_probabilities(q_bits, k_bits, H, Hkv, w, scale):
+    """Attention probabilities from torch's SDPA (float64, V = identity)."""
+    import torch
+    q = torch.from_numpy(_widen(q_bits))            # [w][H][d]
+    k = torch.from_numpy(_widen(k_bits))            # [N][Hkv][d]
+    N = k.shape[0]
+    G = H // Hkv
+    qh = q.permute(1, 0, 2)                         # [H][w][d]
+    kh = k.permute(1, 0, 2).repeat_interleave(G, dim=0)   # [H][N][d], query head h -> KV head h // G
+    eye = torch.eye(N, dtype=torch.float64).expand(H, N, N)
+    pos = N - w + torch.arange(w)
+    mask = torch.arange(N)[None, :] <= pos[:, None]       # [w][N]
+    P = torch.nn.functional.scaled_dot_product_attention(qh, kh, eye, attn_mask=mask, scale=scale)
+    return P.numpy()                                # [H][w][N]
+
+
+def pin_sdpa(orc):
+    rng = np.random.default_rng(11)
+    for (N, H, Hkv, d, w) in [(48, 6, 2, 64, 5), (70, 8, 2, 128, 12), (24, 3, 3, 64, 24)]:
+        q, k = _rand_qk(rng, N, H, Hkv, d, w, qscale=1.5)
+        scale = 1 / math.sqrt(d)
+        A = orc.window_scores(q, k, H, Hkv, w, scale)
+        P = sdpa_probabilities(q, k, H, Hkv, w, scale)
+        G = H // Hkv
+        ref = P.reshape(Hkv, G, w, N).sum(axis=(1, 2))
+        err = np.max(np.abs(A - ref) / np.maximum(ref, 1e-300))
+        if err > 1e-10:
+            return f"SDPA(V=I) mismatch (N={N}, H={H}, Hkv={Hkv}, w={w}): rel err {err:.3e}"
+    return None
+
+
+def mpmath_scores(q_bits, k_bits, H, Hkv, w, scale, dps=40):
+    import mpmath
+    mpmath.mp.dps = dps
+    q = _widen(q_bits)
+    k = _widen(k_bits)
+    N, _, d = k.shape
+    G = H // Hkv
+    A = [[mpmath.mpf(0) for _ in range(N)] for _ in range(Hkv)]
+    sc = mpmath.mpf(scale)
+    for h in range(H):
+        g = h // G
+        for i in range(w):
+            last = N - w + i
+            s = [sc * mpmath.fsum(mpmath.mpf(float(q[i, h, c])) * mpmath.mpf(float(k[j, g, c]))
+                                  for c in range(d)) for j in range(last + 1)]
+            e = [mpmath.exp(x) for x in s]
+            z = mpmath.fsum(e)
+            for j in range(last + 1):
+                A[g][j] += e[j] / z
+    return np.array([[float(x) for x in row] for row in A])
+
+
+def pin_mpmath(orc):
+    rng = np.random.default_rng(13)
+    N, H, Hkv, d, w = 12, 4, 2, 8, 3
+    q, k = _rand_qk(rng, N, H, Hkv, d, w, qscale=3.0, kscale=2.0)
+    scale = 1 / math.sqrt(d)
+    A = orc.window_scores(q, k, H, Hkv, w, scale)
+    ref = mpmath_scores(q, k, H, Hkv, w, scale)
+    err = np.max(np.abs(A - ref) / ref)
+    if err > 1e-12:
+        return f"mpmath brute force mismatch: rel err {err:.3e}"
+    return None
+
+
+def pin_mass(orc):
+    rng = np.random.default_rng(17)
+    N, H, Hkv, d, w = 300, 8, 2, 64, 8
+    q, k = _rand_qk(rng, N, H, Hkv, d, w, qscale=2.0)
+    A = orc.window_scores(q, k, H, Hkv, w, 1 / math.sqrt(d))
+    tot = A.sum(axis=1)
+    err = np.max(np.abs(tot - w * (H // Hkv)))
+    if err > 1e-9:
+        return f"total mass != w*G (err {err:.3e})"
+    return None
+
+
+def pin_dominant_key(orc):
+    """A key far more aligned with every window query than any other takes
+    (almost) all the mass of every row that can see it."""
+    rng = np.random.default_rng(19)
+    N, H, Hkv, d, w = 64, 4, 2, 64, 4
+    q = _bf16(np.abs(rng.standard_normal((w, H, d))))
+    k = _bf16(rng.standard_normal((N, Hkv, d)) * 0.05)
+    k[10, :, :] = _bf16(np.full((Hkv, d), 8.0))
+    A = orc.window_scores(q, k, H, Hkv, w, 1 / math.sqrt(d))
+    G = H // Hkv
+    if np.any(A[:, 10] < w * G * (1 - 1e-9)):
+        return f"dominant key mass {A[:, 10]} below w*G={w * G}"
+    return None
+
+
+# --------------------------------------------------------------------------- #
+# pooling
+# --------------------------------------------------------------------------- #
+def pin_pool(orc):
+    from scipy.ndimage import uniform_filter1d
+    rng = np.random.default_rng(23)
+    for L in (1, 2, 5, 9, 100):
+        for p in (1, 3, 7):
+            x = rng.random(L)
+            y = orc.avg_pool(x, p)
+            ref = uniform_filter1d(x, size=p, mode="constant", cval=0.0)
+            if np.max(np.abs(y - ref)) > 1e-14:
+                return f"pool mismatch vs scipy uniform_filter1d (L={L}, p={p})"
+    # closed form on a constant vector: c * (h + 1 + t) / p at distance t < h from an end
+    c, p, L = 3.0, 7, 20
+    y = orc.avg_pool(np.full(L, c), p)
+    h = p // 2
+    for t in range(h):
+        want = c * (h + 1 + t) / p
+        if abs(y[t] - want) > 1e-14 or abs(y[L - 1 - t] - want) > 1e-14:
+            return f"pool edge closed form violated at t={t}"
+    if np.max(np.abs(y[h:L - h] - c)) > 1e-14:
+        return "pool interior of a constant vector is not the constant"
+    return None
+
+
+# --------------------------------------------------------------------------- #
+# selection
+# --------------------------------------------------------------------------- #
+def check_selection(S, N, w, k, idx):
+    """Defining property of the selection; returns a message or None."""
+    idx = np.asarray(idx)
+    if k >= N:
+        return None if np.array_equal(idx, np.arange(N)) else "k >= N must keep every position"
+    if len(idx) != k:
+        return f"|set| = {len(idx)} != k = {k}"
+    if np.any(np.diff(idx) <= 0):
+        return "indices not strictly increasing"
+    L = N - w
+    if not np.all(np.isin(np.arange(L, N), idx)):
+        return "window not kept"
+    chosen = idx[idx < L]
+    if len(chosen) != k - w:
+        return "wrong number of prefix positions"
+    mask = np.zeros(L, bool)
+    mask[chosen] = True
+    if mask.all() or not mask.any():
+        return None
+    lo = S[mask].min()
+    hi = S[~mask].max()
+    if lo < hi:
+        return "an unselected prefix position outranks a selected one"
+    if lo == hi:
+        # equal scores at the boundary: selected ones must have the lower positions
+        sel_eq = np.flatnonzero(mask & (S == lo))
+        uns_eq = np.flatnonzero(~mask & (S == lo))
+        if sel_eq.max() > uns_eq.min():
+            return "tie at the boundary not broken toward the lower position"
+    return None
+
+
+def pin_select(orc):
+    rng = np.random.default_rng(29)
+    for trial in range(200):
+        N = int(rng.integers(2, 60))
+        w = int(rng.integers(1, N + 1))
+        k = int(rng.integers(w, N + 3))
+        S = rng.integers(0, 4, size=N - w).astype(np.float64)   # many ties
+        idx = orc.select_topk(S, N, w, k)
+        msg = check_selection(S, N, w, k, idx)
+        if msg:
+            return f"{msg} (N={N}, w={w}, k={k})"
+    # all scores equal: the lowest k-w prefix positions plus the window
+    N, w, k = 50, 5, 12
+    idx = orc.select_topk(np.ones(N - w), N, w, k)
+    want = np.concatenate([np.arange(k - w), np.arange(N - w, N)])
+    if not np.array_equal(idx, want):
+        return "all-equal scores must select 0..k-w-1 plus the window"
+    return None
+
+
+# --------------------------------------------------------------------------- #
+# gather
+# --------------------------------------------------------------------------- #
+def pin_gather(orc):
+    rng = np.random.default_rng(31)
+    src = rng.integers(0, 1 << 16, size=(50, 3, 16), dtype=np.uint16)
+    idx = np.array([3, 0, 49, 7, -1, 12], dtype=np.int32)
+    for g in range(3):
+        out, bad = orc.gather_rows(src[:, g, :], idx)
+        ref = src[np.where(idx < 0, 0, idx), g, :].copy()
+        ref[idx < 0] = 0
+        if bad != 0 or not np.array_equal(out, ref):
+            return "gather differs from numpy indexing"
+    out, bad = orc.gather_rows(src[:, 0, :], np.array([1, 50, -7, 2], dtype=np.int32))
+    if bad != 2 or np.any(out[1:3] != 0):
+        return "out-of-range indices must be counted and zero-filled"
+    return None
+
+
+# --------------------------------------------------------------------------- #
+# statistics
+# --------------------------------------------------------------------------- #
+def pin_stats(orc):
+    from scipy.stats import entropy
+    N = 1000
+    m = (N + 99) // 100
+    uni = orc.layer_stats(np.full(N, 5.0), 5.0 * N)
+    if abs(uni[0] - math.log(N)) > 1e-12 or abs(uni[1] - m / N) > 1e-12 or abs(uni[2]) > 1e-18:
+        return f"uniform closed form violated: {uni}"
+    one = np.zeros(N)
+    one[37] = 2.5
+    oh = orc.layer_stats(one, 2.5)
+    if abs(oh[0]) > 1e-15 or abs(oh[1] - 1.0) > 1e-15 or abs(oh[2] - (1 / N) * (1 - 1 / N)) > 1e-15:
+        return f"one-hot closed form violated: {oh}"
+    rng = np.random.default_rng(37)
+    a = rng.random(777) ** 3
+    st = orc.layer_stats(a, a.sum())
+    ah = a / a.sum()
+    top = np.sort(ah)[::-1][: (777 + 99) // 100].sum()
+    if (abs(st[0] - entropy(ah)) > 1e-12 or abs(st[1] - top) > 1e-12
+            or abs(st[2] - np.var(ah)) > 1e-15):
+        return "stats differ from scipy.stats.entropy / numpy.var / sorted sum"
+    return None
+
+
+ALL_PINS = [pin_zero_keys, pin_sdpa, pin_mpmath, pin_mass, pin_dominant_key, pin_pool,
+            pin_select, pin_gather, pin_stats]
