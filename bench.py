@@ -1,0 +1,372 @@
+"""Benchmark: one layer of window-attention scoring, selection and compaction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+A step is the whole path over one synthetic Llama-3-8B-shaped layer at
+N = 131072 context tokens (32 query heads, 8 KV heads, head_dim 128, window
+32, average pooling 7): window scores -> per-KV-head top-k (10 %, 13107 kept)
+-> K/V gather -> all-head TSP top-k (20 %, 26214 kept) -> hidden-state gather
+([N][4096] bf16).  Inputs are resident in HBM before the timed region; they
+are larger than L2 (K 268 MB, X 1.07 GB), so no explicit flush is used.
+
+With N > 1 (torchrun, one process per GPU) every rank compresses its own
+layer (independent sequences: weak scaling, no collective on the data path);
+time is the max over ranks.  `--impl reference` times the float64 CPU
+oracle on the same workload (bounded sample per step) instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "context tokens scored+compressed/s at N=128K per layer; achieved HBM GB/s"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def algorithmic_bytes(cfg) -> dict:
+    """Minimum HBM bytes of each call of one layer (reads + writes)."""
+    N, Hkv, d, H, w = cfg.N, cfg.Hkv, cfg.d, cfg.H, cfg.w
+    kk, kt, D = cfg.k_kv, cfg.k_tsp, cfg.hidden
+    return {
+        "score": N * Hkv * d * 2 + w * H * d * 2 + Hkv * N * 4,      # K once, Q_win, scores out
+        "select_kv": Hkv * N * 4 + Hkv * kk * 4,                     # scores in, indices out
+        "gather_kv": 2 * 2 * Hkv * kk * d * 2 + Hkv * kk * 4,        # K,V rows in+out, indices
+        "select_tsp": Hkv * N * 4 + kt * 4,
+        "gather_hidden": 2 * kt * D * 2 + kt * 4,
+    }
+
+
+def layer_bytes(cfg) -> int:
+    """Algorithmic bytes of the whole step (scores written once and read once)."""
+    b = algorithmic_bytes(cfg)
+    return (b["score"] + b["gather_kv"] + b["gather_hidden"] + cfg.Hkv * cfg.N * 4
+            + (cfg.Hkv * cfg.k_kv + cfg.k_tsp) * 4)
+
+
+def workload_config(cfg) -> dict:
+    return {"workload": cfg.name, "N": cfg.N, "H": cfg.H, "Hkv": cfg.Hkv, "d": cfg.d, "w": cfg.w,
+            "pool": cfg.pool, "k_kv": cfg.k_kv, "k_tsp": cfg.k_tsp, "hidden": cfg.hidden,
+            "l2": "inputs larger than L2 (K 268 MB, X 1.07 GB); no flush",
+            "parallelism": "one independent layer per rank"}
+
+
+# --------------------------------------------------------------------------- #
+# clocks (read-only NVML sampling during the timed region)
+# --------------------------------------------------------------------------- #
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+            0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """Median SM clock and active slowdown reasons while the GPU works."""
+
+    def __init__(self, cuda_index: int, period_s: float = 0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._t = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            pr = torch.cuda.get_device_properties(cuda_index)
+            try:
+                bus = f"{pr.pci_domain_id:08x}:{pr.pci_bus_id:02x}:{pr.pci_device_id:02x}.0"
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(cuda_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self._reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = self._reasons_fn(self.h)
+                for b, name in _REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's
+    source is unchanged since the capture; else None."""
+    try:
+        data = json.load(open(TRAFFIC_FILE))
+        ent = data[kernel]
+        src = os.path.join(ROOT, ent["source"])
+        if hashlib.sha256(open(src, "rb").read()).hexdigest() != ent["source_sha256"]:
+            return None
+        return ent["dram_bytes_per_launch"]
+    except Exception:
+        return None
+
+
+def measured_peaks():
+    try:
+        mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return float(mp["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# --------------------------------------------------------------------------- #
+# CPU oracle (baseline / reference arm)
+# --------------------------------------------------------------------------- #
+def oracle_head_step(orc, lay, cfg, g: int) -> None:
+    """One KV head of the layer on the oracle: its window scores over all N
+    keys, its pooled top-k and K/V gather, and 1/Hkv of the hidden gather."""
+    G = cfg.G
+    q = lay.q[:, g * G:(g + 1) * G, :]
+    k = lay.k[:, g:g + 1, :]
+    A = orc.window_scores(q, k, G, 1, cfg.w, cfg.scale)
+    S = orc.rank_scores(A[0], cfg.N, cfg.w, cfg.pool)
+    idx = orc.select_topk(S, cfg.N, cfg.w, cfg.k_kv)
+    orc.gather_rows(lay.k[:, g, :], idx, nsrc=cfg.N)
+    orc.gather_rows(lay.v[:, g, :], idx, nsrc=cfg.N)
+    it = orc.select_topk(S, cfg.N, cfg.w, cfg.k_tsp)
+    part = it[g::cfg.Hkv]
+    orc.gather_rows(lay.x, part)
+
+
+def cpu_baseline(orc, lay, cfg, heads: int = 8) -> dict:
+    t0 = time.perf_counter()
+    for g in range(heads):
+        oracle_head_step(orc, lay, cfg, g)
+    dt = time.perf_counter() - t0
+    per_layer = dt * cfg.Hkv / heads
+    return {"value": cfg.N / per_layer, "unit": "tokens/s", "cores": orc.max_threads(), "kind": "oracle",
+            "sample": f"{heads} of {cfg.Hkv} KV heads of one N={cfg.N} layer (scores over all keys, pooled "
+                      f"top-k, K/V gather, 1/{cfg.Hkv} of the hidden gather each), scaled to a full layer; "
+                      f"{dt:.1f} s wall"}
+
+
+def run_reference(args, cfg, rank: int) -> None:
+    if rank != 0:
+        return
+    import oracle
+    import workloads
+
+    orc = oracle.get()
+    lay = workloads.make_layer(cfg)
+    for s in range(args.warmup):
+        oracle_head_step(orc, lay, cfg, s % cfg.Hkv)
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        oracle_head_step(orc, lay, cfg, s % cfg.Hkv)
+    dt = (time.perf_counter() - t0) / args.steps  # seconds per head-step
+    value = cfg.N / (dt * cfg.Hkv)
+    sample = (f"each step: one KV head of the N={cfg.N} layer (scores over all keys, pooled top-k, K/V gather, "
+              f"1/{cfg.Hkv} of the hidden gather); a layer = {cfg.Hkv} steps")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 * cfg.Hkv,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(cfg),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": orc.max_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- #
+# CUDA arm
+# --------------------------------------------------------------------------- #
+def main() -> None:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    import workloads
+
+    cfg = workloads.C3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, cfg, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import long_context_kv_window_b200 as kvc
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    # ---- inputs: this rank's own layer, resident in HBM ----------------------
+    lay = workloads.make_layer(cfg, seed=cfg.seed + 1000 * rank)
+    q, k, v, x = (workloads.torch_bf16(a, dev) for a in (lay.q, lay.k, lay.v, lay.x))
+    plan = kvc.LayerPlan(cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden, True, dev,
+                         pool_kernel=cfg.pool)
+    st = torch.cuda.current_stream(dev)
+    calls = ["score", "select_kv", "gather_kv", "select_tsp", "gather_hidden"]
+
+    def step(evs=None):
+        def mark(i):
+            if evs is not None:
+                evs[i].record(st)
+        mark(0)
+        kvc.kvc_score(q, k, scores=plan.scores, ws=plan.ws_score, dev_err=plan.dev_err)
+        mark(1)
+        kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_kv, idx=plan.idx_kv, ws=plan.ws_sel_kv)
+        mark(2)
+        kvc.kvc_gather_kv(k, v, plan.idx_kv, k_out=plan.k_c, v_out=plan.v_c, dev_err=plan.dev_err)
+        mark(3)
+        kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_tsp, row_group=cfg.Hkv, idx=plan.idx_tsp,
+                            ws=plan.ws_sel_tsp)
+        mark(4)
+        kvc.kvc_gather_hidden(x, plan.idx_tsp.view(-1), out=plan.x_c, dev_err=plan.dev_err)
+        mark(5)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if plan.dev_err.item() != 0:
+        raise RuntimeError(f"device error word {plan.dev_err.item()}")
+
+    # ---- timed region ----------------------------------------------------------
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    launches0 = kvc.launch_count()
+    with sampler:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t_start.record(st)
+        for s in range(args.steps):
+            step(evs[s])
+        t_end.record(st)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    launches = kvc.launch_count() - launches0
+    ms_total = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_step = ms_total / args.steps
+    per_call = {c: sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps
+                for i, c in enumerate(calls)}
+
+    # ---- end to end through the public API with host buffers ------------------
+    hq, hk, hv, hx = (workloads.torch_bf16(a).pin_memory() for a in (lay.q, lay.k, lay.v, lay.x))
+    h_idx_kv = torch.empty(plan.idx_kv.shape, dtype=torch.int32).pin_memory()
+    h_idx_tsp = torch.empty(plan.idx_tsp.shape, dtype=torch.int32).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hx))
+    d2h = h_idx_kv.numel() * 4 + h_idx_tsp.numel() * 4
+
+    def e2e_step():
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        x.copy_(hx, non_blocking=True)
+        plan.run(q, k, v, x)
+        h_idx_kv.copy_(plan.idx_kv, non_blocking=True)
+        h_idx_tsp.copy_(plan.idx_tsp, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(st)
+    torch.cuda.synchronize(dev)
+    ms_e2e = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+
+    # ---- roofline of the dominant call -----------------------------------------
+    peak, peak_kind = measured_peaks()
+    alg = algorithmic_bytes(cfg)
+    dom = max(per_call, key=per_call.get)
+    ach = alg[dom] / (per_call[dom] * 1e-3) / 1e9
+    breakdown = {c: {"ms": round(per_call[c], 5), "alg_bytes": alg[c],
+                     "gbs": round(alg[c] / (per_call[c] * 1e-3) / 1e9, 1)} for c in calls}
+
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            cpu = cpu_baseline(oracle.get(), lay, cfg)
+        line = {
+            "metric": METRIC, "value": world * cfg.N / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(cfg),
+            "hbm_gbs": round(layer_bytes(cfg) / (ms_step * 1e-3) / 1e9, 1),
+            "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
+                         "traffic": load_traffic(dom)},
+            "calls": breakdown,
+            "e2e": {"value": world * cfg.N / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
+            "gpu_launches": launches,
+            "clocks": sampler.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,382 @@
+"""Python binding of libkvc: window-attention token scoring, top-k selection
+that keeps the window, and K/V / hidden-state compaction on B200 (sm_100a).
+
+Argument marshalling only.  Every step runs in the CUDA kernels of
+``libkvc.so`` (built in-tree by ``python -m long_context_kv_window_b200.build``);
+PyTorch supplies device memory and the current stream.  There is no CPU path:
+if the library is missing, importing the functions raises.
+
+Names follow the C ABI in ``include/kvc.h``.  Tensors are CUDA tensors; bf16
+inputs may be ``torch.bfloat16`` or raw ``int16``/``uint16`` bit patterns.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libkvc.so")
+
+KVC_OK = 0
+KVC_DEV_ERR_INDEX = 1
+KVC_DEV_ERR_SEQLENS = 2
+KVC_DEV_ERR_TIMEOUT = 4
+
+
+class KvcError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str):
+        super().__init__(f"{where}: {status_string(status)} ({detail})")
+        self.status = status
+
+
+class ScoreParams(ctypes.Structure):
+    _fields_ = [("num_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("window", ctypes.c_int32), ("scale", ctypes.c_float)]
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_I32 = ctypes.c_int32
+_SZ = ctypes.c_size_t
+
+_SIGS = {
+    "kvc_abi_version": ([], _I32),
+    "kvc_status_string": ([_I32], ctypes.c_char_p),
+    "kvc_last_error": ([], ctypes.c_char_p),
+    "kvc_launch_count": ([], _I64),
+    "kvc_score_workspace_size": ([_P, _I32, _I64, _P], _I32),
+    "kvc_score": ([_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
+    "kvc_score_varlen": ([_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I32, _I64, _I64, _P, _P, _P, _P,
+                          _P, _SZ, _P, _P], _I32),
+    "kvc_select_workspace_size": ([_I32, _I32, _I64, _P], _I32),
+    "kvc_select_topk": ([_P, _I32, _I64, _I32, _I64, _I32, _I32, _I64, _P, _I64, _P, _P, _SZ, _P], _I32),
+    "kvc_select_topk_varlen": ([_P, _I32, _I64, _I32, _P, _I32, _I64, _I64, _I32, _I32, _I64, _P, _P, _P,
+                                _SZ, _P, _P], _I32),
+    "kvc_gather_kv": ([_P, _P, _I64, _I64, _I64, _I32, _I32, _P, _I64, _I64, _P, _P, _P, _P], _I32),
+    "kvc_gather_kv_varlen": ([_P, _P, _I64, _I64, _P, _I32, _I64, _I32, _I32, _P, _I64, _P, _P, _P, _P],
+                             _I32),
+    "kvc_gather_hidden": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P, _P], _I32),
+    "kvc_stats_workspace_size": ([_I32, _I64, _P], _I32),
+    "kvc_layer_stats": ([_P, _I32, _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P], _I32),
+}
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libkvc.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m long_context_kv_window_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().kvc_status_string(s).decode()
+
+
+def last_error() -> str:
+    return lib().kvc_last_error().decode()
+
+
+def launch_count() -> int:
+    """Kernels launched by libkvc in this process."""
+    return int(lib().kvc_launch_count())
+
+
+def abi_version() -> int:
+    return int(lib().kvc_abi_version())
+
+
+def _check(status: int, where: str) -> None:
+    if status != KVC_OK:
+        raise KvcError(status, where, last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream]):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
+        raise TypeError(f"{name} must hold bf16 values (bfloat16 or int16/uint16 bits)")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name} must be contiguous in its last dimension")
+    return t
+
+
+def _dev(t: torch.Tensor, name: str, dtype: torch.dtype) -> torch.Tensor:
+    if t.dtype != dtype or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA {dtype} tensor")
+    return t
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# --------------------------------------------------------------------------- #
+# scoring
+# --------------------------------------------------------------------------- #
+def score_params(H: int, Hkv: int, d: int, w: int, scale: Optional[float] = None) -> ScoreParams:
+    return ScoreParams(H, Hkv, d, w, float(1.0 / math.sqrt(d) if scale is None else scale))
+
+
+def score_workspace_size(p: ScoreParams, batch: int, total: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().kvc_score_workspace_size(ctypes.byref(p), batch, total, ctypes.byref(out)),
+           "kvc_score_workspace_size")
+    return int(out.value)
+
+
+def kvc_score(q_win: torch.Tensor, k: torch.Tensor, scale: Optional[float] = None,
+              scores: Optional[torch.Tensor] = None, tsp: Optional[torch.Tensor] = None,
+              accum: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+              dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Window-attention aggregate A [Hkv][n] (fp32) of q_win [w][H][d] over k [n][Hkv][d]."""
+    _bf16(q_win, "q_win")
+    _bf16(k, "k")
+    w, H, d = q_win.shape
+    n, Hkv, dk = k.shape
+    if dk != d:
+        raise ValueError("head_dim of q_win and k differ")
+    p = score_params(H, Hkv, d, w, scale)
+    if scores is None:
+        scores = torch.empty((Hkv, n), dtype=torch.float32, device=k.device)
+    if ws is None:
+        ws = _workspace(score_workspace_size(p, 1, n), k.device)
+    _check(lib().kvc_score(_ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k), k.stride(0), k.stride(1),
+                           n, ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum), _ptr(ws),
+                           ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)), "kvc_score")
+    return scores
+
+
+def kvc_score_varlen(q_win: torch.Tensor, k: torch.Tensor, cu_seqlens: torch.Tensor, max_seqlen: int,
+                     scale: Optional[float] = None, scores: Optional[torch.Tensor] = None,
+                     tsp: Optional[torch.Tensor] = None, accum: Optional[torch.Tensor] = None,
+                     ws: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Ragged batch: q_win [B][w][H][d], k [total][Hkv][d] packed, cu_seqlens int32 [B+1]."""
+    _bf16(q_win, "q_win")
+    _bf16(k, "k")
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    B, w, H, d = q_win.shape
+    total, Hkv, _ = k.shape
+    p = score_params(H, Hkv, d, w, scale)
+    if scores is None:
+        scores = torch.empty((Hkv, total), dtype=torch.float32, device=k.device)
+    if ws is None:
+        ws = _workspace(score_workspace_size(p, B, total), k.device)
+    _check(lib().kvc_score_varlen(_ptr(q_win), q_win.stride(0), q_win.stride(1), q_win.stride(2), _ptr(k),
+                                  k.stride(0), k.stride(1), _ptr(cu_seqlens), B, total, int(max_seqlen),
+                                  ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum), _ptr(ws),
+                                  ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)),
+           "kvc_score_varlen")
+    return scores
+
+
+# --------------------------------------------------------------------------- #
+# selection
+# --------------------------------------------------------------------------- #
+def select_workspace_size(out_rows: int, batch: int, total: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().kvc_select_workspace_size(out_rows, batch, total, ctypes.byref(out)),
+           "kvc_select_workspace_size")
+    return int(out.value)
+
+
+def kvc_select_topk(scores: torch.Tensor, window: int, pool_kernel: int, k: int, row_group: int = 1,
+                    n: Optional[int] = None, idx: Optional[torch.Tensor] = None,
+                    pooled: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                    stream=None) -> torch.Tensor:
+    """Per output row: the k - window best (pooled) prefix positions plus the
+    window, ascending.  scores [rows][>= n] fp32; returns int32 [rows/row_group][min(k, n)]."""
+    _dev(scores, "scores", torch.float32)
+    rows = scores.shape[0]
+    n = scores.shape[1] if n is None else n
+    out_rows = rows // row_group
+    kout = min(k, n)
+    if idx is None:
+        idx = torch.empty((out_rows, kout), dtype=torch.int32, device=scores.device)
+    if ws is None and pooled is None:
+        ws = _workspace(select_workspace_size(out_rows, 1, n), scores.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().kvc_select_topk(_ptr(scores), rows, scores.stride(0), row_group, n, window, pool_kernel, k,
+                                 _ptr(idx), idx.stride(0), _ptr(pooled), _ptr(ws), nbytes, _stream(stream)),
+           "kvc_select_topk")
+    return idx
+
+
+def kvc_select_topk_varlen(scores: torch.Tensor, cu_seqlens: torch.Tensor, max_seqlen: int, window: int,
+                           pool_kernel: int, k: int, row_group: int = 1, idx: Optional[torch.Tensor] = None,
+                           counts: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                           dev_err: Optional[torch.Tensor] = None,
+                           stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Ragged batch; returns (idx int32 [B][rows/row_group][k] local positions, -1 padded,
+    counts int32 [B])."""
+    _dev(scores, "scores", torch.float32)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    rows, total = scores.shape[0], scores.shape[1]
+    B = cu_seqlens.numel() - 1
+    out_rows = rows // row_group
+    if idx is None:
+        idx = torch.empty((B, out_rows, k), dtype=torch.int32, device=scores.device)
+    if counts is None:
+        counts = torch.empty((B,), dtype=torch.int32, device=scores.device)
+    if ws is None:
+        ws = _workspace(select_workspace_size(out_rows, B, total), scores.device)
+    _check(lib().kvc_select_topk_varlen(_ptr(scores), rows, scores.stride(0), row_group, _ptr(cu_seqlens), B,
+                                        total, int(max_seqlen), window, pool_kernel, k, _ptr(idx),
+                                        _ptr(counts), _ptr(ws), ws.numel() * ws.element_size(),
+                                        _ptr(dev_err), _stream(stream)), "kvc_select_topk_varlen")
+    return idx, counts
+
+
+# --------------------------------------------------------------------------- #
+# gathers
+# --------------------------------------------------------------------------- #
+def kvc_gather_kv(k: torch.Tensor, v: Optional[torch.Tensor], idx: torch.Tensor,
+                  k_out: Optional[torch.Tensor] = None, v_out: Optional[torch.Tensor] = None,
+                  dev_err: Optional[torch.Tensor] = None, stream=None):
+    """k, v [n][Hkv][d]; idx int32 [Hkv][kk] (or [1][kk] broadcast) -> k_out, v_out [Hkv][kk][d]."""
+    _bf16(k, "k")
+    if v is not None:
+        _bf16(v, "v")
+        if v.stride() != k.stride() or v.shape != k.shape:
+            raise ValueError("k and v must have the same shape and strides")
+    _dev(idx, "idx", torch.int32)
+    n, Hkv, d = k.shape
+    kk = idx.shape[-1]
+    irs = 0 if idx.shape[0] == 1 and Hkv > 1 else idx.stride(0)
+    if k_out is None:
+        k_out = torch.empty((Hkv, kk, d), dtype=k.dtype, device=k.device)
+    if v is not None and v_out is None:
+        v_out = torch.empty((Hkv, kk, d), dtype=v.dtype, device=v.device)
+    _check(lib().kvc_gather_kv(_ptr(k), _ptr(v), k.stride(0), k.stride(1), n, Hkv, d, _ptr(idx), irs, kk,
+                               _ptr(k_out), _ptr(v_out if v is not None else None), _ptr(dev_err),
+                               _stream(stream)), "kvc_gather_kv")
+    return k_out, v_out
+
+
+def kvc_gather_kv_varlen(k: torch.Tensor, v: Optional[torch.Tensor], cu_seqlens: torch.Tensor,
+                         idx: torch.Tensor, k_out: Optional[torch.Tensor] = None,
+                         v_out: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                         stream=None):
+    """k, v [total][Hkv][d]; idx int32 [B][Hkv][kk] local positions -> [B][Hkv][kk][d]."""
+    _bf16(k, "k")
+    _dev(idx, "idx", torch.int32)
+    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    total, Hkv, d = k.shape
+    B, _, kk = idx.shape
+    if k_out is None:
+        k_out = torch.empty((B, Hkv, kk, d), dtype=k.dtype, device=k.device)
+    if v is not None and v_out is None:
+        v_out = torch.empty((B, Hkv, kk, d), dtype=v.dtype, device=v.device)
+    _check(lib().kvc_gather_kv_varlen(_ptr(k), _ptr(v), k.stride(0), k.stride(1), _ptr(cu_seqlens), B, total,
+                                      Hkv, d, _ptr(idx), kk, _ptr(k_out), _ptr(v_out if v is not None else None),
+                                      _ptr(dev_err), _stream(stream)), "kvc_gather_kv_varlen")
+    return k_out, v_out
+
+
+def kvc_gather_hidden(x: torch.Tensor, idx: torch.Tensor, out: Optional[torch.Tensor] = None,
+                      dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """x [n][D] -> out [kk][D] = x[idx]."""
+    _bf16(x, "x")
+    _dev(idx, "idx", torch.int32)
+    n, D = x.shape
+    kk = idx.numel()
+    if out is None:
+        out = torch.empty((kk, D), dtype=x.dtype, device=x.device)
+    _check(lib().kvc_gather_hidden(_ptr(x), x.stride(0), n, D, _ptr(idx), kk, _ptr(out), _ptr(dev_err),
+                                   _stream(stream)), "kvc_gather_hidden")
+    return out
+
+
+# --------------------------------------------------------------------------- #
+# statistics
+# --------------------------------------------------------------------------- #
+def kvc_layer_stats(scores: torch.Tensor, mass_norm: float, n: Optional[int] = None,
+                    out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Per row of scores: [entropy, top-1% mass, variance] of scores/mass_norm."""
+    _dev(scores, "scores", torch.float32)
+    rows = scores.shape[0]
+    n = scores.shape[1] if n is None else n
+    if out is None:
+        out = torch.empty((rows, 3), dtype=torch.float32, device=scores.device)
+    _check(lib().kvc_layer_stats(_ptr(scores), rows, scores.stride(0), n, float(mass_norm), _ptr(out), None, 0,
+                                 _stream(stream)), "kvc_layer_stats")
+    return out
+
+
+# --------------------------------------------------------------------------- #
+# one layer of the method, composed from the calls above
+# --------------------------------------------------------------------------- #
+@dataclass
+class LayerOutputs:
+    scores: torch.Tensor                    # [Hkv][n] fp32
+    idx_kv: torch.Tensor                    # [Hkv][k_kv] int32
+    k_c: torch.Tensor                       # [Hkv][k_kv][d]
+    v_c: Optional[torch.Tensor]
+    idx_tsp: Optional[torch.Tensor] = None  # [1][k_tsp] int32
+    x_c: Optional[torch.Tensor] = None      # [k_tsp][D]
+    tsp: Optional[torch.Tensor] = None      # [n] fp32 (when requested)
+
+
+class LayerPlan:
+    """Pre-allocated buffers for repeated calls of ``compress_layer`` on one shape."""
+
+    def __init__(self, n: int, H: int, Hkv: int, d: int, w: int, k_kv: int, k_tsp: Optional[int],
+                 hidden: Optional[int], with_v: bool, device, pool_kernel: int = 1):
+        self.n, self.H, self.Hkv, self.d, self.w = n, H, Hkv, d, w
+        self.k_kv, self.k_tsp, self.hidden, self.pool = k_kv, k_tsp, hidden, pool_kernel
+        f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
+        self.params = score_params(H, Hkv, d, w)
+        self.scores = torch.empty((Hkv, n), dtype=f32, device=device)
+        self.ws_score = _workspace(score_workspace_size(self.params, 1, n), device)
+        self.ws_sel_kv = _workspace(select_workspace_size(Hkv, 1, n), device)
+        self.idx_kv = torch.empty((Hkv, min(k_kv, n)), dtype=i32, device=device)
+        self.k_c = torch.empty((Hkv, min(k_kv, n), d), dtype=bf, device=device)
+        self.v_c = torch.empty_like(self.k_c) if with_v else None
+        self.dev_err = torch.zeros(1, dtype=i32, device=device)
+        if k_tsp is not None:
+            self.ws_sel_tsp = _workspace(select_workspace_size(1, 1, n), device)
+            self.idx_tsp = torch.empty((1, min(k_tsp, n)), dtype=i32, device=device)
+            self.x_c = (torch.empty((min(k_tsp, n), hidden), dtype=bf, device=device)
+                        if hidden else None)
+
+    def run(self, q_win, k, v=None, x=None, stream=None) -> LayerOutputs:
+        """Score -> per-KV-head top-k -> K/V gather; with a TSP budget also the
+        all-head top-k -> hidden-state gather.  Nothing is synchronised."""
+        kvc_score(q_win, k, scores=self.scores, ws=self.ws_score, dev_err=self.dev_err, stream=stream)
+        kvc_select_topk(self.scores, self.w, self.pool, self.k_kv, idx=self.idx_kv, ws=self.ws_sel_kv,
+                        stream=stream)
+        kvc_gather_kv(k, v, self.idx_kv, k_out=self.k_c, v_out=self.v_c, dev_err=self.dev_err, stream=stream)
+        out = LayerOutputs(self.scores, self.idx_kv, self.k_c, self.v_c)
+        if self.k_tsp is not None:
+            kvc_select_topk(self.scores, self.w, self.pool, self.k_tsp, row_group=self.Hkv, idx=self.idx_tsp,
+                            ws=self.ws_sel_tsp, stream=stream)
+            out.idx_tsp = self.idx_tsp
+            if x is not None and self.x_c is not None:
+                kvc_gather_hidden(x, self.idx_tsp.view(-1), out=self.x_c, dev_err=self.dev_err, stream=stream)
+                out.x_c = self.x_c
+        return out

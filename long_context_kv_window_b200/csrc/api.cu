@@ -1,0 +1,62 @@
+// api.cu -- library-wide entry points: version, status strings, diagnostics.
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+
+namespace kvc {
+
+std::atomic<int64_t> g_launches{0};
+
+namespace {
+thread_local std::string t_last_error;
+}
+
+void set_error(const std::string& msg) { t_last_error = msg; }
+void clear_error() { t_last_error.clear(); }
+
+kvc_status fail(kvc_status s, const std::string& msg) {
+  set_error(msg);
+  return s;
+}
+
+kvc_status cuda_fail(cudaError_t e, const char* what) {
+  set_error(std::string(what) + ": " + cudaGetErrorString(e));
+  return KVC_ERR_CUDA;
+}
+
+int num_sms() {
+  static std::mutex mu;
+  static std::vector<int> cache;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+}  // namespace kvc
+
+extern "C" int32_t kvc_abi_version(void) { return KVC_ABI_VERSION; }
+
+extern "C" const char* kvc_status_string(kvc_status s) {
+  switch (s) {
+    case KVC_OK: return "KVC_OK";
+    case KVC_ERR_INVALID_ARG: return "KVC_ERR_INVALID_ARG";
+    case KVC_ERR_UNSUPPORTED: return "KVC_ERR_UNSUPPORTED";
+    case KVC_ERR_CUDA: return "KVC_ERR_CUDA";
+    case KVC_ERR_WORKSPACE: return "KVC_ERR_WORKSPACE";
+  }
+  return "KVC_ERR_UNKNOWN";
+}
+
+extern "C" const char* kvc_last_error(void) { return kvc::t_last_error.c_str(); }
+
+extern "C" int64_t kvc_launch_count(void) { return kvc::g_launches.load(); }

@@ -1,0 +1,80 @@
+// common.cuh -- shared host/device helpers of libkvc (sm_100a only).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+#include <string>
+
+#include "kvc.h"
+
+namespace kvc {
+
+// ---------------------------------------------------------------- host side
+// Thread-local reason of the last failing call (kvc_last_error).
+void set_error(const std::string& msg);
+void clear_error();
+kvc_status fail(kvc_status s, const std::string& msg);
+kvc_status cuda_fail(cudaError_t e, const char* what);
+
+// Count of kernels launched by this library (kvc_launch_count).
+extern std::atomic<int64_t> g_launches;
+inline void count_launch(int64_t n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Number of SMs of the current device (cached per device).
+int num_sms();
+
+inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+constexpr size_t kWsAlign = 256;
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Bump allocator over the caller's workspace.
+struct WsCursor {
+  char* base;
+  size_t cap;
+  size_t off = 0;
+  bool ok = true;
+  template <class T>
+  T* take(size_t count) {
+    size_t bytes = round_up(count * sizeof(T), kWsAlign);
+    if (off + bytes > cap) {
+      ok = false;
+      return nullptr;
+    }
+    T* p = reinterpret_cast<T*>(base + off);
+    off += bytes;
+    return p;
+  }
+};
+
+#define KVC_CUDA_TRY(expr)                                   \
+  do {                                                       \
+    cudaError_t _e = (expr);                                 \
+    if (_e != cudaSuccess) return ::kvc::cuda_fail(_e, #expr); \
+  } while (0)
+
+#define KVC_CHECK_ARG(cond, msg) \
+  do {                           \
+    if (!(cond)) return ::kvc::fail(KVC_ERR_INVALID_ARG, msg); \
+  } while (0)
+
+// -------------------------------------------------------------- device side
+__device__ __forceinline__ void set_dev_err(int32_t* err, int32_t bit) {
+  if (err) atomicOr(err, bit);
+}
+
+// Sequence b of a (possibly ragged) batch: [start, start + len).
+// cu == nullptr means a single sequence of length `n`.
+struct SeqSpan {
+  int64_t start;
+  int64_t len;
+};
+__device__ __forceinline__ SeqSpan seq_span(const int32_t* cu, int b, int64_t n) {
+  if (cu == nullptr) return {0, n};
+  int64_t s = cu[b], e = cu[b + 1];
+  return {s, e - s};
+}
+
+}  // namespace kvc

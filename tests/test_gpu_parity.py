@@ -1,0 +1,287 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle on
+the same seeded inputs.  Scores within relative 1e-3, index sets identical
+up to the near-tie band, gathers bit-exact (see tests/parity.py)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import long_context_kv_window_b200 as kvc
+import oracle
+import workloads
+from tests import parity
+from tests.gpu_helpers import check_layer, dev_bf16, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    kvc.lib()  # fail loudly if the library is missing
+    torch.cuda.set_device(0)
+
+
+def _err_word():
+    return torch.zeros(1, dtype=torch.int32, device="cuda")
+
+
+# --------------------------------------------------------------------------- #
+# gathers
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("d", [64, 128])
+def test_gather_kv_bit_exact(d):
+    rng = np.random.default_rng(5)
+    N, Hkv, kk = 777, 3, 100
+    k = rng.integers(0, 1 << 16, size=(N, Hkv, d), dtype=np.uint16)
+    v = rng.integers(0, 1 << 16, size=(N, Hkv, d), dtype=np.uint16)
+    idx = np.sort(rng.choice(N, size=(Hkv, kk), replace=True), axis=1).astype(np.int32)
+    idx[1, 5] = -1
+    err = _err_word()
+    ko, vo = kvc.kvc_gather_kv(dev_bf16(k), dev_bf16(v), torch.from_numpy(idx).cuda(), dev_err=err)
+    orc = oracle.get()
+    ref_k, bad_k = orc.gather_kv(k, idx)
+    ref_v, _ = orc.gather_kv(v, idx)
+    assert bad_k == 0 and err.item() == 0
+    assert np.array_equal(host_bits(ko), ref_k) and np.array_equal(host_bits(vo), ref_v)
+    # out-of-range indices: zero rows and the device error bit
+    idx[0, 0] = N
+    idx[2, 3] = -5
+    ko, vo = kvc.kvc_gather_kv(dev_bf16(k), dev_bf16(v), torch.from_numpy(idx).cuda(), dev_err=err)
+    ref_k, bad = orc.gather_kv(k, idx)
+    assert bad == 2 and err.item() == kvc.KVC_DEV_ERR_INDEX
+    assert np.array_equal(host_bits(ko), ref_k)
+
+
+def test_gather_kv_broadcast_index_row():
+    rng = np.random.default_rng(6)
+    N, Hkv, d, kk = 300, 4, 128, 37
+    k = rng.integers(0, 1 << 16, size=(N, Hkv, d), dtype=np.uint16)
+    idx = np.sort(rng.choice(N, size=kk, replace=False)).astype(np.int32)
+    ko, vo = kvc.kvc_gather_kv(dev_bf16(k), None, torch.from_numpy(idx[None]).cuda())
+    assert vo is None
+    ref, _ = oracle.get().gather_kv(k, np.tile(idx, (Hkv, 1)))
+    assert np.array_equal(host_bits(ko), ref)
+
+
+@pytest.mark.parametrize("D", [4096, 1000, 8])
+def test_gather_hidden_bit_exact(D):
+    rng = np.random.default_rng(7)
+    N, kk = 513, 200
+    x = rng.integers(0, 1 << 16, size=(N, D), dtype=np.uint16)
+    idx = rng.integers(-1, N, size=kk).astype(np.int32)
+    err = _err_word()
+    out = kvc.kvc_gather_hidden(dev_bf16(x), torch.from_numpy(idx).cuda(), dev_err=err)
+    ref, bad = oracle.get().gather_rows(x, idx)
+    assert bad == 0 and err.item() == 0
+    assert np.array_equal(host_bits(out), ref)
+
+
+# --------------------------------------------------------------------------- #
+# selection on given scores
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("n,w,k", [(50, 5, 12), (1000, 8, 64), (4097, 32, 1000), (20000, 32, 2048),
+                                   (300, 10, 10), (300, 10, 300), (300, 10, 1000), (131072, 32, 13107)])
+def test_select_exact_on_given_scores_no_pool(n, w, k):
+    """Without pooling the GPU ranks exactly the values the oracle ranks: the
+    sets must be identical (ties included: many repeated values)."""
+    rng = np.random.default_rng(n + k)
+    S = rng.integers(0, 50, size=(3, n)).astype(np.float32) * 0.25
+    idx = kvc.kvc_select_topk(torch.from_numpy(S).cuda(), w, 1, k).cpu().numpy()
+    orc = oracle.get()
+    for r in range(3):
+        ref = orc.select_topk(S[r, : n - w].astype(np.float64), n, w, k)
+        assert np.array_equal(idx[r], ref), f"row {r}"
+
+
+@pytest.mark.parametrize("pool", [3, 7])
+def test_select_pooled_and_grouped(pool):
+    rng = np.random.default_rng(pool)
+    n, w, k, rows, grp = 9000, 16, 700, 8, 4
+    S = (rng.random((rows, n)) ** 4).astype(np.float32)
+    pooled = torch.empty((rows // grp, n - w), dtype=torch.float32, device="cuda")
+    idx = kvc.kvc_select_topk(torch.from_numpy(S).cuda(), w, pool, k, row_group=grp, pooled=pooled)
+    idx = idx.cpu().numpy()
+    orc = oracle.get()
+    for o in range(rows // grp):
+        T = orc.sum_rows(S[o * grp:(o + 1) * grp].astype(np.float64))
+        Sp = orc.rank_scores(T, n, w, pool)
+        ref = orc.select_topk(Sp, n, w, k)
+        parity.assert_scores_close(pooled[o].cpu().numpy(), Sp, rtol=1e-6, what="pooled")
+        parity.assert_selection_matches(idx[o], ref, Sp, n, w, k)
+
+
+# --------------------------------------------------------------------------- #
+# scoring + selection + gathers on the configurations
+# --------------------------------------------------------------------------- #
+def _run_layer(lay, cfg, k_kv=None, k_tsp=None):
+    q = dev_bf16(lay.q)
+    kd = dev_bf16(lay.k)
+    vd = dev_bf16(lay.v) if lay.v is not None else None
+    N = lay.k.shape[0]
+    err = _err_word()
+    tsp = torch.empty(N, dtype=torch.float32, device="cuda") if k_tsp else None
+    scores = kvc.kvc_score(q, kd, tsp=tsp, dev_err=err)
+    idx = kvc.kvc_select_topk(scores, cfg.w, cfg.pool, k_kv or cfg.k_kv)
+    ko, vo = kvc.kvc_gather_kv(kd, vd, idx, dev_err=err)
+    out = dict(scores=scores.cpu().numpy(), idx=idx.cpu().numpy(), k_c=host_bits(ko),
+               v_c=host_bits(vo) if vo is not None else None, err=err.item())
+    if k_tsp:
+        it = kvc.kvc_select_topk(scores, cfg.w, cfg.pool, k_tsp, row_group=cfg.Hkv)
+        out["tsp"] = tsp.cpu().numpy()
+        out["idx_tsp"] = it.cpu().numpy()[0]
+    return out
+
+
+def test_tiny_config_end_to_end():
+    cfg = workloads.C1
+    lay = workloads.make_layer(cfg)
+    g = _run_layer(lay, cfg)
+    assert g["err"] == 0
+    res, err, kinds = check_layer(lay, cfg, g["scores"], g["idx"], what="tiny")
+    assert err < 1e-4, err
+    ref_k, _ = oracle.get().gather_kv(lay.k, g["idx"])
+    ref_v, _ = oracle.get().gather_kv(lay.v, g["idx"])
+    assert np.array_equal(g["k_c"], ref_k) and np.array_equal(g["v_c"], ref_v)
+    for gg in range(cfg.Hkv):
+        assert np.all(np.isin(lay.hitters[0], g["idx"][gg]))
+    assert np.allclose(g["scores"].sum(axis=1), cfg.rows, rtol=1e-5)
+
+
+@pytest.mark.parametrize("N", [8, 9, 100, 127, 128, 129, 1000, 4097])
+def test_tiny_heads_edge_lengths(N):
+    """Tile edges, ragged tails and the window covering (almost) everything."""
+    cfg = workloads.shrink(workloads.C1, N=N, n_hitters=min(4, max(0, N - 8 - 1)), k_kv=min(64, N), seed=1000 + N)
+    lay = workloads.make_layer(cfg)
+    g = _run_layer(lay, cfg)
+    check_layer(lay, cfg, g["scores"], g["idx"], what=f"N={N}")
+
+
+@pytest.mark.parametrize("N,H,Hkv,w,pool,k", [(129, 32, 8, 32, 7, 64), (300, 32, 8, 32, 7, 100),
+                                                (2000, 40, 8, 32, 1, 500), (3000, 16, 2, 8, 5, 333),
+                                                (5000, 8, 8, 16, 7, 999)])
+def test_d128_shapes(N, H, Hkv, w, pool, k):
+    cfg = workloads.shrink(workloads.C2, N=N, H=H, Hkv=Hkv, w=w, pool=pool, k_kv=k,
+                           n_sinks=min(4, N - w), n_hitters=min(8, N - w - 4), seed=2000 + N)
+    lay = workloads.make_layer(cfg)
+    g = _run_layer(lay, cfg)
+    check_layer(lay, cfg, g["scores"], g["idx"], what=f"H={H} Hkv={Hkv} N={N}")
+
+
+def test_llama_32k_full_size():
+    cfg = workloads.C2
+    lay = workloads.make_layer(cfg)
+    g = _run_layer(lay, cfg)
+    assert g["err"] == 0
+    res, err, kinds = check_layer(lay, cfg, g["scores"], g["idx"], what="32K")
+    print(f"32K: max score rel err {err:.2e}, selection kinds {kinds}")
+    for gg in range(cfg.Hkv):
+        assert np.all(np.isin(lay.sinks[0], g["idx"][gg]))
+        assert np.all(np.isin(lay.hitters[0], g["idx"][gg]))
+    ref_k, _ = oracle.get().gather_kv(lay.k, g["idx"])
+    assert np.array_equal(g["k_c"], ref_k)
+
+
+def test_tsp_aggregate_and_selection():
+    cfg = workloads.shrink(workloads.C3, N=20000, k_kv=2000, k_tsp=4000, hidden=None, n_hitters=32, seed=3001)
+    lay = workloads.make_layer(cfg, with_x=False)
+    g = _run_layer(lay, cfg, k_tsp=cfg.k_tsp)
+    res = oracle.layer(lay.q, lay.k, cfg.H, cfg.Hkv, cfg.w, cfg.scale, cfg.pool, cfg.k_kv, k_tsp=cfg.k_tsp)
+    parity.assert_scores_close(g["tsp"], res.T, what="tsp")
+    parity.assert_selection_matches(g["idx_tsp"], res.idx_tsp, res.pooled_tsp, cfg.N, cfg.w, cfg.k_tsp)
+    assert abs(g["tsp"].sum() - cfg.w * cfg.H) < 1e-3 * cfg.w * cfg.H
+
+
+def test_cross_layer_accumulation():
+    cfg = workloads.shrink(workloads.C5, N=3000, layers=3, k_kv=256, k_tsp=450, n_hitters=16)
+    C = torch.zeros((cfg.Hkv, cfg.N), dtype=torch.float32, device="cuda")
+    Cref = np.zeros((cfg.Hkv, cfg.N))
+    for ell in range(1, cfg.layers + 1):
+        lay = workloads.make_layer(cfg, layer=ell)
+        kvc.kvc_score(dev_bf16(lay.q), dev_bf16(lay.k), accum=C)
+        Cref += oracle.get().window_scores(lay.q, lay.k, cfg.H, cfg.Hkv, cfg.w, cfg.scale)
+    parity.assert_scores_close(C.cpu().numpy(), Cref, what="C_global")
+
+
+# --------------------------------------------------------------------------- #
+# ragged batch
+# --------------------------------------------------------------------------- #
+def test_varlen_matches_oracle_and_single_sequence_calls():
+    cfg = workloads.shrink(workloads.C4, len_range=(200, 5000), k_kv=150, n_hitters=4, seed=4001)
+    lay = workloads.make_layer(cfg)
+    B = lay.batch
+    lens = lay.lengths()
+    cu = torch.from_numpy(lay.cu_seqlens).cuda()
+    q = dev_bf16(lay.q).view(B, cfg.w, cfg.H, cfg.d)
+    kd = dev_bf16(lay.k)
+    vd = dev_bf16(lay.v)
+    err = _err_word()
+    scores = kvc.kvc_score_varlen(q, kd, cu, int(lens.max()), dev_err=err)
+    idx, counts = kvc.kvc_select_topk_varlen(scores, cu, int(lens.max()), cfg.w, cfg.pool, cfg.k_kv, dev_err=err)
+    ko, vo = kvc.kvc_gather_kv_varlen(kd, vd, cu, idx, dev_err=err)
+    assert err.item() == 0
+    S = scores.cpu().numpy()
+    I = idx.cpu().numpy()
+    KO = host_bits(ko)
+    assert np.array_equal(counts.cpu().numpy(), np.minimum(cfg.k_kv, lens))
+    orc = oracle.get()
+    for b in range(B):
+        s0, s1 = lay.cu_seqlens[b], lay.cu_seqlens[b + 1]
+        qb, kb = lay.q[b * cfg.w:(b + 1) * cfg.w], lay.k[s0:s1]
+        res = oracle.layer(qb, kb, cfg.H, cfg.Hkv, cfg.w, cfg.scale, cfg.pool, cfg.k_kv)
+        parity.assert_scores_close(S[:, s0:s1], res.A, what=f"seq {b}")
+        m = min(cfg.k_kv, lens[b])
+        for g in range(cfg.Hkv):
+            parity.assert_selection_matches(I[b, g, :m], res.idx_kv[g], res.pooled[g], lens[b], cfg.w, cfg.k_kv)
+            assert np.all(I[b, g, m:] == -1)
+        ref_k, _ = orc.gather_kv(kb, I[b, :, :m])
+        assert np.array_equal(KO[b, :, :m], ref_k)
+        assert np.all(KO[b, :, m:] == 0)
+        # the same sequence through the single-sequence entry points: bit-identical
+        s_single = kvc.kvc_score(dev_bf16(qb), dev_bf16(kb))
+        i_single = kvc.kvc_select_topk(s_single, cfg.w, cfg.pool, cfg.k_kv)
+        assert np.array_equal(s_single.cpu().numpy(), S[:, s0:s1])
+        assert np.array_equal(i_single.cpu().numpy(), I[b, :, :m])
+
+
+def test_varlen_bad_seqlens_flagged():
+    cfg = workloads.shrink(workloads.C4, len_range=(100, 300), batch=3, n_hitters=2)
+    lay = workloads.make_layer(cfg)
+    cu_np = lay.cu_seqlens.copy()
+    cu_np[2] = cu_np[1] + 10  # sequence 1 shorter than the window
+    cu = torch.from_numpy(cu_np).cuda()
+    q = dev_bf16(lay.q).view(3, cfg.w, cfg.H, cfg.d)
+    err = _err_word()
+    scores = kvc.kvc_score_varlen(q, dev_bf16(lay.k), cu, 400, dev_err=err)
+    idx, counts = kvc.kvc_select_topk_varlen(scores, cu, 400, cfg.w, cfg.pool, 64, dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() & kvc.KVC_DEV_ERR_SEQLENS
+    assert counts[1].item() == 0 and torch.all(idx[1] == -1)
+
+
+# --------------------------------------------------------------------------- #
+# statistics
+# --------------------------------------------------------------------------- #
+def test_layer_stats_against_oracle():
+    cfg = workloads.shrink(workloads.C5, N=6000, layers=1, k_tsp=None)
+    lay = workloads.make_layer(cfg, layer=1)
+    A = oracle.get().window_scores(lay.q, lay.k, cfg.H, cfg.Hkv, cfg.w, cfg.scale)
+    gpu_scores = kvc.kvc_score(dev_bf16(lay.q), dev_bf16(lay.k))
+    st = kvc.kvc_layer_stats(gpu_scores, cfg.w * cfg.G).cpu().numpy()
+    for g in range(cfg.Hkv):
+        ref = oracle.get().layer_stats(A[g], cfg.w * cfg.G)
+        parity.assert_scores_close(st[g], ref, what=f"stats head {g}")
+
+
+def test_layer_stats_closed_forms():
+    n = 5000
+    uni = torch.full((1, n), 3.0, device="cuda")
+    st = kvc.kvc_layer_stats(uni, 3.0 * n).cpu().numpy()[0]
+    assert abs(st[0] - math.log(n)) < 1e-4 * math.log(n)
+    assert abs(st[1] - 50 / n) < 1e-6 and abs(st[2]) < 1e-12
+    one = torch.zeros((1, n), device="cuda")
+    one[0, 17] = 2.0
+    st = kvc.kvc_layer_stats(one, 2.0).cpu().numpy()[0]
+    assert abs(st[0]) < 1e-7 and abs(st[1] - 1) < 1e-6 and abs(st[2] - (1 / n) * (1 - 1 / n)) < 1e-9

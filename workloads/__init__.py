@@ -145,6 +145,14 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.asarray(b, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32)
 
 
+def torch_bf16(bits: np.ndarray, device=None):
+    """uint16 bf16 bit patterns -> torch.bfloat16 tensor with the same bits
+    (on `device` when given)."""
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16)
+    return t if device is None else t.to(device)
+
+
 def normal_bf16(seedseq: np.random.SeedSequence, shape) -> np.ndarray:
     n = int(np.prod(shape))
     return f32_to_bf16_bits(_normal_f32(seedseq, n)).reshape(shape)
