@@ -58,7 +58,8 @@ def layer_bytes(cfg) -> int:
 def workload_config(cfg) -> dict:
     return {"workload": cfg.name, "N": cfg.N, "H": cfg.H, "Hkv": cfg.Hkv, "d": cfg.d, "w": cfg.w,
             "pool": cfg.pool, "k_kv": cfg.k_kv, "k_tsp": cfg.k_tsp, "hidden": cfg.hidden,
-            "l2": "inputs larger than L2 (K 268 MB, X 1.07 GB); no flush",
+            "l2": (f"inputs larger than L2 (K {cfg.N * cfg.Hkv * cfg.d * 2 / 1e6:.0f} MB, "
+                   f"X {cfg.N * cfg.hidden * 2 / 1e9:.2f} GB); no flush"),
             "parallelism": "one independent layer per rank"}
 
 
@@ -217,12 +218,19 @@ def main() -> None:
     ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="same layer structure at another N (small cases for profiling)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    args.e2e_steps = max(args.e2e_steps, 1)
 
     import workloads
 
     cfg = workloads.C3
+    if args.tokens:
+        cfg = workloads.shrink(cfg, name=f"{cfg.name}_at_n{args.tokens}", N=args.tokens,
+                               k_kv=int(0.1 * args.tokens), k_tsp=int(0.2 * args.tokens),
+                               n_hitters=min(cfg.n_hitters, args.tokens // 64))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -235,6 +243,7 @@ def main() -> None:
     import torch.distributed as dist
 
     import long_context_kv_window_b200 as kvc
+    from long_context_kv_window_b200 import shard
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -291,11 +300,7 @@ def main() -> None:
         if world > 1:
             dist.barrier()
     launches = kvc.launch_count() - launches0
-    ms_total = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = shard.max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     ms_step = ms_total / args.steps
     per_call = {c: sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps
                 for i, c in enumerate(calls)}
@@ -327,11 +332,7 @@ def main() -> None:
         e2e_step()
     e1.record(st)
     torch.cuda.synchronize(dev)
-    ms_e2e = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([ms_e2e], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_e2e = float(t.item())
+    ms_e2e = shard.max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dist, dev)
 
     # ---- roofline of the dominant call -----------------------------------------
     peak, peak_kind = measured_peaks()

@@ -178,6 +178,8 @@ kvc_status kvc_select_topk(const float* scores, int32_t rows, int64_t row_stride
  * output row, min(k, len_b) LOCAL positions (0-based within the sequence)
  * are written to idx[(b*out_rows + o)*k ...] and the rest of the k entries
  * are set to -1.  counts [B] int32 out (or NULL) receives min(k, len_b).
+ * max_seqlen must bound every sequence length: a longer sequence is not
+ * ranked (its row is -1, counts 0) and sets KVC_DEV_ERR_SEQLENS.
  */
 kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, int64_t row_stride,
                                   int32_t row_group, const int32_t* cu_seqlens, int32_t batch,

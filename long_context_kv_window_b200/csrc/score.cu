@@ -13,10 +13,12 @@
 // aggregate takes two passes over K:
 //   pass 1 (rows on the MMA M axis, keys on N): each epilogue thread owns one
 //          row and keeps an online max / sum of 2^(s*log2e - max) over its
-//          chunk of keys; chunk partials are combined by the last CTA of the
-//          (sequence, head) into one bias b_r = max_r + log2(sum_r) per row;
-//   pass 2 (keys on M, rows on N): each epilogue thread owns one key and sums
-//          2^(s*log2e - b_r) over the rows -- a thread-local reduction.
+//          chunk of keys and writes that chunk partial to the workspace;
+//   pass 2 (keys on M, rows on N): the epilogue first combines the chunk
+//          partials of its (sequence, head) into one bias
+//          b_r = max_r + log2(sum_r) per row, while TMA and MMA already run;
+//          then each epilogue thread owns one key and sums 2^(s*log2e - b_r)
+//          over the rows -- a thread-local reduction.
 // Both passes stream the same K tiles (TMA, 128-byte swizzle) into a
 // multi-stage shared-memory ring; heads are processed in groups whose K fits
 // in L2, so pass 2 re-reads K from L2 rather than HBM.
@@ -61,8 +63,6 @@ struct ScoreArgs {
   float c;                   // scale * log2(e)
   float* part_m;             // [Hkv][max_chunks][Rq]
   double* part_l;            // [Hkv][max_chunks][Rq]
-  float* bias;               // [B][Hkv][Rq]
-  int* counters;             // [B][Hkv]
   float* scores;             // [Hkv][total]
   float* accum;              // [Hkv][total] or nullptr
   int64_t total;
@@ -112,8 +112,6 @@ struct Barriers {
   uint64_t tempty[2];
   uint32_t tmem_base;
   int abort;
-  int last;
-  int epi_ok;
 };
 
 // Q rows of KV head g into the K-major 128-byte swizzled layout; rows past R
@@ -166,7 +164,7 @@ __device__ __forceinline__ void produce(const void* kmap, Barriers* bars, uint8_
 __device__ __forceinline__ void record_timeout(int32_t* err) { set_dev_err(err, KVC_DEV_ERR_TIMEOUT); }
 
 // --------------------------------------------------------------------------
-// pass 1: per-row max / sum over a chunk of keys; last CTA builds the bias
+// pass 1: per-row max / sum over a chunk of keys
 // --------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kThreadsScore, 1)
@@ -200,7 +198,6 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
       tc::mbar_init(&bars->tempty[s], kEpiWarps);
     }
     bars->abort = 0;
-    bars->last = 0;
     tc::fence_mbar_init();
   }
   if (warp == 0 && lane == 0) tc::prefetch_tmap(&kmap);
@@ -274,17 +271,22 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
         }
         const int r = mb * kTile + rl;
         if (r >= a.R) continue;
-        const int64_t last_key = first_window_key + r / a.G;  // causal bound of this row
         const bool full_tile = (j0 + kTile - 1 <= first_window_key);
-        float tmax = -INFINITY;
+        if (!full_tile) {
+          // keys past this row's own position (or past the sequence) are masked to -inf
+          const int64_t last_key = first_window_key + r / a.G;
+#pragma unroll
+          for (int cc = 0; cc < 4; ++cc)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (j0 + cc * 32 + e > last_key) x[cc][e] = __float_as_uint(-INFINITY);
+        }
+        float t4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float v = __uint_as_float(x[cc][e]);
-            const bool ok = full_tile || (j0 + cc * 32 + e <= last_key);
-            tmax = ok ? fmaxf(tmax, v) : tmax;
-          }
+          for (int e = 0; e < 32; ++e) t4[e & 3] = fmaxf(t4[e & 3], __uint_as_float(x[cc][e]));
+        const float tmax = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
         if (tmax == -INFINITY) continue;
         const float ynew = tmax * a.c;
         if (ynew > m_run[mb]) {
@@ -296,20 +298,12 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float v = __uint_as_float(x[cc][e]);
-            const bool ok = full_tile || (j0 + cc * 32 + e <= last_key);
-            const float p = tc::ex2_approx(fmaf(v, a.c, mneg));
-            s4[e & 3] += ok ? p : 0.f;
-          }
+          for (int e = 0; e < 32; ++e) s4[e & 3] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e]), a.c, mneg));
         l_run[mb] += (double)((s4[0] + s4[1]) + (s4[2] + s4[3]));
       }
     }
-    // ---- chunk partials, then the last CTA of (sequence, head) combines ----
-    tc::named_bar_sync(1, 32 * kEpiWarps);
-    if (warp == 2 && lane == 0) bars->epi_ok = !bars->abort;
-    tc::named_bar_sync(1, 32 * kEpiWarps);
-    if (bars->epi_ok) {
+    // ---- chunk partials (combined by pass 2) ----------------------------------
+    if (!bars->abort) {
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb) {
         if (mb >= a.nb1) break;
@@ -318,33 +312,6 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
         const size_t slot = ((size_t)g * a.max_chunks + wk.gid) * a.Rq + r;
         a.part_m[slot] = m_run[mb];
         a.part_l[slot] = l_run[mb];
-      }
-      __threadfence();
-      tc::named_bar_sync(1, 32 * kEpiWarps);
-      if (warp == 2 && lane == 0) {
-        const int prev = atomicAdd(&a.counters[wk.b * a.Hkv + g], 1);
-        bars->last = (prev == wk.nchunks - 1);
-      }
-      tc::named_bar_sync(1, 32 * kEpiWarps);
-      if (bars->last) {
-        __threadfence();
-        const int gid0 = wk.gid - wk.chunk;
-        for (int mb = 0; mb < a.nb1; ++mb) {
-          const int r = mb * kTile + rl;
-          if (r >= a.R) continue;
-          float mx = -INFINITY;
-          for (int cidx = 0; cidx < wk.nchunks; ++cidx)
-            mx = fmaxf(mx, __ldcg(&a.part_m[((size_t)g * a.max_chunks + gid0 + cidx) * a.Rq + r]));
-          double l = 0.0;
-          for (int cidx = 0; cidx < wk.nchunks; ++cidx) {
-            const size_t slot = ((size_t)g * a.max_chunks + gid0 + cidx) * a.Rq + r;
-            const float mc = __ldcg(&a.part_m[slot]);
-            if (mc == -INFINITY) continue;
-            l += __ldcg(&a.part_l[slot]) * exp2((double)mc - (double)mx);
-          }
-          a.bias[((size_t)wk.b * a.Hkv + g) * a.Rq + r] = (float)((double)mx + log2(l));
-        }
-        if (warp == 2 && lane == 0) a.counters[wk.b * a.Hkv + g] = 0;
       }
     }
   }
@@ -402,9 +369,6 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
     tc::tmem_relinquish();
   }
   load_q_swizzled<D>(a, wk.b, g, qs);
-  // padded columns get +inf bias, so 2^(x*c - inf) = 0 needs no mask
-  for (int r = threadIdx.x; r < a.Rn; r += blockDim.x)
-    bias_s[r] = (r < a.R) ? a.bias[((size_t)wk.b * a.Hkv + g) * a.Rq + r] : INFINITY;
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
@@ -437,6 +401,46 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
       if (t > 0) tc::mbar_drain(&bars->tfull[(t - 1) & 1], ((t - 1) >> 1) & 1);
     }
   } else {
+    // ---- epilogue prologue: per-row bias from the pass-1 chunk partials --------
+    // b_r = M + log2(sum_c l_c 2^(m_c - M)), M = max_c m_c.  Padded columns get
+    // b = +inf, so 2^(x*c - inf) = 0 needs no mask.  The producer and MMA warps
+    // are already filling the pipeline meanwhile.
+    {
+      const int et = threadIdx.x - 64;  // 0..127
+      const size_t base_slot = ((size_t)g * a.max_chunks + (wk.gid - wk.chunk)) * a.Rq;
+      for (int r = et; r < a.Rn; r += 32 * kEpiWarps) {
+        if (r >= a.R) {
+          bias_s[r] = INFINITY;
+          continue;
+        }
+        constexpr int kB = 8;
+        float mx = -INFINITY;
+        for (int c0 = 0; c0 < wk.nchunks; c0 += kB) {
+          float mv[kB];
+#pragma unroll
+          for (int u = 0; u < kB; ++u)
+            mv[u] = (c0 + u < wk.nchunks) ? __ldcg(&a.part_m[base_slot + (size_t)(c0 + u) * a.Rq + r]) : -INFINITY;
+#pragma unroll
+          for (int u = 0; u < kB; ++u) mx = fmaxf(mx, mv[u]);
+        }
+        double l = 0.0;
+        for (int c0 = 0; c0 < wk.nchunks; c0 += kB) {
+          float mv[kB];
+          double lv[kB];
+#pragma unroll
+          for (int u = 0; u < kB; ++u) {
+            const bool in = c0 + u < wk.nchunks;
+            mv[u] = in ? __ldcg(&a.part_m[base_slot + (size_t)(c0 + u) * a.Rq + r]) : -INFINITY;
+            lv[u] = in ? __ldcg(&a.part_l[base_slot + (size_t)(c0 + u) * a.Rq + r]) : 0.0;
+          }
+#pragma unroll
+          for (int u = 0; u < kB; ++u)
+            if (mv[u] != -INFINITY) l += lv[u] * (double)exp2f(mv[u] - mx);
+        }
+        bias_s[r] = (float)((double)mx + log2(l));
+      }
+      tc::named_bar_sync(1, 32 * kEpiWarps);
+    }
     // ---- epilogue: one key per thread ------------------------------------------
     const int q = warp & 3;
     const int kl = 32 * q + lane;              // key within the tile
@@ -472,43 +476,42 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&bars->tempty[acc]);
         }
-        if (!masked_tile) {
+        if (masked_tile) {
+          // window rows see only keys up to their own position; later keys (and
+          // keys past the sequence) get logit -inf, i.e. probability 0
 #pragma unroll
           for (int cc = 0; cc < 4; ++cc) {
             if (cc >= nfull) break;
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float4 bb = *reinterpret_cast<const float4*>(&bias_s[col0 + cc * 32 + e]);
-              s4[0] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 0]), a.c, -bb.x));
-              s4[1] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 1]), a.c, -bb.y));
-              s4[2] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 2]), a.c, -bb.z));
-              s4[3] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 3]), a.c, -bb.w));
-            }
+            for (int e = 0; e < 32; ++e)
+              if (j > first_window_key + (col0 + cc * 32 + e) / a.G) x[cc][e] = __float_as_uint(-INFINITY);
           }
           if (tail16) {
 #pragma unroll
-            for (int e = 0; e < 16; e += 4) {
-              const float4 bb = *reinterpret_cast<const float4*>(&bias_s[col0 + nfull * 32 + e]);
-              s4[0] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 0]), a.c, -bb.x));
-              s4[1] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 1]), a.c, -bb.y));
-              s4[2] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 2]), a.c, -bb.z));
-              s4[3] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 3]), a.c, -bb.w));
-            }
+            for (int e = 0; e < 16; ++e)
+              if (j > first_window_key + (col0 + nfull * 32 + e) / a.G) xt[e] = __float_as_uint(-INFINITY);
           }
-        } else {
+        }
 #pragma unroll
-          for (int cc = 0; cc < 5; ++cc) {
-            const int width = (cc < nfull) ? 32 : ((cc == nfull && tail16) ? 16 : 0);
-            if (width == 0) break;
+        for (int cc = 0; cc < 4; ++cc) {
+          if (cc >= nfull) break;
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              if (e >= width) break;
-              const int r = col0 + cc * 32 + e;
-              const uint32_t raw = (cc < 4 && cc < nfull) ? x[cc < 4 ? cc : 0][e] : xt[e];
-              const bool ok = (r < a.R) && (j <= first_window_key + r / a.G);
-              const float p = tc::ex2_approx(fmaf(__uint_as_float(raw), a.c, -bias_s[r]));
-              s4[e & 3] += ok ? p : 0.f;
-            }
+          for (int e = 0; e < 32; e += 4) {
+            const float4 bb = *reinterpret_cast<const float4*>(&bias_s[col0 + cc * 32 + e]);
+            s4[0] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 0]), a.c, -bb.x));
+            s4[1] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 1]), a.c, -bb.y));
+            s4[2] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 2]), a.c, -bb.z));
+            s4[3] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 3]), a.c, -bb.w));
+          }
+        }
+        if (tail16) {
+#pragma unroll
+          for (int e = 0; e < 16; e += 4) {
+            const float4 bb = *reinterpret_cast<const float4*>(&bias_s[col0 + nfull * 32 + e]);
+            s4[0] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 0]), a.c, -bb.x));
+            s4[1] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 1]), a.c, -bb.y));
+            s4[2] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 2]), a.c, -bb.z));
+            s4[3] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 3]), a.c, -bb.w));
           }
         }
       }
@@ -594,8 +597,6 @@ size_t score_ws_bytes(const kvc_score_params* p, int B, int64_t total) {
   const Geometry gm = geometry(p);
   const int mc = max_chunks_bound(total, B);
   size_t s = kWsAlign;                                                              // reserved
-  s += round_up((size_t)B * p->num_kv_heads * sizeof(int), kWsAlign);               // counters
-  s += round_up((size_t)B * p->num_kv_heads * gm.Rq * sizeof(float), kWsAlign);     // bias
   s += round_up((size_t)p->num_kv_heads * mc * gm.Rq * sizeof(float), kWsAlign);    // part_m
   s += round_up((size_t)p->num_kv_heads * mc * gm.Rq * sizeof(double), kWsAlign);   // part_l
   return s;
@@ -661,13 +662,10 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
   const int Hkv = p->num_kv_heads, d = p->head_dim;
   WsCursor wc{static_cast<char*>(ws), ws_bytes};
   wc.take<char>(kWsAlign);
-  int* counters = wc.take<int>((size_t)B * Hkv);
-  float* bias = wc.take<float>((size_t)B * Hkv * gm.Rq);
   const int mc = max_chunks_bound(total, B);
   float* part_m = wc.take<float>((size_t)Hkv * mc * gm.Rq);
   double* part_l = wc.take<double>((size_t)Hkv * mc * gm.Rq);
   if (!wc.ok) return fail(KVC_ERR_WORKSPACE, "score workspace too small");
-  KVC_CUDA_TRY(cudaMemsetAsync(counters, 0, (size_t)B * Hkv * sizeof(int), st));
 
   auto encode = get_encode_fn();
   if (!encode) return fail(KVC_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
@@ -717,8 +715,6 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
   a.c = (float)((double)p->scale * kLog2e);
   a.part_m = part_m;
   a.part_l = part_l;
-  a.bias = bias;
-  a.counters = counters;
   a.scores = scores;
   a.accum = accum;
   a.total = total;

@@ -16,6 +16,9 @@
 // threshold go to the lowest positions.
 #include <cooperative_groups.h>
 
+#include <algorithm>
+#include <mutex>
+
 #include "common.cuh"
 
 namespace cg = cooperative_groups;
@@ -26,7 +29,6 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCS = 8;          // CTAs per ranking row (portable cluster size)
-constexpr int kStage = 4096;    // pooled outputs per staging round
 constexpr int kMaxHalf = 32;    // pool_kernel <= 65
 constexpr int kBins = 2048;     // radix bins of the first two passes
 constexpr int kPerTile = 4;     // elements per thread in the compaction tiles
@@ -124,22 +126,39 @@ struct SelArgs {
   int32_t* idx;
   int64_t idx_row_stride;  // per output row (single); varlen uses k
   int32_t* counts;         // varlen only, may be nullptr
-  float* vals;             // pooled prefix scores
+  float* vals_g;           // pooled prefix scores in global memory, or nullptr
   int64_t vals_stride;     // per output row
-  bool vals_packed;        // vals indexed by packed token offset (varlen / workspace)
+  bool vals_packed;        // vals_g indexed by packed token offset (varlen / workspace)
+  bool smem_vals;          // keep this CTA's pooled segment in shared memory
+  int64_t seg_cap;         // smem mode: longest segment the dynamic smem holds
   int out_rows;
   int32_t* err;
 };
 
 struct SelShared {
   RadixShared rx;
-  float stage[kStage + 2 * kMaxHalf];
   uint32_t cnt_gt, cnt_eq;  // this CTA's counts for the output phase
 };
+
+// Warp-aggregated histogram increment: lanes with the same bin add once.
+// Every lane of the warp must call it (inactive lanes with active = false).
+__device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool active) {
+  const unsigned mask = __ballot_sync(0xffffffffu, active);
+  if (!active) return;
+  const unsigned peers = __match_any_sync(mask, bin);
+  if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+}
+
+// Dynamic shared memory of the selection kernel: the staged row sums of the
+// segment plus halo, and the pooled values of the segment (smem mode).
+__host__ __device__ inline size_t sel_dyn_smem(int64_t seg, int half, bool smem_vals) {
+  return smem_vals ? (size_t)(2 * seg + 2 * half + 8) * sizeof(float) : 0;
+}
 
 __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kThreads, 1)
 select_kernel(const SelArgs a) {
   __shared__ SelShared sh;
+  extern __shared__ float dyn[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
   const int o = blockIdx.y;
@@ -152,6 +171,8 @@ select_kernel(const SelArgs a) {
     start = a.cu[b];
     len = (int64_t)a.cu[b + 1] - start;
     bad = (start < 0 || len < a.w);
+    // a sequence longer than the max_seqlen the launch was sized for
+    if (!bad && a.smem_vals && (len - a.w + kCS - 1) / kCS > a.seg_cap) bad = true;
   }
   const int64_t orow = varlen ? ((int64_t)b * a.out_rows + o) : o;
   int32_t* out = a.idx + orow * (varlen ? a.k : a.idx_row_stride);
@@ -181,51 +202,87 @@ select_kernel(const SelArgs a) {
     for (int64_t t = (int64_t)crank * kThreads + threadIdx.x; t < a.w; t += (int64_t)kCS * kThreads)
       out[kk + t] = (int32_t)(L + t);
   }
+  const bool need_rank = (a.k < len) && kk > 0;
+  if (!need_rank && a.vals_g == nullptr) return;  // nothing to rank, nothing to report
 
-  // ---- segment of this CTA and the pooled scores --------------------------
+  // ---- segment of this CTA: row sums (+halo), then pooled values -------------
   const int64_t seg = (L + kCS - 1) / kCS;
   const int64_t s0 = (int64_t)crank * seg < L ? (int64_t)crank * seg : L;
   const int64_t s1 = s0 + seg < L ? s0 + seg : L;
+  const int nseg = (int)(s1 - s0);
   const int half = a.pool / 2;
   const float pool_div = (float)a.pool;
   const float* rows0 = a.scores + (int64_t)o * a.row_group * a.row_stride + start;
-  float* vals = a.vals + (int64_t)o * a.vals_stride + (a.vals_packed ? start : 0);
-  const bool need_rank = (a.k < len) && kk > 0;
+  float* gvals = a.vals_g ? a.vals_g + (int64_t)o * a.vals_stride + (a.vals_packed ? start : 0) : nullptr;
+  // pooled values of the segment, indexed 0..nseg-1 (shared or global memory)
+  float* v = a.smem_vals ? dyn + (nseg + 2 * half + 8) : gvals + s0;
 
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[0][i] = 0;
   __syncthreads();
 
-  for (int64_t c0 = s0; c0 < s1; c0 += kStage) {
-    const int64_t c1 = c0 + kStage < s1 ? c0 + kStage : s1;
-    const int64_t lo = c0 - half;
-    const int span = (int)(c1 - c0) + 2 * half;
-    for (int t = threadIdx.x; t < span; t += kThreads) {
-      const int64_t u = lo + t;
-      float s = 0.f;
-      if (u >= 0 && u < L) {
-        for (int r = 0; r < a.row_group; ++r) s += rows0[(int64_t)r * a.row_stride + u];
+  constexpr int kU = 4;
+  if (a.smem_vals) {
+    float* stage = dyn;  // row sums over [s0 - half, s1 + half)
+    const int span = nseg + 2 * half;
+    for (int t0 = 0; t0 < span; t0 += kThreads * kU) {
+      float acc[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) acc[u] = 0.f;
+      for (int r = 0; r < a.row_group; ++r) {
+        const float* row = rows0 + (int64_t)r * a.row_stride;
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+          const int t = t0 + u * kThreads + threadIdx.x;
+          const int64_t pos = s0 - half + t;
+          if (t < span && pos >= 0 && pos < L) acc[u] += row[pos];
+        }
       }
-      sh.stage[t] = s;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int t = t0 + u * kThreads + threadIdx.x;
+        if (t < span) stage[t] = acc[u];
+      }
     }
     __syncthreads();
-    for (int t = threadIdx.x; t < (int)(c1 - c0); t += kThreads) {
-      float v;
-      if (a.pool == 1) {
-        v = sh.stage[t];
-      } else {
-        float s = 0.f;
-        for (int q = 0; q <= 2 * half; ++q) s += sh.stage[t + q];
-        v = s / pool_div;
+    for (int base = 0; base < nseg; base += kThreads) {
+      const int t = base + threadIdx.x;
+      const bool in = t < nseg;
+      float val = 0.f;
+      if (in) {
+        if (a.pool == 1) {
+          val = stage[t];
+        } else {
+          float sum = 0.f;
+          for (int q = 0; q <= 2 * half; ++q) sum += stage[t + q];
+          val = sum / pool_div;
+        }
+        v[t] = val;
+        if (gvals) gvals[s0 + t] = val;
       }
-      vals[c0 + t] = v;  // pooled scores are always materialised
-      if (need_rank) atomicAdd(&sh.rx.hist[0][order_key(v) >> 21], 1);
+      if (need_rank) hist_add(sh.rx.hist[0], order_key(val) >> 21, in);
     }
-    __syncthreads();
+  } else {
+    // long rows: pooled values go straight to global memory (L2-resident)
+    for (int base = 0; base < nseg; base += kThreads) {
+      const int t = base + threadIdx.x;
+      const bool in = t < nseg;
+      float val = 0.f;
+      if (in) {
+        float sum = 0.f;
+        for (int q = -half; q <= half; ++q) {
+          const int64_t pos = s0 + t + q;
+          if (pos < 0 || pos >= L) continue;
+          float rs = 0.f;
+          for (int r = 0; r < a.row_group; ++r) rs += rows0[(int64_t)r * a.row_stride + pos];
+          sum += rs;
+        }
+        val = (a.pool == 1) ? sum : sum / pool_div;
+        v[t] = val;
+      }
+      if (need_rank) hist_add(sh.rx.hist[0], order_key(val) >> 21, in);
+    }
   }
-  if (!need_rank) {
-    cluster.sync();  // keep every CTA resident until the cluster is done
-    return;
-  }
+  if (!need_rank) return;
 
   // ---- radix passes ---------------------------------------------------------
   cluster.sync();
@@ -235,9 +292,10 @@ select_kernel(const SelArgs a) {
 
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[1][i] = 0;
   __syncthreads();
-  for (int64_t j = s0 + threadIdx.x; j < s1; j += kThreads) {
-    const uint32_t key = order_key(vals[j]);
-    if ((key >> 21) == b1) atomicAdd(&sh.rx.hist[1][(key >> 10) & 2047u], 1);
+  for (int base = 0; base < nseg; base += kThreads) {
+    const int t = base + threadIdx.x;
+    const uint32_t key = t < nseg ? order_key(v[t]) : 0u;
+    hist_add(sh.rx.hist[1], (key >> 10) & 2047u, t < nseg && (key >> 21) == b1);
   }
   cluster.sync();
   cluster_find_bucket(cluster, sh.rx, 1, kBins, want);
@@ -247,9 +305,10 @@ select_kernel(const SelArgs a) {
 
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[0][i] = 0;
   __syncthreads();
-  for (int64_t j = s0 + threadIdx.x; j < s1; j += kThreads) {
-    const uint32_t key = order_key(vals[j]);
-    if ((key >> 10) == pre2) atomicAdd(&sh.rx.hist[0][key & 1023u], 1);
+  for (int base = 0; base < nseg; base += kThreads) {
+    const int t = base + threadIdx.x;
+    const uint32_t key = t < nseg ? order_key(v[t]) : 0u;
+    hist_add(sh.rx.hist[0], key & 1023u, t < nseg && (key >> 10) == pre2);
   }
   cluster.sync();
   cluster_find_bucket(cluster, sh.rx, 0, 1024, want);
@@ -258,8 +317,8 @@ select_kernel(const SelArgs a) {
 
   // ---- counts per CTA, then cluster prefix ---------------------------------
   uint32_t gt = 0, eq = 0;
-  for (int64_t j = s0 + threadIdx.x; j < s1; j += kThreads) {
-    const uint32_t key = order_key(vals[j]);
+  for (int t = threadIdx.x; t < nseg; t += kThreads) {
+    const uint32_t key = order_key(v[t]);
     gt += key > T;
     eq += key == T;
   }
@@ -279,15 +338,15 @@ select_kernel(const SelArgs a) {
   }
 
   // ---- order-preserving compaction -----------------------------------------
-  for (int64_t t0 = s0; t0 < s1; t0 += (int64_t)kThreads * kPerTile) {
-    const int64_t j0 = t0 + (int64_t)threadIdx.x * kPerTile;
+  for (int t0 = 0; t0 < nseg; t0 += kThreads * kPerTile) {
+    const int tb = t0 + threadIdx.x * kPerTile;
     uint32_t keys[kPerTile];
     uint32_t my_gt = 0, my_eq = 0;
 #pragma unroll
     for (int q = 0; q < kPerTile; ++q) {
-      const int64_t j = j0 + q;
-      keys[q] = (j < s1) ? order_key(vals[j]) : 0u;
-      if (j < s1) {
+      const int t = tb + q;
+      keys[q] = (t < nseg) ? order_key(v[t]) : 0u;
+      if (t < nseg) {
         my_gt += keys[q] > T;
         my_eq += keys[q] == T;
       }
@@ -298,13 +357,14 @@ select_kernel(const SelArgs a) {
     const uint32_t quota = eq_seen < need_eq ? need_eq - eq_seen : 0u;
 #pragma unroll
     for (int q = 0; q < kPerTile; ++q) {
-      const int64_t j = j0 + q;
-      if (j >= s1) break;
+      const int t = tb + q;
+      if (t >= nseg) break;
+      const int32_t j = (int32_t)(s0 + t);
       if (keys[q] > T) {
-        out[out_base + g_before + (e_before < quota ? e_before : quota)] = (int32_t)j;
+        out[out_base + g_before + (e_before < quota ? e_before : quota)] = j;
         ++g_before;
       } else if (keys[q] == T) {
-        if (e_before < quota) out[out_base + g_before + e_before] = (int32_t)j;
+        if (e_before < quota) out[out_base + g_before + e_before] = j;
         ++e_before;
       }
     }
@@ -437,6 +497,29 @@ stats_kernel(const StatArgs a) {
   cluster.sync();
 }
 
+constexpr size_t kSelDynMax = 180 * 1024;  // dynamic smem budget for pooled segments
+
+kvc_status launch_select(const SelArgs& a, int out_rows, int batch, int64_t seg, cudaStream_t st) {
+  const size_t dyn = sel_dyn_smem(seg, a.pool / 2, a.smem_vals);
+  static std::mutex mu;
+  static uint64_t done = 0;
+  int dev = 0;
+  KVC_CUDA_TRY(cudaGetDevice(&dev));
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 64 || !((done >> dev) & 1)) {
+      KVC_CUDA_TRY(cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        (int)kSelDynMax));
+      if (dev < 64) done |= (uint64_t)1 << dev;
+    }
+  }
+  dim3 grid(kCS, out_rows, batch);
+  select_kernel<<<grid, kThreads, dyn, st>>>(a);
+  count_launch();
+  KVC_CUDA_TRY(cudaGetLastError());
+  return KVC_OK;
+}
+
 kvc_status check_select_common(const float* scores, int32_t rows, int64_t row_stride,
                                int32_t row_group, int32_t w, int32_t pool, int64_t k,
                                const int32_t* idx) {
@@ -491,24 +574,25 @@ extern "C" kvc_status kvc_select_topk(const float* scores, int32_t rows, int64_t
   a.counts = nullptr;
   a.out_rows = out_rows;
   a.err = nullptr;
+  const int64_t seg = (n - window + kCS - 1) / kCS;
+  a.smem_vals = sel_dyn_smem(seg, pool_kernel / 2, true) <= kSelDynMax;
+  a.seg_cap = seg;
   if (pooled) {
-    a.vals = pooled;
+    a.vals_g = pooled;
     a.vals_stride = n - window;
     a.vals_packed = false;
+  } else if (a.smem_vals) {
+    a.vals_g = nullptr;
   } else {
     size_t need = 0;
     kvc_select_workspace_size(out_rows, 1, n, &need);
     if (!ws || ws_bytes < need || !aligned(ws, kWsAlign))
       return fail(KVC_ERR_WORKSPACE, "select workspace missing, too small or not 256-B aligned");
-    a.vals = static_cast<float*>(ws);
+    a.vals_g = static_cast<float*>(ws);
     a.vals_stride = n;
     a.vals_packed = true;
   }
-  dim3 grid(kCS, out_rows, 1);
-  select_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(a);
-  count_launch();
-  KVC_CUDA_TRY(cudaGetLastError());
-  return KVC_OK;
+  return launch_select(a, out_rows, 1, seg, (cudaStream_t)stream);
 }
 
 extern "C" kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, int64_t row_stride,
@@ -527,7 +611,9 @@ extern "C" kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, 
   const int out_rows = rows / row_group;
   size_t need = 0;
   kvc_select_workspace_size(out_rows, batch, total, &need);
-  if (!ws || ws_bytes < need || !aligned(ws, kWsAlign))
+  const int64_t seg_max = (std::max<int64_t>(max_seqlen, window) - window + kCS - 1) / kCS;
+  if (sel_dyn_smem(seg_max, pool_kernel / 2, true) > kSelDynMax &&
+      (!ws || ws_bytes < need || !aligned(ws, kWsAlign)))
     return fail(KVC_ERR_WORKSPACE, "select workspace missing, too small or not 256-B aligned");
   SelArgs a{};
   a.scores = scores;
@@ -541,16 +627,16 @@ extern "C" kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, 
   a.idx = idx;
   a.idx_row_stride = k;
   a.counts = counts;
-  a.vals = static_cast<float*>(ws);
+  a.vals_g = nullptr;
   a.vals_stride = total;
   a.vals_packed = true;
   a.out_rows = out_rows;
   a.err = dev_err;
-  dim3 grid(kCS, out_rows, batch);
-  select_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(a);
-  count_launch();
-  KVC_CUDA_TRY(cudaGetLastError());
-  return KVC_OK;
+  const int64_t seg = (std::max<int64_t>(max_seqlen, window) - window + kCS - 1) / kCS;
+  a.smem_vals = sel_dyn_smem(seg, pool_kernel / 2, true) <= kSelDynMax;
+  a.seg_cap = seg;
+  if (!a.smem_vals) a.vals_g = static_cast<float*>(ws);
+  return launch_select(a, out_rows, batch, seg, (cudaStream_t)stream);
 }
 
 extern "C" kvc_status kvc_stats_workspace_size(int32_t rows, int64_t n, size_t* bytes) {
