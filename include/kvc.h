@@ -141,6 +141,37 @@ kvc_status kvc_score_varlen(const uint16_t* q_win, int64_t q_stride_b, int64_t q
                             float* scores, float* tsp, float* accum, void* ws, size_t ws_bytes,
                             int32_t* dev_err, void* stream);
 
+/*
+ * kvc_score for callers that cannot allocate.  The paper has no counterpart:
+ * this is a deployment variant of kvc_score, same arguments minus the
+ * workspace, same results.
+ *
+ * Some callers cannot hand the library a workspace: an operator running
+ * inside another runtime's plugin interface that offers no scratch buffer,
+ * or a serving loop that must not call cudaMalloc once it is running
+ * (cudaMalloc can synchronise the device and stall every other stream).
+ * This entry point takes its scratch from a static device array of
+ * KVC_NOALLOC_SCRATCH_BYTES inside the library instead, and itself calls no
+ * cudaMalloc, cudaFree or other allocating routine.  The array exists on
+ * every GPU that loads the library and is held until the process exits.
+ *  - Size limit: a call whose scratch need (kvc_score_workspace_size(p, 1, n))
+ *    exceeds KVC_NOALLOC_SCRATCH_BYTES is rejected with KVC_ERR_WORKSPACE and
+ *    launches nothing (8 KV heads x 128 window rows fit up to ~330K tokens).
+ *  - First call on a device: it looks up (once per device, with that device
+ *    current) the device address of the array.  Make the first call on each
+ *    device before any stream capture.
+ *  - Sharing: every call on a device uses the same array, which keeps the
+ *    previous call's contents (nothing in it needs to start at zero: each
+ *    call writes every entry it later reads).  Calls that may overlap on the
+ *    GPU -- on different streams, or from different threads -- race on the
+ *    array and give wrong results; serialise them (one stream).
+ */
+#define KVC_NOALLOC_SCRATCH_BYTES (8u << 20)
+kvc_status kvc_score_noalloc(const uint16_t* q_win, int64_t q_stride_w, int64_t q_stride_h,
+                             const uint16_t* k, int64_t k_stride_n, int64_t k_stride_h, int64_t n,
+                             const kvc_score_params* p, float* scores, float* tsp, float* accum,
+                             int32_t* dev_err, void* stream);
+
 /* Selection -------------------------------------------------------------- */
 
 /* Workspace bytes for kvc_select_topk(_varlen) with `out_rows` ranking rows. */

@@ -53,6 +53,7 @@ _SIGS = {
     "kvc_score": ([_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _SZ, _P, _P], _I32),
     "kvc_score_varlen": ([_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I32, _I64, _I64, _P, _P, _P, _P,
                           _P, _SZ, _P, _P], _I32),
+    "kvc_score_noalloc": ([_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _I32),
     "kvc_select_workspace_size": ([_I32, _I32, _I64, _P], _I32),
     "kvc_select_topk": ([_P, _I32, _I64, _I32, _I64, _I32, _I32, _I64, _P, _I64, _P, _P, _SZ, _P], _I32),
     "kvc_select_topk_varlen": ([_P, _I32, _I64, _I32, _P, _I32, _I64, _I64, _I32, _I32, _I64, _P, _P, _P,
@@ -168,6 +169,27 @@ def kvc_score(q_win: torch.Tensor, k: torch.Tensor, scale: Optional[float] = Non
     _check(lib().kvc_score(_ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k), k.stride(0), k.stride(1),
                            n, ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum), _ptr(ws),
                            ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)), "kvc_score")
+    return scores
+
+
+def kvc_score_noalloc(q_win: torch.Tensor, k: torch.Tensor, scale: Optional[float] = None,
+                      scores: Optional[torch.Tensor] = None, tsp: Optional[torch.Tensor] = None,
+                      accum: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                      stream=None) -> torch.Tensor:
+    """kvc_score without a caller workspace: the library's static device
+    scratch is used instead (for callers that cannot allocate; calls that
+    overlap on the GPU race on that scratch).  Pass `scores` to avoid even the
+    output allocation here."""
+    _bf16(q_win, "q_win")
+    _bf16(k, "k")
+    w, H, d = q_win.shape
+    n, Hkv, _ = k.shape
+    p = score_params(H, Hkv, d, w, scale)
+    if scores is None:
+        scores = torch.empty((Hkv, n), dtype=torch.float32, device=k.device)
+    _check(lib().kvc_score_noalloc(_ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k), k.stride(0),
+                                   k.stride(1), n, ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum),
+                                   _ptr(dev_err), _stream(stream)), "kvc_score_noalloc")
     return scores
 
 

@@ -774,3 +774,64 @@ extern "C" kvc_status kvc_score_varlen(const uint16_t* q_win, int64_t q_stride_b
   return score_impl(q_win, q_stride_b, q_stride_w, q_stride_h, k, k_stride_n, k_stride_h, cu_seqlens, batch,
                     total, p, scores, tsp, accum, ws, ws_bytes, dev_err, (cudaStream_t)stream);
 }
+
+// --------------------------------------------------------------------------
+// Scoring with library-owned scratch, for callers that cannot allocate.
+// --------------------------------------------------------------------------
+// Some callers have no way to hand the library a workspace: an operator
+// running inside another runtime's plugin interface that offers no scratch
+// buffer, or a serving loop that must never call cudaMalloc once it is up
+// (cudaMalloc can synchronise the device and stall every other stream).
+// For them the chunk partials live in this file-scope device array instead
+// of a caller buffer.  It is allocated when the library's module is loaded
+// and every GPU that loads the library keeps its copy until the process
+// exits.
+namespace kvc {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[KVC_NOALLOC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device.  Host code may
+// not use the symbol itself (it names a host-side shadow, not device
+// memory), so the address is looked up once per device with that device
+// current and cached.
+kvc_status noalloc_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static void* cache[64] = {};
+  int dev = 0;
+  KVC_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(KVC_ERR_UNSUPPORTED, "device ordinal >= 64");
+  std::lock_guard<std::mutex> lk(mu);
+  if (cache[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+    cache[dev] = p;
+  }
+  *out = cache[dev];
+  return KVC_OK;
+}
+
+}  // namespace
+}  // namespace kvc
+
+extern "C" kvc_status kvc_score_noalloc(const uint16_t* q_win, int64_t q_stride_w, int64_t q_stride_h,
+                                        const uint16_t* k, int64_t k_stride_n, int64_t k_stride_h, int64_t n,
+                                        const kvc_score_params* p, float* scores, float* tsp, float* accum,
+                                        int32_t* dev_err, void* stream) {
+  clear_error();
+  kvc_status s = check_params(p);
+  if (s != KVC_OK) return s;
+  KVC_CHECK_ARG(n >= p->window && n < (int64_t(1) << 31), "need window <= n < 2^31");
+  const size_t need = score_ws_bytes(p, 1, n);
+  if (need > (size_t)KVC_NOALLOC_SCRATCH_BYTES)
+    return fail(KVC_ERR_WORKSPACE, "kvc_score_noalloc needs " + std::to_string(need) +
+                                       " bytes of scratch; its static scratch holds " +
+                                       std::to_string((size_t)KVC_NOALLOC_SCRATCH_BYTES) +
+                                       " (use kvc_score with a workspace)");
+  void* ws = nullptr;
+  s = noalloc_scratch_ptr(&ws);
+  if (s != KVC_OK) return s;
+  return score_impl(q_win, 0, q_stride_w, q_stride_h, k, k_stride_n, k_stride_h, nullptr, 1, n, p, scores, tsp,
+                    accum, ws, (size_t)KVC_NOALLOC_SCRATCH_BYTES, dev_err, (cudaStream_t)stream);
+}
