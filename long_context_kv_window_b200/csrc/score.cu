@@ -20,11 +20,14 @@
 //          then each epilogue thread owns one key and sums 2^(s*log2e - b_r)
 //          over the rows -- a thread-local reduction.
 // Both passes stream the same K tiles (TMA, 128-byte swizzle) into a
-// multi-stage shared-memory ring; heads are processed in groups whose K fits
-// in L2, so pass 2 re-reads K from L2 rather than HBM.
+// multi-stage shared-memory ring.  One launch per pass covers every KV head,
+// so the CTAs of a key range read whole token rows of K together (HBM
+// streams best that way); pass 2 walks each chunk backwards, starting on the
+// tiles pass 1 read last, which are still in L2.
 //
 // Warp roles per CTA: warp 0 issues TMA, warp 1 allocates TMEM and issues
-// MMAs, warps 2..5 drain TMEM (epilogue).  Every wait is bounded; on a
+// MMAs, warps 2..9 drain TMEM (epilogue; two warps per TMEM lane quarter,
+// taking alternate tiles).  Every wait is bounded; on a
 // timeout the CTA records KVC_DEV_ERR_TIMEOUT, lets in-flight copies and MMAs
 // land, frees TMEM and exits.
 #include <cuda.h>
@@ -33,17 +36,22 @@
 #include <algorithm>
 #include <mutex>
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "tc.cuh"
 
 namespace kvc {
 namespace {
 
-constexpr int kTile = 128;  // keys per tile
-constexpr int kStages = 4;
-constexpr int kEpiWarps = 4;
+constexpr int kTile = 128;       // keys per tile
+constexpr int kMaxStages = 8;    // TMA ring depth bound (the host picks what fits)
+constexpr int kMaxBufs = 4;      // TMEM accumulator buffers
+constexpr int kEpiWarps = 8;     // two per TMEM lane quarter; the halves take alternate tiles
 constexpr int kThreadsScore = 64 + 32 * kEpiWarps;
+constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kMinChunkTiles = 4;
+constexpr int kBarEpi = 1;       // named barrier of all epilogue warps
 constexpr double kLog2e = 1.4426950408889634;
 
 struct ScoreArgs {
@@ -54,15 +62,18 @@ struct ScoreArgs {
   int B;
   int Hkv, G, w, R, Rq, Rn;  // rows per KV head, rows in smem, MMA N (pass 2)
   int nb1;                   // 128-row blocks in pass 1
-  int acc_stride1;           // pass 1: TMEM columns between the two accumulator buffers
-  int acc_stride;            // pass 2: TMEM columns between the two accumulator buffers
-  uint32_t tmem_cols;        // TMEM columns allocated
+  int acc_stride;            // TMEM columns between accumulator buffers (this pass)
+  int nbuf;                  // TMEM accumulator buffers (this pass): 2 or 4
+  int stages;                // TMA ring depth
+  int fold;                  // pass 2: the row bias rides in one extra MMA K-step
+  uint32_t tmem_cols;        // TMEM columns allocated (this pass)
   int g0;                    // first KV head of this launch
   int chunk_keys;
   int max_chunks;            // partial slots per KV head
   float c;                   // scale * log2(e)
-  float* part_m;             // [Hkv][max_chunks][Rq]
+  float* part_m;             // [Hkv][max_chunks][Rq]: one row of partials per chunk
   double* part_l;            // [Hkv][max_chunks][Rq]
+  uint2* qsplit;             // [B][Hkv][Rq]: -bias/c as three bf16 parts (words w0, w1)
   float* scores;             // [Hkv][total]
   float* accum;              // [Hkv][total] or nullptr
   int64_t total;
@@ -82,7 +93,19 @@ struct Work {
 
 // Map a linear chunk index onto (sequence, chunk).  Malformed sequences
 // (non-monotone cu_seqlens or shorter than the window) own one chunk each.
-__device__ __forceinline__ Work map_work(const ScoreArgs& a, int linear) {
+// reverse: CTA 0 takes the last chunk (pass 2 walks the keys backwards, so
+// it starts on what pass 1 left in L2).
+__device__ __forceinline__ Work map_work(const ScoreArgs& a, int linear, bool reverse) {
+  if (reverse) {
+    int total = 0;
+    for (int b = 0; b < a.B; ++b) {
+      const SeqSpan s = seq_span(a.cu, b, a.n);
+      const bool bad = s.start < 0 || s.len < a.w || s.start + s.len > a.total;
+      total += bad ? 1 : (int)((s.len + a.chunk_keys - 1) / a.chunk_keys);
+    }
+    if (linear >= total) return Work{0, 0, 0, 0, 0, 0, false, false};
+    linear = total - 1 - linear;
+  }
   int base = 0;
   for (int b = 0; b < a.B; ++b) {
     const SeqSpan s = seq_span(a.cu, b, a.n);
@@ -94,24 +117,55 @@ __device__ __forceinline__ Work map_work(const ScoreArgs& a, int linear) {
   return Work{0, 0, 0, 0, 0, 0, false, false};
 }
 
+struct Barriers {
+  uint64_t full[kMaxStages];
+  uint64_t empty[kMaxStages];
+  uint64_t tfull[kMaxBufs];
+  uint64_t tempty[kMaxBufs];
+  uint64_t bias_ready;  // pass 2: the epilogue wrote the bias block
+  uint32_t tmem_base;
+  int abort;
+};
+
+// Shared memory: [Q rows, swizzled][pass 2: ones | bias block][K stage ring]
+// [barriers | bias | exchange].  The pass-2 blocks hold one extra K-step of
+// the MMA: a [128 keys x 16] block of (1, 1, 1, 0, ...) and a [Rq x 16] block
+// of each row's (h1, h2, h3, 0, ...) with h1 + h2 + h3 = -bias / c (three
+// bf16 parts of an fp32-accurate value), laid out like the K tiles.
 template <int D>
 struct Smem {
-  static constexpr int kChunks = D / 64;            // 64-element (128 B) swizzle columns
+  static constexpr int kChunks = D / 64;  // 64-element (128 B) swizzle columns
   static constexpr int kStageBytes = kChunks * kTile * 128;
+  static constexpr size_t kOnesBytes = (size_t)kTile * 128;
+  static constexpr size_t kTail = 512 /*barriers*/ + 256 * 4 /*bias*/ + 256 * 4 + 256 * 8 /*exchange*/;
   __host__ __device__ static size_t q_bytes(int Rq) { return (size_t)kChunks * Rq * 128; }
-  __host__ __device__ static size_t total(int Rq) {
-    return 1024 /*alignment slack*/ + q_bytes(Rq) + (size_t)kStages * kStageBytes + 256 /*barriers*/ +
-           (size_t)Rq * sizeof(float) /*bias*/ + 64;
+  __host__ __device__ static size_t fold_bytes(int Rq, int fold) { return fold ? kOnesBytes + (size_t)Rq * 128 : 0; }
+  __host__ __device__ static size_t total(int Rq, int stages, int fold) {
+    return 1024 /*alignment slack*/ + q_bytes(Rq) + fold_bytes(Rq, fold) + (size_t)stages * kStageBytes + kTail;
   }
 };
 
-struct Barriers {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t tfull[2];
-  uint64_t tempty[2];
-  uint32_t tmem_base;
-  int abort;
+template <int D>
+struct SmemPtrs {
+  uint8_t* qs;
+  uint8_t* ones;  // pass 2 only
+  uint8_t* qb;    // pass 2 only
+  uint8_t* kst;
+  Barriers* bars;
+  float* bias;   // [256]
+  float* ex_m;   // [256]
+  double* ex_l;  // [256]
+  __device__ SmemPtrs(uint8_t* raw, const ScoreArgs& a) {
+    uint8_t* s = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
+    qs = s;
+    ones = qs + Smem<D>::q_bytes(a.Rq);
+    qb = ones + Smem<D>::kOnesBytes;
+    kst = qs + Smem<D>::q_bytes(a.Rq) + Smem<D>::fold_bytes(a.Rq, a.fold);
+    bars = reinterpret_cast<Barriers*>(kst + (size_t)a.stages * Smem<D>::kStageBytes);
+    bias = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);
+    ex_m = bias + 256;
+    ex_l = reinterpret_cast<double*>(ex_m + 256);
+  }
 };
 
 // Q rows of KV head g into the K-major 128-byte swizzled layout; rows past R
@@ -136,32 +190,160 @@ __device__ __forceinline__ void load_q_swizzled(const ScoreArgs& a, int b, int g
   tc::fence_proxy_async_smem();
 }
 
+// Barrier init (one thread) for the stage ring and the TMEM buffers.  Buffer
+// b is drained by the four epilogue warps of half b % 2.
+__device__ __forceinline__ void init_barriers(Barriers* bars, int stages, int nbuf) {
+  for (int s = 0; s < stages; ++s) {
+    tc::mbar_init(&bars->full[s], 1);
+    tc::mbar_init(&bars->empty[s], 1);
+  }
+  for (int s = 0; s < nbuf; ++s) {
+    tc::mbar_init(&bars->tfull[s], 1);
+    tc::mbar_init(&bars->tempty[s], kEpiWarps / 2);
+  }
+  tc::mbar_init(&bars->bias_ready, kEpiThreads);
+  bars->abort = 0;
+  tc::fence_mbar_init();
+}
+
 // Producer: stream the chunk's K tiles of head g into the stage ring.
 template <int D>
-__device__ __forceinline__ void produce(const void* kmap, Barriers* bars, uint8_t* kst, int g, int64_t row0,
-                                        int ntiles) {
+__device__ __forceinline__ void produce(const void* kmap, Barriers* bars, uint8_t* kst, int stages, int g,
+                                        int64_t row0, int ntiles, bool reverse) {
   constexpr int kChunks = D / 64;
   constexpr uint32_t kBytes = (uint32_t)Smem<D>::kStageBytes;
   int issued = 0;
   for (int t = 0; t < ntiles; ++t) {
-    const int s = t % kStages;
-    const int u = t / kStages;
+    const int s = t % stages;
+    const int u = t / stages;
     if (u > 0 && !tc::mbar_wait(&bars->empty[s], (u - 1) & 1, &bars->abort)) break;
     tc::mbar_arrive_expect_tx(&bars->full[s], kBytes);
     uint8_t* dst = kst + (size_t)s * Smem<D>::kStageBytes;
 #pragma unroll
     for (int c = 0; c < kChunks; ++c)
-      tc::tma_load_3d(dst + c * kTile * 128, kmap, &bars->full[s], c * 64, g, (int)(row0 + (int64_t)t * kTile));
+      tc::tma_load_3d(dst + c * kTile * 128, kmap, &bars->full[s], c * 64, g,
+                      (int)(row0 + (int64_t)(reverse ? ntiles - 1 - t : t) * kTile));
     issued = t + 1;
   }
   if (bars->abort) {
     // let every copy already issued land before the CTA can exit
-    for (int t = std::max(0, issued - kStages); t < issued; ++t)
-      tc::mbar_drain(&bars->full[t % kStages], (t / kStages) & 1);
+    for (int t = std::max(0, issued - stages); t < issued; ++t)
+      tc::mbar_drain(&bars->full[t % stages], (t / stages) & 1);
   }
 }
 
+// MMA issuer (one thread).  kRowsOnM: pass 1 (A = Q rows, B = K tile);
+// otherwise pass 2 (A = K tile, B = Q rows, N = Rn).
+template <int D, bool kRowsOnM>
+__device__ __forceinline__ void issue_mmas(const ScoreArgs& a, Barriers* bars, uint32_t tmem, uint8_t* qs,
+                                           uint8_t* kst, uint8_t* ones, uint8_t* qb, int ntiles) {
+  constexpr int kChunks = D / 64;
+  const uint32_t idesc = kRowsOnM ? tc::idesc_bf16_f32(128, kTile) : tc::idesc_bf16_f32(128, a.Rn);
+  const uint32_t qbase = tc::smem_u32(qs), kbase = tc::smem_u32(kst);
+  const uint64_t ones_desc = tc::desc_k_sw128(tc::smem_u32(ones));
+  const uint64_t qb_desc = tc::desc_k_sw128(tc::smem_u32(qb));
+  int issued = 0;
+  const bool go = kRowsOnM || tc::mbar_wait(&bars->bias_ready, 0, &bars->abort);
+  for (int t = 0; go && t < ntiles; ++t) {
+    const int s = t % a.stages;
+    const int buf = t % a.nbuf, ub = t / a.nbuf;
+    if (!tc::mbar_wait(&bars->full[s], (t / a.stages) & 1, &bars->abort)) break;
+    if (ub > 0 && !tc::mbar_wait(&bars->tempty[buf], (ub - 1) & 1, &bars->abort)) break;
+    tc::tc_fence_after();
+    const uint32_t kst_s = kbase + (uint32_t)(s * Smem<D>::kStageBytes);
+    const int nblk = kRowsOnM ? a.nb1 : 1;
+    for (int mb = 0; mb < nblk; ++mb) {
+      const uint32_t d = tmem + (uint32_t)(buf * a.acc_stride + mb * kTile);
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          const uint32_t qa = qbase + (uint32_t)(c * a.Rq * 128 + mb * kTile * 128 + ks * 32);
+          const uint32_t ka = kst_s + (uint32_t)(c * kTile * 128 + ks * 32);
+          if (kRowsOnM)
+            tc::mma_bf16(d, tc::desc_k_sw128(qa), tc::desc_k_sw128(ka), idesc, (c | ks) != 0);
+          else
+            tc::mma_bf16(d, tc::desc_k_sw128(ka), tc::desc_k_sw128(qa), idesc, (c | ks) != 0);
+        }
+      // pass 2: + (h1 + h2 + h3) = -bias/c on every (key, row)
+      if (!kRowsOnM) tc::mma_bf16(d, ones_desc, qb_desc, idesc, 1u);
+    }
+    tc::mma_commit(&bars->empty[s]);
+    tc::mma_commit(&bars->tfull[buf]);
+    issued = t + 1;
+  }
+  if (issued > 0)  // the last MMAs landed before TMEM can be freed
+    tc::mbar_drain(&bars->tfull[(issued - 1) % a.nbuf], ((issued - 1) / a.nbuf) & 1);
+}
+
 __device__ __forceinline__ void record_timeout(int32_t* err) { set_dev_err(err, KVC_DEV_ERR_TIMEOUT); }
+
+// Online merge of (m, l) pairs in the log2 domain: l * 2^(m - M) summed.
+__device__ __forceinline__ void merge_ml(float& M, double& L, float m2, double l2) {
+  if (m2 == -INFINITY) return;
+  if (M == -INFINITY) {
+    M = m2;
+    L = l2;
+    return;
+  }
+  const float Mn = fmaxf(M, m2);
+  L = L * (double)exp2f(M - Mn) + l2 * (double)exp2f(m2 - Mn);
+  M = Mn;
+}
+
+
+// Load `ncol` (16, 32, 48 or 64) fp32 columns of this warp's 32 TMEM lanes
+// starting at taddr into x[0..ncol).  Completion: KVC_TMEM_WAIT_LD64(x).
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&x)[64], int ncol) {
+  if (ncol == 64) {
+    KVC_TMEM_LD64(taddr, x);
+  } else if (ncol == 48) {
+    KVC_TMEM_LD32(taddr, x);
+    KVC_TMEM_LD16(taddr + 32, (x + 32));
+  } else if (ncol == 32) {
+    KVC_TMEM_LD32(taddr, x);
+  } else {
+    KVC_TMEM_LD16(taddr, x);
+  }
+}
+
+// sum_e 2^(x[e]*c + off) over 64 values, 8 independent accumulators
+__device__ __forceinline__ float sum_ex2_64(const uint32_t (&x)[64], float c, float off) {
+  float s8[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) s8[u] = 0.f;
+#pragma unroll
+  for (int e = 0; e < 64; ++e) s8[e & 7] += tc::ex2_approx(fmaf(__uint_as_float(x[e]), c, off));
+  return ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+}
+
+__device__ __forceinline__ float max_64(const uint32_t (&x)[64]) {
+  float m8[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) m8[u] = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(x[e]));
+  return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+}
+
+// Pass-1 update of one row with 64 logits (raw dot products) of consecutive
+// keys.  The exponentials use the row's running reference `ref` (log2
+// domain) instead of a fresh per-tile max: only when that would overflow the
+// fp32 partial sum (a logit more than ~94 above the reference) -- and on the
+// first values a row sees, when ref is -inf -- is the exact max taken and the
+// running sum rescaled.
+__device__ __forceinline__ void pass1_group(uint32_t (&x)[64], float c, float& ref, double& l) {
+  float s = sum_ex2_64(x, c, -ref);
+  if (!(s < 0x1p100f)) {  // overflow, or NaN from ref = -inf
+    const float hmax = max_64(x);
+    if (hmax == -INFINITY) return;  // every key masked
+    const float nr = fmaxf(ref, hmax * c);
+    if (ref != -INFINITY) l *= (double)exp2f(ref - nr);
+    ref = nr;
+    s = sum_ex2_64(x, c, -ref);
+  }
+  l += (double)s;
+}
 
 // --------------------------------------------------------------------------
 // pass 1: per-row max / sum over a chunk of keys
@@ -169,16 +351,13 @@ __device__ __forceinline__ void record_timeout(int32_t* err) { set_dev_err(err, 
 template <int D>
 __global__ void __launch_bounds__(kThreadsScore, 1)
 score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) {
-  constexpr int kChunks = D / 64;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qs = smem;
-  uint8_t* kst = qs + Smem<D>::q_bytes(a.Rq);
-  Barriers* bars = reinterpret_cast<Barriers*>(kst + (size_t)kStages * Smem<D>::kStageBytes);
+  const SmemPtrs<D> sp(smem_raw, a);
+  Barriers* bars = sp.bars;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = a.g0 + blockIdx.y;
-  const Work wk = map_work(a, blockIdx.x);
+  const Work wk = map_work(a, blockIdx.x, false);
   if (!wk.valid) return;
   if (wk.bad) {
     if (threadIdx.x == 0 && blockIdx.y == 0) set_dev_err(a.err, KVC_DEV_ERR_SEQLENS);
@@ -188,130 +367,103 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   const int64_t k1 = std::min<int64_t>(wk.len, k0 + a.chunk_keys);
   const int ntiles = (int)((k1 - k0 + kTile - 1) / kTile);
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&bars->full[s], 1);
-      tc::mbar_init(&bars->empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->tfull[s], 1);
-      tc::mbar_init(&bars->tempty[s], kEpiWarps);
-    }
-    bars->abort = 0;
-    tc::fence_mbar_init();
-  }
+  if (threadIdx.x == 0) init_barriers(bars, a.stages, a.nbuf);
   if (warp == 0 && lane == 0) tc::prefetch_tmap(&kmap);
   if (warp == 1) {
     tc::tmem_alloc(&bars->tmem_base, a.tmem_cols);
     tc::tmem_relinquish();
   }
-  load_q_swizzled<D>(a, wk.b, g, qs);
+  load_q_swizzled<D>(a, wk.b, g, sp.qs);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) produce<D>(&kmap, bars, kst, g, wk.start + k0, ntiles);
+    if (lane == 0) produce<D>(&kmap, bars, sp.kst, a.stages, g, wk.start + k0, ntiles, false);
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = tc::idesc_bf16_f32(128, kTile);
-      const uint32_t qbase = tc::smem_u32(qs), kbase = tc::smem_u32(kst);
-      int t = 0;
-      for (; t < ntiles; ++t) {
-        const int s = t % kStages, acc = t & 1;
-        if (!tc::mbar_wait(&bars->full[s], (t / kStages) & 1, &bars->abort)) break;
-        if (t >= 2 && !tc::mbar_wait(&bars->tempty[acc], ((t >> 1) - 1) & 1, &bars->abort)) break;
-        tc::tc_fence_after();
-        for (int mb = 0; mb < a.nb1; ++mb) {
-          const uint32_t d = tmem + (uint32_t)(acc * a.acc_stride1 + mb * kTile);
-#pragma unroll
-          for (int c = 0; c < kChunks; ++c)
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const uint64_t ad = tc::desc_k_sw128(qbase + (uint32_t)(c * a.Rq * 128 + mb * kTile * 128 + ks * 32));
-              const uint64_t bd = tc::desc_k_sw128(kbase + (uint32_t)(s * Smem<D>::kStageBytes + c * kTile * 128 + ks * 32));
-              tc::mma_bf16(d, ad, bd, idesc, (c | ks) != 0);
-            }
-        }
-        tc::mma_commit(&bars->empty[s]);
-        tc::mma_commit(&bars->tfull[acc]);
-      }
-      if (t > 0) tc::mbar_drain(&bars->tfull[(t - 1) & 1], ((t - 1) >> 1) & 1);  // last MMAs landed
-    }
+    if (lane == 0) issue_mmas<D, true>(a, bars, tmem, sp.qs, sp.kst, sp.ones, sp.qb, ntiles);
   } else {
-    // ---- epilogue: one row per thread and row block --------------------------
+    // ---- epilogue: one row per thread and row block; halves take alternate tiles.
+    // A tile is 2 * nb1 groups of 64 columns; the next group's TMEM load is in
+    // flight while the current one is reduced.
+    const int half = (warp - 2) >> 2;
     const int q = warp & 3;
     const int rl = 32 * q + lane;  // lane within a 128-row block
     float m_run[2] = {-INFINITY, -INFINITY};
     double l_run[2] = {0.0, 0.0};
     const int64_t first_window_key = wk.len - a.w;  // earliest window row sees keys <= this
-    for (int t = 0; t < ntiles; ++t) {
-      const int acc = t & 1;
-      if (!tc::mbar_wait(&bars->tfull[acc], (t >> 1) & 1, &bars->abort)) break;
+    const int ng = 2 * a.nb1;
+    for (int t = half; t < ntiles; t += 2) {
+      const int buf = t % a.nbuf;
+      if (!tc::mbar_wait(&bars->tfull[buf], (t / a.nbuf) & 1, &bars->abort)) break;
       tc::tc_fence_after();
       const int64_t j0 = k0 + (int64_t)t * kTile;  // first key of the tile (sequence-local)
-#pragma unroll
-      for (int mb = 0; mb < 2; ++mb) {
-        if (mb >= a.nb1) break;
-        uint32_t x[4][32];
-        const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * a.acc_stride1 + mb * kTile);
-        KVC_TMEM_LD32(base + 0, x[0]);
-        KVC_TMEM_LD32(base + 32, x[1]);
-        KVC_TMEM_LD32(base + 64, x[2]);
-        KVC_TMEM_LD32(base + 96, x[3]);
-        KVC_TMEM_WAIT_LD32(x[0]);
-        KVC_TMEM_TIE32(x[1]);
-        KVC_TMEM_TIE32(x[2]);
-        KVC_TMEM_TIE32(x[3]);
-        if (mb == a.nb1 - 1) {
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&bars->tempty[acc]);
-        }
+      const bool masked = (j0 + kTile - 1 > first_window_key);
+      const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * a.acc_stride);
+      auto release = [&]() {
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->tempty[buf]);
+      };
+      auto proc = [&](int gi, uint32_t(&x)[64]) {
+        const int mb = gi >> 1;
         const int r = mb * kTile + rl;
-        if (r >= a.R) continue;
-        const bool full_tile = (j0 + kTile - 1 <= first_window_key);
-        if (!full_tile) {
-          // keys past this row's own position (or past the sequence) are masked to -inf
-          const int64_t last_key = first_window_key + r / a.G;
+        if (r >= a.R) return;
+        if (masked) {
+          // keys past this row's own position (or past the sequence) get -inf
+          const int64_t lim = first_window_key + r / a.G - (j0 + (gi & 1) * 64);
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (j0 + cc * 32 + e > last_key) x[cc][e] = __float_as_uint(-INFINITY);
+          for (int e = 0; e < 64; ++e)
+            if (e > lim) x[e] = __float_as_uint(-INFINITY);
         }
-        float t4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) t4[e & 3] = fmaxf(t4[e & 3], __uint_as_float(x[cc][e]));
-        const float tmax = fmaxf(fmaxf(t4[0], t4[1]), fmaxf(t4[2], t4[3]));
-        if (tmax == -INFINITY) continue;
-        const float ynew = tmax * a.c;
-        if (ynew > m_run[mb]) {
-          l_run[mb] *= (double)exp2f(m_run[mb] - ynew);
-          m_run[mb] = ynew;
+        if (mb == 0)
+          pass1_group(x, a.c, m_run[0], l_run[0]);
+        else
+          pass1_group(x, a.c, m_run[1], l_run[1]);
+      };
+      uint32_t xa[64], xb[64];
+      KVC_TMEM_LD64(base, xa);
+      KVC_TMEM_WAIT_LD64(xa);
+      if (ng > 1) KVC_TMEM_LD64(base + 64, xb); else release();
+      proc(0, xa);
+      if (ng > 1) {
+        KVC_TMEM_WAIT_LD64(xb);
+        if (ng > 2) KVC_TMEM_LD64(base + kTile, xa); else release();
+        proc(1, xb);
+        if (ng > 2) {
+          KVC_TMEM_WAIT_LD64(xa);
+          KVC_TMEM_LD64(base + kTile + 64, xb);
+          proc(2, xa);
+          KVC_TMEM_WAIT_LD64(xb);
+          release();
+          proc(3, xb);
         }
-        const float mneg = -m_run[mb];
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc)
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s4[e & 3] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e]), a.c, mneg));
-        l_run[mb] += (double)((s4[0] + s4[1]) + (s4[2] + s4[3]));
       }
     }
-    // ---- chunk partials (combined by pass 2) ----------------------------------
-    if (!bars->abort) {
+    // ---- merge the two halves, then one chunk partial per row (combined by pass 2)
+    tc::named_bar_sync(kBarEpi, kEpiThreads);
+    if (half == 1) {
+#pragma unroll
+      for (int mb = 0; mb < 2; ++mb) {
+        if (mb >= a.nb1) break;
+        sp.ex_m[mb * kTile + rl] = m_run[mb];
+        sp.ex_l[mb * kTile + rl] = l_run[mb];
+      }
+    }
+    tc::named_bar_sync(kBarEpi, kEpiThreads);
+    if (half == 0 && !bars->abort) {
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb) {
         if (mb >= a.nb1) break;
         const int r = mb * kTile + rl;
         if (r >= a.R) continue;
+        float M = m_run[mb];
+        double L = l_run[mb];
+        merge_ml(M, L, sp.ex_m[mb * kTile + rl], sp.ex_l[mb * kTile + rl]);
         const size_t slot = ((size_t)g * a.max_chunks + wk.gid) * a.Rq + r;
-        a.part_m[slot] = m_run[mb];
-        a.part_l[slot] = l_run[mb];
+        a.part_m[slot] = M;
+        a.part_l[slot] = L;
       }
     }
   }
@@ -324,22 +476,84 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
 }
 
 // --------------------------------------------------------------------------
+// between the passes: per (sequence, KV head, row) combine the chunk partials
+// into the row's bias b_r = M + log2(sum_c l_c 2^(m_c - M)), M = max_c m_c,
+// and store -b_r / c as three bf16 parts (their fp32 sum is accurate to
+// ~2^-26 relative; each part holds the rounding residual of the previous
+// one).  Pass 2 multiplies them by ones in one extra MMA K-step.
+// --------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) score_combine_kernel(const ScoreArgs a) {
+  const int g = blockIdx.x, b = blockIdx.y;
+  int gid0 = 0, nch = 0;
+  bool bad = false;
+  for (int bb = 0; bb <= b; ++bb) {
+    const SeqSpan sp = seq_span(a.cu, bb, a.n);
+    const bool bd = sp.start < 0 || sp.len < a.w || sp.start + sp.len > a.total;
+    const int n = bd ? 1 : (int)((sp.len + a.chunk_keys - 1) / a.chunk_keys);
+    if (bb < b) {
+      gid0 += n;
+    } else {
+      nch = n;
+      bad = bd;
+    }
+  }
+  if (bad) return;
+  for (int r = threadIdx.x; r < a.Rn; r += blockDim.x) {
+    uint32_t w0 = 0xFF7Fu, w1 = 0u;  // padded row: -3.39e38, so 2^(x * c) = 0
+    if (r < a.R) {
+      const float* pm = a.part_m + ((size_t)g * a.max_chunks + gid0) * a.Rq + r;
+      const double* pl = a.part_l + ((size_t)g * a.max_chunks + gid0) * a.Rq + r;
+      const size_t cs = (size_t)a.Rq;  // stride between consecutive chunks
+      float M = -INFINITY;
+      double L = 0.0;
+      constexpr int kB = 16;
+      for (int c0 = 0; c0 < nch; c0 += kB) {
+        float mv[kB];
+        double lv[kB];
+#pragma unroll
+        for (int u = 0; u < kB; ++u) {
+          const bool in = c0 + u < nch;
+          mv[u] = in ? pm[(c0 + u) * cs] : -INFINITY;
+          lv[u] = in ? pl[(c0 + u) * cs] : 0.0;
+        }
+        float bm = -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kB; ++u) bm = fmaxf(bm, mv[u]);
+        if (bm == -INFINITY) continue;
+        const float Mn = fmaxf(M, bm);
+        double acc = 0.0;
+#pragma unroll
+        for (int u = 0; u < kB; ++u)
+          if (mv[u] != -INFINITY) acc += lv[u] * (double)exp2f(mv[u] - Mn);
+        L = (M == -INFINITY) ? acc : L * (double)exp2f(M - Mn) + acc;
+        M = Mn;
+      }
+      const double v = -((double)M + log2(L)) / (double)a.c;
+      const __nv_bfloat16 h1 = __float2bfloat16_rn((float)v);
+      const double r1 = v - (double)__bfloat162float(h1);
+      const __nv_bfloat16 h2 = __float2bfloat16_rn((float)r1);
+      const double r2 = r1 - (double)__bfloat162float(h2);
+      const __nv_bfloat16 h3 = __float2bfloat16_rn((float)r2);
+      w0 = (uint32_t)__bfloat16_as_ushort(h1) | ((uint32_t)__bfloat16_as_ushort(h2) << 16);
+      w1 = (uint32_t)__bfloat16_as_ushort(h3);
+    }
+    a.qsplit[((size_t)b * a.Hkv + g) * a.Rq + r] = make_uint2(w0, w1);
+  }
+}
+
+// --------------------------------------------------------------------------
 // pass 2: per-key sum of normalised probabilities over the window rows
 // --------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(kThreadsScore, 1)
 score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) {
-  constexpr int kChunks = D / 64;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qs = smem;
-  uint8_t* kst = qs + Smem<D>::q_bytes(a.Rq);
-  Barriers* bars = reinterpret_cast<Barriers*>(kst + (size_t)kStages * Smem<D>::kStageBytes);
-  float* bias_s = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);
+  const SmemPtrs<D> sp(smem_raw, a);
+  Barriers* bars = sp.bars;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = a.g0 + blockIdx.y;
-  const Work wk = map_work(a, blockIdx.x);
+  const Work wk = map_work(a, blockIdx.x, true);
   if (!wk.valid) return;
   if (wk.bad) {
     // leave nothing stale behind: zero whatever part of the row is addressable
@@ -351,172 +565,115 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   const int64_t k1 = std::min<int64_t>(wk.len, k0 + a.chunk_keys);
   const int ntiles = (int)((k1 - k0 + kTile - 1) / kTile);
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      tc::mbar_init(&bars->full[s], 1);
-      tc::mbar_init(&bars->empty[s], 1);
-    }
-    for (int s = 0; s < 2; ++s) {
-      tc::mbar_init(&bars->tfull[s], 1);
-      tc::mbar_init(&bars->tempty[s], kEpiWarps);
-    }
-    bars->abort = 0;
-    tc::fence_mbar_init();
-  }
+  if (threadIdx.x == 0) init_barriers(bars, a.stages, a.nbuf);
   if (warp == 0 && lane == 0) tc::prefetch_tmap(&kmap);
   if (warp == 1) {
     tc::tmem_alloc(&bars->tmem_base, a.tmem_cols);
     tc::tmem_relinquish();
   }
-  load_q_swizzled<D>(a, wk.b, g, qs);
+  {
+    // constant operands of the extra K-step: ones block (keys) and a zeroed
+    // bias block (rows); row r's 16-byte chunk 0 sits at chunk (r & 7)
+    uint4* ones4 = reinterpret_cast<uint4*>(sp.ones);
+    for (int v = threadIdx.x; v < (int)(Smem<D>::kOnesBytes / 16); v += blockDim.x) {
+      const int r = v >> 3, ch = v & 7;
+      ones4[v] = (ch == (r & 7)) ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint4* qb4 = reinterpret_cast<uint4*>(sp.qb);
+    for (int v = threadIdx.x; v < a.Rq * 8; v += blockDim.x) qb4[v] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  load_q_swizzled<D>(a, wk.b, g, sp.qs);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) produce<D>(&kmap, bars, kst, g, wk.start + k0, ntiles);
+    if (lane == 0) produce<D>(&kmap, bars, sp.kst, a.stages, g, wk.start + k0, ntiles, true);
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = tc::idesc_bf16_f32(128, a.Rn);
-      const uint32_t qbase = tc::smem_u32(qs), kbase = tc::smem_u32(kst);
-      int t = 0;
-      for (; t < ntiles; ++t) {
-        const int s = t % kStages, acc = t & 1;
-        if (!tc::mbar_wait(&bars->full[s], (t / kStages) & 1, &bars->abort)) break;
-        if (t >= 2 && !tc::mbar_wait(&bars->tempty[acc], ((t >> 1) - 1) & 1, &bars->abort)) break;
-        tc::tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(acc * a.acc_stride);
-#pragma unroll
-        for (int c = 0; c < kChunks; ++c)
-#pragma unroll
-          for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = tc::desc_k_sw128(kbase + (uint32_t)(s * Smem<D>::kStageBytes + c * kTile * 128 + ks * 32));
-            const uint64_t bd = tc::desc_k_sw128(qbase + (uint32_t)(c * a.Rq * 128 + ks * 32));
-            tc::mma_bf16(d, ad, bd, idesc, (c | ks) != 0);
-          }
-        tc::mma_commit(&bars->empty[s]);
-        tc::mma_commit(&bars->tfull[acc]);
-      }
-      if (t > 0) tc::mbar_drain(&bars->tfull[(t - 1) & 1], ((t - 1) >> 1) & 1);
-    }
+    if (lane == 0) issue_mmas<D, false>(a, bars, tmem, sp.qs, sp.kst, sp.ones, sp.qb, ntiles);
   } else {
-    // ---- epilogue prologue: per-row bias from the pass-1 chunk partials --------
-    // b_r = M + log2(sum_c l_c 2^(m_c - M)), M = max_c m_c.  Padded columns get
-    // b = +inf, so 2^(x*c - inf) = 0 needs no mask.  The producer and MMA warps
-    // are already filling the pipeline meanwhile.
+    // ---- epilogue prologue: this (sequence, head)'s bias rows into the bias
+    // block of the extra MMA K-step, so the accumulator already holds
+    // x - b_r / c.  TMA fills the pipeline meanwhile; the MMA waits for
+    // bias_ready.
     {
-      const int et = threadIdx.x - 64;  // 0..127
-      const size_t base_slot = ((size_t)g * a.max_chunks + (wk.gid - wk.chunk)) * a.Rq;
-      for (int r = et; r < a.Rn; r += 32 * kEpiWarps) {
-        if (r >= a.R) {
-          bias_s[r] = INFINITY;
-          continue;
-        }
-        constexpr int kB = 8;
-        float mx = -INFINITY;
-        for (int c0 = 0; c0 < wk.nchunks; c0 += kB) {
-          float mv[kB];
-#pragma unroll
-          for (int u = 0; u < kB; ++u)
-            mv[u] = (c0 + u < wk.nchunks) ? __ldcg(&a.part_m[base_slot + (size_t)(c0 + u) * a.Rq + r]) : -INFINITY;
-#pragma unroll
-          for (int u = 0; u < kB; ++u) mx = fmaxf(mx, mv[u]);
-        }
-        double l = 0.0;
-        for (int c0 = 0; c0 < wk.nchunks; c0 += kB) {
-          float mv[kB];
-          double lv[kB];
-#pragma unroll
-          for (int u = 0; u < kB; ++u) {
-            const bool in = c0 + u < wk.nchunks;
-            mv[u] = in ? __ldcg(&a.part_m[base_slot + (size_t)(c0 + u) * a.Rq + r]) : -INFINITY;
-            lv[u] = in ? __ldcg(&a.part_l[base_slot + (size_t)(c0 + u) * a.Rq + r]) : 0.0;
-          }
-#pragma unroll
-          for (int u = 0; u < kB; ++u)
-            if (mv[u] != -INFINITY) l += lv[u] * (double)exp2f(mv[u] - mx);
-        }
-        bias_s[r] = (float)((double)mx + log2(l));
+      const int r = threadIdx.x - 64;
+      if (r < a.Rn) {
+        const uint2 wv = a.qsplit[((size_t)wk.b * a.Hkv + g) * a.Rq + r];
+        *reinterpret_cast<uint4*>(sp.qb + (size_t)r * 128 + (size_t)(r & 7) * 16) = make_uint4(wv.x, wv.y, 0u, 0u);
       }
-      tc::named_bar_sync(1, 32 * kEpiWarps);
+      tc::fence_proxy_async_smem();  // visible to the MMA's operand reads
+      tc::mbar_arrive(&bars->bias_ready);
     }
-    // ---- epilogue: one key per thread ------------------------------------------
+    // ---- epilogue: one key per thread; halves take alternate tiles.  The R
+    // columns of a tile come in groups of <= 64; the next group's TMEM load is
+    // in flight while the current one is reduced.
+    const int half = (warp - 2) >> 2;
     const int q = warp & 3;
-    const int kl = 32 * q + lane;              // key within the tile
+    const int kl = 32 * q + lane;  // key within the tile
     const int64_t first_window_key = wk.len - a.w;
-    const int ngroups = (a.Rn + 127) / 128;    // groups of up to 4 x 32 columns
-    for (int t = 0; t < ntiles; ++t) {
-      const int acc = t & 1;
-      if (!tc::mbar_wait(&bars->tfull[acc], (t >> 1) & 1, &bars->abort)) break;
+    const int ng = (a.Rn + 63) / 64;
+    for (int t = half; t < ntiles; t += 2) {
+      const int buf = t % a.nbuf;
+      if (!tc::mbar_wait(&bars->tfull[buf], (t / a.nbuf) & 1, &bars->abort)) break;
       tc::tc_fence_after();
-      const int64_t j = k0 + (int64_t)t * kTile + kl;  // this thread's key (sequence-local)
-      const bool masked_tile = (k0 + (int64_t)t * kTile + kTile - 1 > first_window_key);
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int grp = 0; grp < ngroups; ++grp) {
-        const int col0 = grp * 128;
-        const int ncol = min(128, a.Rn - col0);  // multiple of 16
-        const int nfull = ncol >> 5;             // whole 32-column chunks (0..4)
-        const bool tail16 = (ncol & 31) != 0;    // one trailing 16-column chunk
-        uint32_t x[4][32];
-        uint32_t xt[32];
-        const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(acc * a.acc_stride + col0);
-        if (nfull > 0) KVC_TMEM_LD32(base + 0, x[0]);
-        if (nfull > 1) KVC_TMEM_LD32(base + 32, x[1]);
-        if (nfull > 2) KVC_TMEM_LD32(base + 64, x[2]);
-        if (nfull > 3) KVC_TMEM_LD32(base + 96, x[3]);
-        if (tail16) KVC_TMEM_LD16(base + 32 * nfull, xt);
-        KVC_TMEM_WAIT_LD32(x[0]);
-        KVC_TMEM_TIE32(x[1]);
-        KVC_TMEM_TIE32(x[2]);
-        KVC_TMEM_TIE32(x[3]);
-        KVC_TMEM_TIE32(xt);
-        if (grp == ngroups - 1) {
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&bars->tempty[acc]);
+      const int tp = ntiles - 1 - t;                    // tiles are walked backwards
+      const int64_t j = k0 + (int64_t)tp * kTile + kl;  // this thread's key (sequence-local)
+      const bool masked = (k0 + (int64_t)tp * kTile + kTile - 1 > first_window_key);
+      const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * a.acc_stride);
+      float s8[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s8[u] = 0.f;
+      auto release = [&]() {
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->tempty[buf]);
+      };
+      auto ncol_of = [&](int gi) { return min(64, a.Rn - gi * 64); };
+      auto proc = [&](int gi, uint32_t(&x)[64]) {
+        const int col0 = gi * 64;
+        const int ncol = ncol_of(gi);
+        // columns past ncol (not loaded) and, on tiles reaching into the window,
+        // keys past a row's own position get -inf, i.e. probability 0.  Both
+        // are rare and warp-uniform, so they sit outside the math loop, which
+        // stays branch-free and lets the 64 exponentials interleave.
+        if (ncol < 64) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (e >= ncol) x[e] = __float_as_uint(-INFINITY);
         }
-        if (masked_tile) {
-          // window rows see only keys up to their own position; later keys (and
-          // keys past the sequence) get logit -inf, i.e. probability 0
+        if (masked) {
+          const int64_t lim = j - first_window_key;  // row r visible iff r / G >= lim
 #pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            if (cc >= nfull) break;
-#pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (j > first_window_key + (col0 + cc * 32 + e) / a.G) x[cc][e] = __float_as_uint(-INFINITY);
-          }
-          if (tail16) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              if (j > first_window_key + (col0 + nfull * 32 + e) / a.G) xt[e] = __float_as_uint(-INFINITY);
-          }
+          for (int e = 0; e < 64; ++e)
+            if ((int64_t)((col0 + e) / a.G) < lim) x[e] = __float_as_uint(-INFINITY);
         }
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          if (cc >= nfull) break;
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const float4 bb = *reinterpret_cast<const float4*>(&bias_s[col0 + cc * 32 + e]);
-            s4[0] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 0]), a.c, -bb.x));
-            s4[1] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 1]), a.c, -bb.y));
-            s4[2] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 2]), a.c, -bb.z));
-            s4[3] += tc::ex2_approx(fmaf(__uint_as_float(x[cc][e + 3]), a.c, -bb.w));
-          }
-        }
-        if (tail16) {
-#pragma unroll
-          for (int e = 0; e < 16; e += 4) {
-            const float4 bb = *reinterpret_cast<const float4*>(&bias_s[col0 + nfull * 32 + e]);
-            s4[0] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 0]), a.c, -bb.x));
-            s4[1] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 1]), a.c, -bb.y));
-            s4[2] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 2]), a.c, -bb.z));
-            s4[3] += tc::ex2_approx(fmaf(__uint_as_float(xt[e + 3]), a.c, -bb.w));
+        for (int e = 0; e < 64; ++e) s8[e & 7] += tc::ex2_approx(__uint_as_float(x[e]) * a.c);
+      };
+      uint32_t xa[64], xb[64];
+      tmem_ld_cols(base, xa, ncol_of(0));
+      KVC_TMEM_WAIT_LD64(xa);
+      if (ng > 1) tmem_ld_cols(base + 64, xb, ncol_of(1)); else release();
+      proc(0, xa);
+      if (ng > 1) {
+        KVC_TMEM_WAIT_LD64(xb);
+        if (ng > 2) tmem_ld_cols(base + 128, xa, ncol_of(2)); else release();
+        proc(1, xb);
+        if (ng > 2) {
+          KVC_TMEM_WAIT_LD64(xa);
+          if (ng > 3) tmem_ld_cols(base + 192, xb, ncol_of(3)); else release();
+          proc(2, xa);
+          if (ng > 3) {
+            KVC_TMEM_WAIT_LD64(xb);
+            release();
+            proc(3, xb);
           }
         }
       }
       if (j < k1) {
-        const float v = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        const float v = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
         const int64_t o = (int64_t)g * a.total + wk.start + j;
         a.scores[o] = v;
         if (a.accum) a.accum[o] += v;
@@ -555,8 +712,10 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
 }
 
 struct Geometry {
-  int G, R, Rq, Rn, nb1, acc_stride1, acc_stride;
-  uint32_t cols1, cols2;  // TMEM columns for pass 1 / pass 2
+  int G, R, Rq, Rn, nb1;
+  int stride1, nbuf1;     // pass 1: TMEM columns per accumulator buffer, buffers
+  int stride2, nbuf2;     // pass 2
+  uint32_t cols1, cols2;  // TMEM columns allocated by pass 1 / pass 2
 };
 
 uint32_t pow2_cols(int c) {
@@ -572,10 +731,13 @@ Geometry geometry(const kvc_score_params* p) {
   g.Rn = (g.R + 15) / 16 * 16;
   g.nb1 = (g.R + kTile - 1) / kTile;
   g.Rq = std::max(g.nb1 * kTile, g.Rn);
-  g.acc_stride1 = g.nb1 * kTile;
-  g.acc_stride = (g.Rn + 31) / 32 * 32;
-  g.cols1 = pow2_cols(2 * g.nb1 * kTile);
-  g.cols2 = pow2_cols(2 * g.acc_stride);
+  // as many accumulator buffers (4, else 2) as the 512 TMEM columns allow
+  g.stride1 = g.nb1 * kTile;
+  g.nbuf1 = (kMaxBufs * g.stride1 <= 512) ? kMaxBufs : 2;
+  g.stride2 = (g.Rn + 31) / 32 * 32;
+  g.nbuf2 = (kMaxBufs * g.stride2 <= 512) ? kMaxBufs : 2;
+  g.cols1 = pow2_cols(g.nbuf1 * g.stride1);
+  g.cols2 = pow2_cols(g.nbuf2 * g.stride2);
   return g;
 }
 
@@ -599,6 +761,7 @@ size_t score_ws_bytes(const kvc_score_params* p, int B, int64_t total) {
   size_t s = kWsAlign;                                                              // reserved
   s += round_up((size_t)p->num_kv_heads * mc * gm.Rq * sizeof(float), kWsAlign);    // part_m
   s += round_up((size_t)p->num_kv_heads * mc * gm.Rq * sizeof(double), kWsAlign);   // part_l
+  s += round_up((size_t)B * p->num_kv_heads * gm.Rq * sizeof(uint2), kWsAlign);     // qsplit
   return s;
 }
 
@@ -620,18 +783,38 @@ kvc_status set_smem_attrs(size_t bytes) {
 
 template <int D>
 kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, int hp, cudaStream_t st) {
-  const size_t smem = Smem<D>::total(a.Rq);
-  kvc_status s = set_smem_attrs<D>(smem);
+  // deepest TMA ring that fits next to the other blocks in 227 KB of shared memory
+  const size_t budget = 227 * 1024;
+  int stages[2];
+  size_t smem[2];
+  for (int pass = 0; pass < 2; ++pass) {
+    const size_t fixed = Smem<D>::total(a.Rq, 0, pass);
+    stages[pass] = fixed >= budget ? 0 : (int)std::min<size_t>(kMaxStages, (budget - fixed) / Smem<D>::kStageBytes);
+    if (stages[pass] < 2) return fail(KVC_ERR_UNSUPPORTED, "score kernel: shared memory too small for 2 stages");
+    smem[pass] = Smem<D>::total(a.Rq, stages[pass], pass);
+  }
+  kvc_status s = set_smem_attrs<D>(std::max(smem[0], smem[1]));
   if (s != KVC_OK) return s;
   const int grid_x = (int)((a.total + a.chunk_keys - 1) / a.chunk_keys) + a.B;
   for (int g0 = 0; g0 < a.Hkv; g0 += hp) {
     a.g0 = g0;
     dim3 grid(grid_x, std::min(hp, a.Hkv - g0));
+    a.acc_stride = gm.stride1;
+    a.nbuf = gm.nbuf1;
     a.tmem_cols = gm.cols1;
-    score_pass1_kernel<D><<<grid, kThreadsScore, smem, st>>>(kmap, a);
+    a.stages = stages[0];
+    a.fold = 0;
+    score_pass1_kernel<D><<<grid, kThreadsScore, smem[0], st>>>(kmap, a);
     KVC_CUDA_TRY(cudaGetLastError());
+    score_combine_kernel<<<dim3(a.Hkv, a.B), 256, 0, st>>>(a);
+    KVC_CUDA_TRY(cudaGetLastError());
+    count_launch();
+    a.acc_stride = gm.stride2;
+    a.nbuf = gm.nbuf2;
     a.tmem_cols = gm.cols2;
-    score_pass2_kernel<D><<<grid, kThreadsScore, smem, st>>>(kmap, a);
+    a.stages = stages[1];
+    a.fold = 1;
+    score_pass2_kernel<D><<<grid, kThreadsScore, smem[1], st>>>(kmap, a);
     KVC_CUDA_TRY(cudaGetLastError());
     count_launch(2);
   }
@@ -665,6 +848,7 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
   const int mc = max_chunks_bound(total, B);
   float* part_m = wc.take<float>((size_t)Hkv * mc * gm.Rq);
   double* part_l = wc.take<double>((size_t)Hkv * mc * gm.Rq);
+  uint2* qsplit = wc.take<uint2>((size_t)B * Hkv * gm.Rq);
   if (!wc.ok) return fail(KVC_ERR_WORKSPACE, "score workspace too small");
 
   auto encode = get_encode_fn();
@@ -680,13 +864,10 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return fail(KVC_ERR_CUDA, "cuTensorMapEncodeTiled failed for K");
 
-  // heads per launch: K of those heads should stay in L2 between the passes
-  int dev = 0, l2 = 0;
-  KVC_CUDA_TRY(cudaGetDevice(&dev));
-  KVC_CUDA_TRY(cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev));
-  const double head_bytes = (double)total * d * 2.0;
-  int hp = (int)std::max(1.0, std::floor(0.6 * (double)l2 / head_bytes));
-  hp = std::min(hp, Hkv);
+  // all KV heads in one launch per pass: the CTAs of one key range read whole
+  // [Hkv][d] token rows together, which keeps HBM streaming efficient (head
+  // subsets per launch re-open every DRAM page once per subset)
+  const int hp = Hkv;
   // chunk size: about one wave of CTAs per launch
   const int sms = num_sms();
   const int64_t tiles = (total + kTile - 1) / kTile + (B > 1 ? B : 0);
@@ -708,13 +889,12 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
   a.Rq = gm.Rq;
   a.Rn = gm.Rn;
   a.nb1 = gm.nb1;
-  a.acc_stride1 = gm.acc_stride1;
-  a.acc_stride = gm.acc_stride;
   a.chunk_keys = (int)(chunk_tiles * kTile);
   a.max_chunks = mc;
   a.c = (float)((double)p->scale * kLog2e);
   a.part_m = part_m;
   a.part_l = part_l;
+  a.qsplit = qsplit;
   a.scores = scores;
   a.accum = accum;
   a.total = total;

@@ -140,13 +140,11 @@ struct SelShared {
   uint32_t cnt_gt, cnt_eq;  // this CTA's counts for the output phase
 };
 
-// Warp-aggregated histogram increment: lanes with the same bin add once.
-// Every lane of the warp must call it (inactive lanes with active = false).
+// Histogram increment.  Contention is modest (a CTA's 16K keys spread over
+// tens of first-pass bins; later passes only see the keys of one bucket), so
+// plain shared-memory atomics beat warp-level match/aggregate here.
 __device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool active) {
-  const unsigned mask = __ballot_sync(0xffffffffu, active);
-  if (!active) return;
-  const unsigned peers = __match_any_sync(mask, bin);
-  if ((int)(threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[bin], __popc(peers));
+  if (active) atomicAdd(&hist[bin], 1);
 }
 
 // Dynamic shared memory of the selection kernel: the staged row sums of the
