@@ -257,24 +257,36 @@ def main() -> None:
     plan = kvc.LayerPlan(cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden, True, dev,
                          pool_kernel=cfg.pool)
     st = torch.cuda.current_stream(dev)
+    side = plan.side
     calls = ["score", "select_kv", "gather_kv", "select_tsp", "gather_hidden"]
+    call_stream = {"score": st, "select_kv": side, "gather_kv": side, "select_tsp": st, "gather_hidden": st}
+    ev_scores, ev_side = torch.cuda.Event(), torch.cuda.Event()
 
     def step(evs=None):
-        def mark(i):
+        """One layer: the K/V chain on a side stream, the TSP chain on the main
+        stream (as LayerPlan.run), with optional per-call timing events
+        recorded on the stream each call runs on."""
+        def timed(name, fn):
             if evs is not None:
-                evs[i].record(st)
-        mark(0)
-        kvc.kvc_score(q, k, scores=plan.scores, ws=plan.ws_score, dev_err=plan.dev_err)
-        mark(1)
-        kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_kv, idx=plan.idx_kv, ws=plan.ws_sel_kv)
-        mark(2)
-        kvc.kvc_gather_kv(k, v, plan.idx_kv, k_out=plan.k_c, v_out=plan.v_c, dev_err=plan.dev_err)
-        mark(3)
-        kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_tsp, row_group=cfg.Hkv, idx=plan.idx_tsp,
-                            ws=plan.ws_sel_tsp)
-        mark(4)
-        kvc.kvc_gather_hidden(x, plan.idx_tsp.view(-1), out=plan.x_c, dev_err=plan.dev_err)
-        mark(5)
+                evs[name][0].record(call_stream[name])
+            fn()
+            if evs is not None:
+                evs[name][1].record(call_stream[name])
+        timed("score", lambda: kvc.kvc_score(q, k, scores=plan.scores, ws=plan.ws_score, dev_err=plan.dev_err,
+                                             stream=st))
+        ev_scores.record(st)
+        side.wait_event(ev_scores)
+        timed("select_kv", lambda: kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_kv, idx=plan.idx_kv,
+                                                       ws=plan.ws_sel_kv, stream=side))
+        timed("gather_kv", lambda: kvc.kvc_gather_kv(k, v, plan.idx_kv, k_out=plan.k_c, v_out=plan.v_c,
+                                                     dev_err=plan.dev_err, stream=side))
+        timed("select_tsp", lambda: kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_tsp,
+                                                        row_group=cfg.Hkv, idx=plan.idx_tsp, ws=plan.ws_sel_tsp,
+                                                        stream=st))
+        timed("gather_hidden", lambda: kvc.kvc_gather_hidden(x, plan.idx_tsp.view(-1), out=plan.x_c,
+                                                             dev_err=plan.dev_err, stream=st))
+        ev_side.record(side)
+        st.wait_event(ev_side)
 
     for _ in range(args.warmup):
         step()
@@ -283,7 +295,8 @@ def main() -> None:
         raise RuntimeError(f"device error word {plan.dev_err.item()}")
 
     # ---- timed region ----------------------------------------------------------
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    evs = [{c: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for c in calls}
+           for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
@@ -302,8 +315,8 @@ def main() -> None:
     launches = kvc.launch_count() - launches0
     ms_total = shard.max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     ms_step = ms_total / args.steps
-    per_call = {c: sum(evs[s][i].elapsed_time(evs[s][i + 1]) for s in range(args.steps)) / args.steps
-                for i, c in enumerate(calls)}
+    per_call = {c: sum(evs[s][c][0].elapsed_time(evs[s][c][1]) for s in range(args.steps)) / args.steps
+                for c in calls}
 
     # ---- end to end through the public API with host buffers ------------------
     hq, hk, hv, hx = (workloads.torch_bf16(a).pin_memory() for a in (lay.q, lay.k, lay.v, lay.x))

@@ -385,20 +385,38 @@ class LayerPlan:
             self.idx_tsp = torch.empty((1, min(k_tsp, n)), dtype=i32, device=device)
             self.x_c = (torch.empty((min(k_tsp, n), hidden), dtype=bf, device=device)
                         if hidden else None)
+        self.side = torch.cuda.Stream(device=device)
+        self._ev_scores = torch.cuda.Event()
+        self._ev_side = torch.cuda.Event()
 
     def run(self, q_win, k, v=None, x=None, stream=None) -> LayerOutputs:
         """Score -> per-KV-head top-k -> K/V gather; with a TSP budget also the
-        all-head top-k -> hidden-state gather.  Nothing is synchronised."""
-        kvc_score(q_win, k, scores=self.scores, ws=self.ws_score, dev_err=self.dev_err, stream=stream)
+        all-head top-k -> hidden-state gather.
+
+        The two selection -> gather chains only share the scores, so the K/V
+        chain runs on a side stream concurrently with the TSP chain; both
+        join the calling stream before returning.  Nothing is synchronised
+        with the host; inputs must stay alive until the work completes."""
+        main = stream if stream is not None else torch.cuda.current_stream(self.scores.device)
+        kvc_score(q_win, k, scores=self.scores, ws=self.ws_score, dev_err=self.dev_err, stream=main)
+        out = LayerOutputs(self.scores, self.idx_kv, self.k_c, self.v_c)
+        if self.k_tsp is None:
+            self._kv_chain(k, v, main)
+            return out
+        self._ev_scores.record(main)
+        self.side.wait_event(self._ev_scores)
+        self._kv_chain(k, v, self.side)
+        kvc_select_topk(self.scores, self.w, self.pool, self.k_tsp, row_group=self.Hkv, idx=self.idx_tsp,
+                        ws=self.ws_sel_tsp, stream=main)
+        out.idx_tsp = self.idx_tsp
+        if x is not None and self.x_c is not None:
+            kvc_gather_hidden(x, self.idx_tsp.view(-1), out=self.x_c, dev_err=self.dev_err, stream=main)
+            out.x_c = self.x_c
+        self._ev_side.record(self.side)
+        main.wait_event(self._ev_side)
+        return out
+
+    def _kv_chain(self, k, v, stream):
         kvc_select_topk(self.scores, self.w, self.pool, self.k_kv, idx=self.idx_kv, ws=self.ws_sel_kv,
                         stream=stream)
         kvc_gather_kv(k, v, self.idx_kv, k_out=self.k_c, v_out=self.v_c, dev_err=self.dev_err, stream=stream)
-        out = LayerOutputs(self.scores, self.idx_kv, self.k_c, self.v_c)
-        if self.k_tsp is not None:
-            kvc_select_topk(self.scores, self.w, self.pool, self.k_tsp, row_group=self.Hkv, idx=self.idx_tsp,
-                            ws=self.ws_sel_tsp, stream=stream)
-            out.idx_tsp = self.idx_tsp
-            if x is not None and self.x_c is not None:
-                kvc_gather_hidden(x, self.idx_tsp.view(-1), out=self.x_c, dev_err=self.dev_err, stream=stream)
-                out.x_c = self.x_c
-        return out

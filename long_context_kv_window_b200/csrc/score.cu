@@ -66,6 +66,7 @@ struct ScoreArgs {
   int nbuf;                  // TMEM accumulator buffers (this pass): 2 or 4
   int stages;                // TMA ring depth
   int fold;                  // pass 2: the row bias rides in one extra MMA K-step
+  float keep_frac;           // pass 1: trailing fraction of each chunk left at normal L2 priority
   uint32_t tmem_cols;        // TMEM columns allocated (this pass)
   int g0;                    // first KV head of this launch
   int chunk_keys;
@@ -207,11 +208,20 @@ __device__ __forceinline__ void init_barriers(Barriers* bars, int stages, int nb
 }
 
 // Producer: stream the chunk's K tiles of head g into the stage ring.
+//
+// L2 policy: K is read by both passes, and more of it than L2 holds.  Pass 1
+// loads the leading part of each chunk evict_first and its trailing
+// `keep_frac` at normal priority; pass 2 walks the chunk backwards, so it
+// starts on those trailing tiles while they are still in L2, and loads
+// everything evict_first (nothing reads K after it).
 template <int D>
 __device__ __forceinline__ void produce(const void* kmap, Barriers* bars, uint8_t* kst, int stages, int g,
-                                        int64_t row0, int ntiles, bool reverse) {
+                                        int64_t row0, int ntiles, bool reverse, float keep_frac) {
   constexpr int kChunks = D / 64;
   constexpr uint32_t kBytes = (uint32_t)Smem<D>::kStageBytes;
+  const uint64_t pol_first = tc::l2_policy_evict_first();
+  const uint64_t pol_keep = tc::l2_policy_evict_normal();
+  const int first_kept = reverse ? ntiles : ntiles - (int)((float)ntiles * keep_frac);
   int issued = 0;
   for (int t = 0; t < ntiles; ++t) {
     const int s = t % stages;
@@ -221,8 +231,9 @@ __device__ __forceinline__ void produce(const void* kmap, Barriers* bars, uint8_
     uint8_t* dst = kst + (size_t)s * Smem<D>::kStageBytes;
 #pragma unroll
     for (int c = 0; c < kChunks; ++c)
-      tc::tma_load_3d(dst + c * kTile * 128, kmap, &bars->full[s], c * 64, g,
-                      (int)(row0 + (int64_t)(reverse ? ntiles - 1 - t : t) * kTile));
+      tc::tma_load_3d_hint(dst + c * kTile * 128, kmap, &bars->full[s], c * 64, g,
+                           (int)(row0 + (int64_t)(reverse ? ntiles - 1 - t : t) * kTile),
+                           t >= first_kept ? pol_keep : pol_first);
     issued = t + 1;
   }
   if (bars->abort) {
@@ -380,7 +391,7 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) produce<D>(&kmap, bars, sp.kst, a.stages, g, wk.start + k0, ntiles, false);
+    if (lane == 0) produce<D>(&kmap, bars, sp.kst, a.stages, g, wk.start + k0, ntiles, false, a.keep_frac);
   } else if (warp == 1) {
     if (lane == 0) issue_mmas<D, true>(a, bars, tmem, sp.qs, sp.kst, sp.ones, sp.qb, ntiles);
   } else {
@@ -589,7 +600,7 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    if (lane == 0) produce<D>(&kmap, bars, sp.kst, a.stages, g, wk.start + k0, ntiles, true);
+    if (lane == 0) produce<D>(&kmap, bars, sp.kst, a.stages, g, wk.start + k0, ntiles, true, a.keep_frac);
   } else if (warp == 1) {
     if (lane == 0) issue_mmas<D, false>(a, bars, tmem, sp.qs, sp.kst, sp.ones, sp.qb, ntiles);
   } else {
@@ -868,6 +879,13 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
   // [Hkv][d] token rows together, which keeps HBM streaming efficient (head
   // subsets per launch re-open every DRAM page once per subset)
   const int hp = Hkv;
+  // trailing fraction of each chunk pass 1 leaves at normal L2 priority:
+  // about 70 % of L2 worth of K (the rest of L2 serves everything else)
+  int dev = 0, l2 = 0;
+  KVC_CUDA_TRY(cudaGetDevice(&dev));
+  KVC_CUDA_TRY(cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev));
+  const double k_bytes = (double)total * Hkv * d * 2.0;
+  const float keep_frac = (float)std::min(1.0, 0.7 * (double)l2 / k_bytes);
   // chunk size: about one wave of CTAs per launch
   const int sms = num_sms();
   const int64_t tiles = (total + kTile - 1) / kTile + (B > 1 ? B : 0);
@@ -892,6 +910,7 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
   a.chunk_keys = (int)(chunk_tiles * kTile);
   a.max_chunks = mc;
   a.c = (float)((double)p->scale * kLog2e);
+  a.keep_frac = keep_frac;
   a.part_m = part_m;
   a.part_l = part_l;
   a.qsplit = qsplit;

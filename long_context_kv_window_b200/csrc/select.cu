@@ -41,7 +41,7 @@ __device__ __forceinline__ float key_value(uint32_t key) {
   return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
-struct RadixShared {
+struct __align__(16) RadixShared {
   int hist[2][kBins];  // local histograms (alternating between passes)
   int tot[kBins];      // cluster-summed histogram
   uint32_t warp_tmp[kWarps + 1];  // [kWarps] holds the last scan's block total
@@ -79,17 +79,37 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_t
   return warp_tmp[warp] + x - v;
 }
 
+// Sum of this CTA's local hist[lo+1 .. nbins) (all threads get it).
+__device__ __forceinline__ uint32_t local_count_above(RadixShared& sh, int buf, int nbins, uint32_t lo) {
+  uint32_t mine = 0;
+  for (int b = threadIdx.x; b < nbins; b += kThreads)
+    if ((uint32_t)b > lo) mine += (uint32_t)sh.hist[buf][b];
+  uint32_t total;
+  block_excl_scan(mine, sh.warp_tmp, &total);
+  return total;
+}
+
 // After every CTA of the cluster filled hist[buf] (and a cluster barrier),
 // sum the kCS histograms and find the bin that holds the want-th largest
 // candidate: count(bins above) < want <= count(bins above) + tot[bin].
 // Bins are visited from the top.  Returns through sh.found_*.
 __device__ void cluster_find_bucket(cg::cluster_group& cluster, RadixShared& sh, int buf, int nbins,
                                     uint32_t want) {
-  for (int b = threadIdx.x; b < nbins; b += kThreads) {
-    int s = 0;
+  // 16-byte loads of every rank's histogram, all issued before the sum: one
+  // round trip through distributed shared memory
+  for (int v4 = threadIdx.x; v4 < nbins / 4; v4 += kThreads) {
+    int4 part[kCS];
 #pragma unroll
-    for (int c = 0; c < kCS; ++c) s += cluster.map_shared_rank(&sh.hist[buf][0], c)[b];
-    sh.tot[b] = s;
+    for (int c = 0; c < kCS; ++c) part[c] = reinterpret_cast<const int4*>(cluster.map_shared_rank(&sh.hist[buf][0], c))[v4];
+    int4 acc = part[0];
+#pragma unroll
+    for (int c = 1; c < kCS; ++c) {
+      acc.x += part[c].x;
+      acc.y += part[c].y;
+      acc.z += part[c].z;
+      acc.w += part[c].w;
+    }
+    reinterpret_cast<int4*>(sh.tot)[v4] = acc;
   }
   __syncthreads();
   // thread t owns the group of bins (kThreads-1-t): higher t = lower bins
@@ -150,7 +170,7 @@ __device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool active) {
 // Dynamic shared memory of the selection kernel: the staged row sums of the
 // segment plus halo, and the pooled values of the segment (smem mode).
 __host__ __device__ inline size_t sel_dyn_smem(int64_t seg, int half, bool smem_vals) {
-  return smem_vals ? (size_t)(2 * seg + 2 * half + 8) * sizeof(float) : 0;
+  return smem_vals ? (size_t)(2 * seg + 2 * half + 16) * sizeof(float) : 0;
 }
 
 __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kThreads, 1)
@@ -213,7 +233,7 @@ select_kernel(const SelArgs a) {
   const float* rows0 = a.scores + (int64_t)o * a.row_group * a.row_stride + start;
   float* gvals = a.vals_g ? a.vals_g + (int64_t)o * a.vals_stride + (a.vals_packed ? start : 0) : nullptr;
   // pooled values of the segment, indexed 0..nseg-1 (shared or global memory)
-  float* v = a.smem_vals ? dyn + (nseg + 2 * half + 8) : gvals + s0;
+  float* v = a.smem_vals ? dyn + ((nseg + 2 * half + 8 + 3) & ~3) : gvals + s0;  // 16-B aligned in smem
 
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[0][i] = 0;
   __syncthreads();
@@ -242,22 +262,40 @@ select_kernel(const SelArgs a) {
       }
     }
     __syncthreads();
-    for (int base = 0; base < nseg; base += kThreads) {
-      const int t = base + threadIdx.x;
-      const bool in = t < nseg;
-      float val = 0.f;
-      if (in) {
-        if (a.pool == 1) {
-          val = stage[t];
-        } else {
-          float sum = 0.f;
-          for (int q = 0; q <= 2 * half; ++q) sum += stage[t + q];
-          val = sum / pool_div;
-        }
-        v[t] = val;
-        if (gvals) gvals[s0 + t] = val;
+    // v[t] = sum of the p staged row sums around t.  Ranking uses this sum: the
+    // average differs by the constant factor 1/p, a monotone map, so the order
+    // (ties to the lower position) is the same; the average itself is only
+    // formed for the optional pooled output.  Four consecutive outputs per
+    // thread and round share one register window of 4 + 2*half staged values.
+    const int span_w = 4 + 2 * half;
+    for (int base = 0; base < nseg; base += 4 * kThreads) {
+      const int t0 = base + 4 * threadIdx.x;
+      float sums[4] = {0.f, 0.f, 0.f, 0.f};
+      if (half <= 8) {
+        float win[4 + 16];
+#pragma unroll
+        for (int q = 0; q < 4 + 16; ++q) win[q] = (q < span_w && t0 + q < span) ? stage[t0 + q] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int q = 0; q < 17; ++q)
+            if (q <= 2 * half) sums[u] += win[u + q];
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          for (int q = 0; q <= 2 * half; ++q)
+            if (t0 + u + q < span) sums[u] += stage[t0 + u + q];
       }
-      if (need_rank) hist_add(sh.rx.hist[0], order_key(val) >> 21, in);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int t = t0 + u;
+        const bool in = t < nseg;
+        if (in) {
+          v[t] = sums[u];
+          if (gvals) gvals[s0 + t] = (a.pool == 1) ? sums[u] : sums[u] / pool_div;
+        }
+        if (need_rank) hist_add(sh.rx.hist[0], order_key(sums[u]) >> 21, in);
+      }
     }
   } else {
     // long rows: pooled values go straight to global memory (L2-resident)
@@ -274,19 +312,32 @@ select_kernel(const SelArgs a) {
           for (int r = 0; r < a.row_group; ++r) rs += rows0[(int64_t)r * a.row_stride + pos];
           sum += rs;
         }
-        val = (a.pool == 1) ? sum : sum / pool_div;
+        val = sum;  // ranked as the pooled sum (see the shared-memory path)
         v[t] = val;
       }
       if (need_rank) hist_add(sh.rx.hist[0], order_key(val) >> 21, in);
     }
   }
-  if (!need_rank) return;
+  // global-memory mode keeps the pooled sums in the caller's buffer while
+  // ranking; it holds the averages once this CTA no longer reads them
+  auto finish_gvals = [&]() {
+    if (!a.smem_vals && gvals && a.pool > 1) {
+      __syncthreads();
+      for (int t = threadIdx.x; t < nseg; t += kThreads) v[t] = v[t] / pool_div;
+    }
+  };
+  if (!need_rank) {
+    finish_gvals();
+    return;
+  }
 
   // ---- radix passes ---------------------------------------------------------
   cluster.sync();
   cluster_find_bucket(cluster, sh.rx, 0, kBins, (uint32_t)kk);
   const uint32_t b1 = sh.rx.found_bucket;
   uint32_t want = sh.rx.found_rem;
+  // keys of this CTA above bucket b1 are selected whatever the finer bits
+  const uint32_t gt1 = local_count_above(sh.rx, 0, kBins, b1);
 
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[1][i] = 0;
   __syncthreads();
@@ -300,6 +351,7 @@ select_kernel(const SelArgs a) {
   const uint32_t b2 = sh.rx.found_bucket;
   want = sh.rx.found_rem;
   const uint32_t pre2 = (b1 << 11) | b2;
+  const uint32_t gt2 = local_count_above(sh.rx, 1, kBins, b2);
 
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[0][i] = 0;
   __syncthreads();
@@ -310,41 +362,69 @@ select_kernel(const SelArgs a) {
   }
   cluster.sync();
   cluster_find_bucket(cluster, sh.rx, 0, 1024, want);
-  const uint32_t T = (pre2 << 10) | sh.rx.found_bucket;
+  const uint32_t b3 = sh.rx.found_bucket;
+  const uint32_t T = (pre2 << 10) | b3;
   const uint32_t need_eq = sh.rx.found_rem;  // how many keys == T are taken (lowest positions)
 
-  // ---- counts per CTA, then cluster prefix ---------------------------------
-  uint32_t gt = 0, eq = 0;
-  for (int t = threadIdx.x; t < nseg; t += kThreads) {
-    const uint32_t key = order_key(v[t]);
-    gt += key > T;
-    eq += key == T;
+  // ---- counts per CTA (from the local histograms), then cluster prefix ------
+  const uint32_t gt3 = local_count_above(sh.rx, 0, 1024, b3);
+  if (threadIdx.x == 0) {
+    sh.cnt_gt = gt1 + gt2 + gt3;
+    sh.cnt_eq = (uint32_t)sh.rx.hist[0][b3];
   }
-  uint32_t tot;
-  block_excl_scan(gt, sh.rx.warp_tmp, &tot);
-  if (threadIdx.x == 0) sh.cnt_gt = tot;
-  block_excl_scan(eq, sh.rx.warp_tmp, &tot);
-  if (threadIdx.x == 0) sh.cnt_eq = tot;
   cluster.sync();
   uint32_t out_base = 0, eq_seen = 0;
-  for (int c = 0; c < crank; ++c) {
-    SelShared* r = cluster.map_shared_rank(&sh, c);
-    const uint32_t e = r->cnt_eq;
-    const uint32_t take = eq_seen < need_eq ? (need_eq - eq_seen < e ? need_eq - eq_seen : e) : 0u;
-    out_base += r->cnt_gt + take;
-    eq_seen += e;
+  if (threadIdx.x < 32) {
+    // lanes c < crank hold rank c's counts; a warp scan gives this CTA's offset
+    const int lane = threadIdx.x;
+    uint32_t cg_ = 0, ce = 0;
+    if (lane < crank) {
+      const SelShared* r = cluster.map_shared_rank(&sh, lane);
+      cg_ = r->cnt_gt;
+      ce = r->cnt_eq;
+    }
+    // equal keys are taken by rank order: rank c takes min(ce, quota left)
+    uint32_t ce_before = ce;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, ce_before, o);
+      if (lane >= o) ce_before += y;
+    }
+    ce_before -= ce;  // exclusive
+    const uint32_t take = ce_before < need_eq ? min(need_eq - ce_before, ce) : 0u;
+    uint32_t sum = cg_ + take;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    uint32_t eqs = ce;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) eqs += __shfl_xor_sync(0xffffffffu, eqs, o);
+    if (lane == 0) {
+      sh.rx.found_bucket = sum;  // reused as scratch: output offset of this CTA
+      sh.rx.found_rem = eqs;     // equal keys in earlier ranks
+    }
   }
+  __syncthreads();
+  out_base = sh.rx.found_bucket;
+  eq_seen = sh.rx.found_rem;
 
   // ---- order-preserving compaction -----------------------------------------
   for (int t0 = 0; t0 < nseg; t0 += kThreads * kPerTile) {
     const int tb = t0 + threadIdx.x * kPerTile;
     uint32_t keys[kPerTile];
     uint32_t my_gt = 0, my_eq = 0;
+    if (a.smem_vals && tb + kPerTile <= nseg) {
+      const float4 f = *reinterpret_cast<const float4*>(v + tb);  // conflict-free 16-B loads
+      keys[0] = order_key(f.x);
+      keys[1] = order_key(f.y);
+      keys[2] = order_key(f.z);
+      keys[3] = order_key(f.w);
+    } else {
+#pragma unroll
+      for (int q = 0; q < kPerTile; ++q) keys[q] = (tb + q < nseg) ? order_key(v[tb + q]) : 0u;
+    }
 #pragma unroll
     for (int q = 0; q < kPerTile; ++q) {
-      const int t = tb + q;
-      keys[q] = (t < nseg) ? order_key(v[t]) : 0u;
-      if (t < nseg) {
+      if (tb + q < nseg) {
         my_gt += keys[q] > T;
         my_eq += keys[q] == T;
       }
@@ -370,6 +450,7 @@ select_kernel(const SelArgs a) {
     out_base += tg + (te < quota ? te : quota);
     eq_seen += te;
   }
+  finish_gvals();
   cluster.sync();  // remote reads of sh are over before any CTA exits
 }
 

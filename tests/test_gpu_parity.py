@@ -96,6 +96,24 @@ def test_select_exact_on_given_scores_no_pool(n, w, k):
         assert np.array_equal(idx[r], ref), f"row {r}"
 
 
+@pytest.mark.parametrize("n,pool", [(420000, 7), (420000, 1)])
+def test_select_long_row_global_memory_mode(n, pool):
+    """Rows too long for the per-CTA shared-memory segments: pooled values
+    live in global memory during ranking and are averages on return."""
+    rng = np.random.default_rng(n + pool)
+    w, k = 32, 4200
+    S = (rng.random((2, n)) ** 4).astype(np.float32)
+    pooled = torch.empty((2, n - w), dtype=torch.float32, device="cuda")
+    idx = kvc.kvc_select_topk(torch.from_numpy(S).cuda(), w, pool, k, pooled=pooled).cpu().numpy()
+    idx_ws = kvc.kvc_select_topk(torch.from_numpy(S).cuda(), w, pool, k).cpu().numpy()
+    assert np.array_equal(idx, idx_ws)
+    orc = oracle.get()
+    for r in range(2):
+        Sp = orc.rank_scores(S[r].astype(np.float64), n, w, pool)
+        parity.assert_scores_close(pooled[r].cpu().numpy(), Sp, rtol=1e-6, what="pooled")
+        parity.assert_selection_matches(idx[r], orc.select_topk(Sp, n, w, k), Sp, n, w, k)
+
+
 @pytest.mark.parametrize("pool", [3, 7])
 def test_select_pooled_and_grouped(pool):
     rng = np.random.default_rng(pool)
