@@ -218,6 +218,8 @@ def main() -> None:
     ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps one by one instead of replaying a CUDA graph")
     ap.add_argument("--tokens", type=int, default=None,
                     help="same layer structure at another N (small cases for profiling)")
     args = ap.parse_args()
@@ -259,13 +261,14 @@ def main() -> None:
     st = torch.cuda.current_stream(dev)
     side = plan.side
     calls = ["score", "select_kv", "gather_kv", "select_tsp", "gather_hidden"]
-    call_stream = {"score": st, "select_kv": side, "gather_kv": side, "select_tsp": st, "gather_hidden": st}
-    ev_scores, ev_side = torch.cuda.Event(), torch.cuda.Event()
-
-    def step(evs=None):
+    def step(evs=None, main=None):
         """One layer: the K/V chain on a side stream, the TSP chain on the main
         stream (as LayerPlan.run), with optional per-call timing events
         recorded on the stream each call runs on."""
+        st = main if main is not None else torch.cuda.current_stream(dev)
+        call_stream = {"score": st, "select_kv": side, "gather_kv": side, "select_tsp": st, "gather_hidden": st}
+        ev_scores, ev_side = torch.cuda.Event(), torch.cuda.Event()
+
         def timed(name, fn):
             if evs is not None:
                 evs[name][0].record(call_stream[name])
@@ -295,24 +298,42 @@ def main() -> None:
         raise RuntimeError(f"device error word {plan.dev_err.item()}")
 
     # ---- timed region ----------------------------------------------------------
-    evs = [{c: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for c in calls}
+    # per-call events; "external" so that, recorded inside a CUDA graph, they
+    # stay readable (timing) after the replay
+    evs = [{c: (torch.cuda.Event(enable_timing=True, external=not args.no_graph),
+                torch.cuda.Event(enable_timing=True, external=not args.no_graph)) for c in calls}
            for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(local)
     launches0 = kvc.launch_count()
+    graph = None
+    if not args.no_graph:
+        # the K steps (with their per-call events) are captured once and
+        # replayed as one CUDA graph: no host launch overhead between kernels
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream(dev)
+            for s in range(args.steps):
+                step(evs[s], main=cap)
+        torch.cuda.synchronize(dev)
+    launches = kvc.launch_count() - launches0
     with sampler:
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
         t_start.record(st)
-        for s in range(args.steps):
-            step(evs[s])
+        if graph is not None:
+            graph.replay()
+        else:
+            for s in range(args.steps):
+                step(evs[s], main=st)
         t_end.record(st)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-    launches = kvc.launch_count() - launches0
+    if graph is None:
+        launches = kvc.launch_count() - launches0
     ms_total = shard.max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
     ms_step = ms_total / args.steps
     per_call = {c: sum(evs[s][c][0].elapsed_time(evs[s][c][1]) for s in range(args.steps)) / args.steps
@@ -373,6 +394,7 @@ def main() -> None:
             "e2e": {"value": world * cfg.N / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": launches,
+            "graph": graph is not None,
             "clocks": sampler.summary(),
             "cpu_baseline": cpu,
         }
