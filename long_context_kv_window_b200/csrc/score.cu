@@ -26,8 +26,10 @@
 // tiles pass 1 read last, which are still in L2.
 //
 // Warp roles per CTA: warp 0 issues TMA, warp 1 allocates TMEM and issues
-// MMAs, warps 2..9 drain TMEM (epilogue; two warps per TMEM lane quarter,
-// taking alternate tiles).  Every wait is bounded; on a
+// MMAs, warps 2..17 drain TMEM (epilogue: four groups of four warps, one warp
+// per TMEM lane quarter; the groups take the tiles in turn, so four warps per
+// SM sub-partition hide each other's TMEM-load and MUFU latencies).  Every
+// wait is bounded; on a
 // timeout the CTA records KVC_DEV_ERR_TIMEOUT, lets in-flight copies and MMAs
 // land, frees TMEM and exits.
 #include <cuda.h>
@@ -47,7 +49,9 @@ namespace {
 constexpr int kTile = 128;       // keys per tile
 constexpr int kMaxStages = 8;    // TMA ring depth bound (the host picks what fits)
 constexpr int kMaxBufs = 4;      // TMEM accumulator buffers
-constexpr int kEpiWarps = 8;     // two per TMEM lane quarter; the halves take alternate tiles
+constexpr int kEpiWarps = 16;    // groups of four, one warp per TMEM lane quarter
+constexpr int kGroups = kEpiWarps / 4;  // the groups take the tiles in turn
+constexpr int kCols = 32;        // accumulator columns per TMEM load
 constexpr int kThreadsScore = 64 + 32 * kEpiWarps;
 constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kMinChunkTiles = 4;
@@ -129,7 +133,7 @@ struct Barriers {
 };
 
 // Shared memory: [Q rows, swizzled][pass 2: ones | bias block][K stage ring]
-// [barriers | bias | exchange].  The pass-2 blocks hold one extra K-step of
+// [barriers | exchange of the pass-1 group partials].  The pass-2 blocks hold one extra K-step of
 // the MMA: a [128 keys x 16] block of (1, 1, 1, 0, ...) and a [Rq x 16] block
 // of each row's (h1, h2, h3, 0, ...) with h1 + h2 + h3 = -bias / c (three
 // bf16 parts of an fp32-accurate value), laid out like the K tiles.
@@ -138,7 +142,7 @@ struct Smem {
   static constexpr int kChunks = D / 64;  // 64-element (128 B) swizzle columns
   static constexpr int kStageBytes = kChunks * kTile * 128;
   static constexpr size_t kOnesBytes = (size_t)kTile * 128;
-  static constexpr size_t kTail = 512 /*barriers*/ + 256 * 4 /*bias*/ + 256 * 4 + 256 * 8 /*exchange*/;
+  static constexpr size_t kTail = 512 /*barriers*/ + (size_t)(kGroups - 1) * 256 * (4 + 8) /*exchange*/;
   __host__ __device__ static size_t q_bytes(int Rq) { return (size_t)kChunks * Rq * 128; }
   __host__ __device__ static size_t fold_bytes(int Rq, int fold) { return fold ? kOnesBytes + (size_t)Rq * 128 : 0; }
   __host__ __device__ static size_t total(int Rq, int stages, int fold) {
@@ -153,9 +157,8 @@ struct SmemPtrs {
   uint8_t* qb;    // pass 2 only
   uint8_t* kst;
   Barriers* bars;
-  float* bias;   // [256]
-  float* ex_m;   // [256]
-  double* ex_l;  // [256]
+  float* ex_m;   // [kGroups - 1][256]
+  double* ex_l;  // [kGroups - 1][256]
   __device__ SmemPtrs(uint8_t* raw, const ScoreArgs& a) {
     uint8_t* s = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     qs = s;
@@ -163,9 +166,8 @@ struct SmemPtrs {
     qb = ones + Smem<D>::kOnesBytes;
     kst = qs + Smem<D>::q_bytes(a.Rq) + Smem<D>::fold_bytes(a.Rq, a.fold);
     bars = reinterpret_cast<Barriers*>(kst + (size_t)a.stages * Smem<D>::kStageBytes);
-    bias = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);
-    ex_m = bias + 256;
-    ex_l = reinterpret_cast<double*>(ex_m + 256);
+    ex_m = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);
+    ex_l = reinterpret_cast<double*>(ex_m + (kGroups - 1) * 256);
   }
 };
 
@@ -191,8 +193,8 @@ __device__ __forceinline__ void load_q_swizzled(const ScoreArgs& a, int b, int g
   tc::fence_proxy_async_smem();
 }
 
-// Barrier init (one thread) for the stage ring and the TMEM buffers.  Buffer
-// b is drained by the four epilogue warps of half b % 2.
+// Barrier init (one thread) for the stage ring and the TMEM buffers.  Each
+// use of a buffer is drained by the four warps of one epilogue group.
 __device__ __forceinline__ void init_barriers(Barriers* bars, int stages, int nbuf) {
   for (int s = 0; s < stages; ++s) {
     tc::mbar_init(&bars->full[s], 1);
@@ -200,7 +202,7 @@ __device__ __forceinline__ void init_barriers(Barriers* bars, int stages, int nb
   }
   for (int s = 0; s < nbuf; ++s) {
     tc::mbar_init(&bars->tfull[s], 1);
-    tc::mbar_init(&bars->tempty[s], kEpiWarps / 2);
+    tc::mbar_init(&bars->tempty[s], kEpiWarps / kGroups);
   }
   tc::mbar_init(&bars->bias_ready, kEpiThreads);
   bars->abort = 0;
@@ -289,6 +291,17 @@ __device__ __forceinline__ void issue_mmas(const ScoreArgs& a, Barriers* bars, u
 
 __device__ __forceinline__ void record_timeout(int32_t* err) { set_dev_err(err, KVC_DEV_ERR_TIMEOUT); }
 
+// Epilogue group: wait until the accumulator of tile t is filled.  An
+// mbarrier wait only tells phases apart by parity, so with fewer buffers than
+// groups (a group then skips uses of its buffer) it first waits for the
+// release of the buffer's previous use, by another group: after that the
+// buffer's tfull barrier is at most one phase behind this use.
+__device__ __forceinline__ bool wait_filled(const ScoreArgs& a, Barriers* bars, int t) {
+  const int buf = t % a.nbuf, ub = t / a.nbuf;
+  if (a.nbuf < kGroups && ub > 0 && !tc::mbar_wait(&bars->tempty[buf], (ub - 1) & 1, &bars->abort)) return false;
+  return tc::mbar_wait(&bars->tfull[buf], ub & 1, &bars->abort);
+}
+
 // Online merge of (m, l) pairs in the log2 domain: l * 2^(m - M) summed.
 __device__ __forceinline__ void merge_ml(float& M, double& L, float m2, double l2) {
   if (m2 == -INFINITY) return;
@@ -303,55 +316,77 @@ __device__ __forceinline__ void merge_ml(float& M, double& L, float m2, double l
 }
 
 
-// Load `ncol` (16, 32, 48 or 64) fp32 columns of this warp's 32 TMEM lanes
-// starting at taddr into x[0..ncol).  Completion: KVC_TMEM_WAIT_LD64(x).
-__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&x)[64], int ncol) {
-  if (ncol == 64) {
-    KVC_TMEM_LD64(taddr, x);
-  } else if (ncol == 48) {
-    KVC_TMEM_LD32(taddr, x);
-    KVC_TMEM_LD16(taddr + 32, (x + 32));
-  } else if (ncol == 32) {
+// Load `ncol` (16 or 32) fp32 columns of this warp's 32 TMEM lanes starting
+// at taddr into x[0..ncol).  Completion: KVC_TMEM_WAIT_LD32(x).
+__device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&x)[kCols], int ncol) {
+  if (ncol == 32) {
     KVC_TMEM_LD32(taddr, x);
   } else {
     KVC_TMEM_LD16(taddr, x);
   }
 }
 
-// sum_e 2^(x[e]*c + off) over 64 values, 8 independent accumulators
-__device__ __forceinline__ float sum_ex2_64(const uint32_t (&x)[64], float c, float off) {
+// Walk columns [0, ncols) of this warp's 32 lanes of one accumulator in
+// groups of kCols: the next group's TMEM load is in flight while the current
+// one is processed (proc(gi, x)); release() runs as soon as the last load has
+// landed, so the MMA may refill the buffer during the last group's math.
+template <class Proc, class Release>
+__device__ __forceinline__ void walk_columns(uint32_t base, int ncols, Proc&& proc, Release&& release) {
+  uint32_t xa[kCols], xb[kCols];
+  const int ng = (ncols + kCols - 1) / kCols;
+  tmem_ld_cols(base, xa, min(kCols, ncols));
+  for (int gi = 0; gi < ng; gi += 2) {
+    KVC_TMEM_WAIT_LD32(xa);
+    if (gi + 1 < ng)
+      tmem_ld_cols(base + (uint32_t)((gi + 1) * kCols), xb, min(kCols, ncols - (gi + 1) * kCols));
+    else
+      release();
+    proc(gi, xa);
+    if (gi + 1 < ng) {
+      KVC_TMEM_WAIT_LD32(xb);
+      if (gi + 2 < ng)
+        tmem_ld_cols(base + (uint32_t)((gi + 2) * kCols), xa, min(kCols, ncols - (gi + 2) * kCols));
+      else
+        release();
+      proc(gi + 1, xb);
+    }
+  }
+}
+
+// sum_e 2^(x[e]*c + off) over kCols values, 8 independent accumulators
+__device__ __forceinline__ float sum_ex2(const uint32_t (&x)[kCols], float c, float off) {
   float s8[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) s8[u] = 0.f;
 #pragma unroll
-  for (int e = 0; e < 64; ++e) s8[e & 7] += tc::ex2_approx(fmaf(__uint_as_float(x[e]), c, off));
+  for (int e = 0; e < kCols; ++e) s8[e & 7] += tc::ex2_approx(fmaf(__uint_as_float(x[e]), c, off));
   return ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
 }
 
-__device__ __forceinline__ float max_64(const uint32_t (&x)[64]) {
+__device__ __forceinline__ float max_cols(const uint32_t (&x)[kCols]) {
   float m8[8];
 #pragma unroll
   for (int u = 0; u < 8; ++u) m8[u] = -INFINITY;
 #pragma unroll
-  for (int e = 0; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(x[e]));
+  for (int e = 0; e < kCols; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(x[e]));
   return fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
 }
 
-// Pass-1 update of one row with 64 logits (raw dot products) of consecutive
+// Pass-1 update of one row with kCols logits (raw dot products) of consecutive
 // keys.  The exponentials use the row's running reference `ref` (log2
 // domain) instead of a fresh per-tile max: only when that would overflow the
 // fp32 partial sum (a logit more than ~94 above the reference) -- and on the
 // first values a row sees, when ref is -inf -- is the exact max taken and the
 // running sum rescaled.
-__device__ __forceinline__ void pass1_group(uint32_t (&x)[64], float c, float& ref, double& l) {
-  float s = sum_ex2_64(x, c, -ref);
+__device__ __forceinline__ void pass1_group(uint32_t (&x)[kCols], float c, float& ref, double& l) {
+  float s = sum_ex2(x, c, -ref);
   if (!(s < 0x1p100f)) {  // overflow, or NaN from ref = -inf
-    const float hmax = max_64(x);
+    const float hmax = max_cols(x);
     if (hmax == -INFINITY) return;  // every key masked
     const float nr = fmaxf(ref, hmax * c);
     if (ref != -INFINITY) l *= (double)exp2f(ref - nr);
     ref = nr;
-    s = sum_ex2_64(x, c, -ref);
+    s = sum_ex2(x, c, -ref);
   }
   l += (double)s;
 }
@@ -395,75 +430,58 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   } else if (warp == 1) {
     if (lane == 0) issue_mmas<D, true>(a, bars, tmem, sp.qs, sp.kst, sp.ones, sp.qb, ntiles);
   } else {
-    // ---- epilogue: one row per thread and row block; halves take alternate tiles.
-    // A tile is 2 * nb1 groups of 64 columns; the next group's TMEM load is in
-    // flight while the current one is reduced.
-    const int half = (warp - 2) >> 2;
-    const int q = warp & 3;
+    // ---- epilogue: one row per thread and row block; the groups take the
+    // tiles in turn.  A tile is nb1 row blocks x 128 key columns.
+    const int grp = (warp - 2) >> 2;
+    const int q = warp & 3;         // TMEM lane quarter of this warp
     const int rl = 32 * q + lane;  // lane within a 128-row block
+    constexpr int kPerBlock = kTile / kCols;
     float m_run[2] = {-INFINITY, -INFINITY};
     double l_run[2] = {0.0, 0.0};
     const int64_t first_window_key = wk.len - a.w;  // earliest window row sees keys <= this
-    const int ng = 2 * a.nb1;
-    for (int t = half; t < ntiles; t += 2) {
+    for (int t = grp; t < ntiles; t += kGroups) {
       const int buf = t % a.nbuf;
-      if (!tc::mbar_wait(&bars->tfull[buf], (t / a.nbuf) & 1, &bars->abort)) break;
+      if (!wait_filled(a, bars, t)) break;
       tc::tc_fence_after();
       const int64_t j0 = k0 + (int64_t)t * kTile;  // first key of the tile (sequence-local)
       const bool masked = (j0 + kTile - 1 > first_window_key);
       const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * a.acc_stride);
-      auto release = [&]() {
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->tempty[buf]);
-      };
-      auto proc = [&](int gi, uint32_t(&x)[64]) {
-        const int mb = gi >> 1;
-        const int r = mb * kTile + rl;
-        if (r >= a.R) return;
-        if (masked) {
-          // keys past this row's own position (or past the sequence) get -inf
-          const int64_t lim = first_window_key + r / a.G - (j0 + (gi & 1) * 64);
+      walk_columns(
+          base, a.nb1 * kTile,
+          [&](int gi, uint32_t(&x)[kCols]) {
+            const int mb = gi / kPerBlock;
+            const int r = mb * kTile + rl;
+            if (r >= a.R) return;
+            if (masked) {
+              // keys past this row's own position (or past the sequence) get -inf
+              const int64_t lim = first_window_key + r / a.G - (j0 + (gi % kPerBlock) * kCols);
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (e > lim) x[e] = __float_as_uint(-INFINITY);
-        }
-        if (mb == 0)
-          pass1_group(x, a.c, m_run[0], l_run[0]);
-        else
-          pass1_group(x, a.c, m_run[1], l_run[1]);
-      };
-      uint32_t xa[64], xb[64];
-      KVC_TMEM_LD64(base, xa);
-      KVC_TMEM_WAIT_LD64(xa);
-      if (ng > 1) KVC_TMEM_LD64(base + 64, xb); else release();
-      proc(0, xa);
-      if (ng > 1) {
-        KVC_TMEM_WAIT_LD64(xb);
-        if (ng > 2) KVC_TMEM_LD64(base + kTile, xa); else release();
-        proc(1, xb);
-        if (ng > 2) {
-          KVC_TMEM_WAIT_LD64(xa);
-          KVC_TMEM_LD64(base + kTile + 64, xb);
-          proc(2, xa);
-          KVC_TMEM_WAIT_LD64(xb);
-          release();
-          proc(3, xb);
-        }
-      }
+              for (int e = 0; e < kCols; ++e)
+                if (e > lim) x[e] = __float_as_uint(-INFINITY);
+            }
+            if (mb == 0)
+              pass1_group(x, a.c, m_run[0], l_run[0]);
+            else
+              pass1_group(x, a.c, m_run[1], l_run[1]);
+          },
+          [&]() {
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->tempty[buf]);
+          });
     }
-    // ---- merge the two halves, then one chunk partial per row (combined by pass 2)
+    // ---- merge the groups, then one chunk partial per row (combined later)
     tc::named_bar_sync(kBarEpi, kEpiThreads);
-    if (half == 1) {
+    if (grp > 0) {
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb) {
         if (mb >= a.nb1) break;
-        sp.ex_m[mb * kTile + rl] = m_run[mb];
-        sp.ex_l[mb * kTile + rl] = l_run[mb];
+        sp.ex_m[(grp - 1) * 256 + mb * kTile + rl] = m_run[mb];
+        sp.ex_l[(grp - 1) * 256 + mb * kTile + rl] = l_run[mb];
       }
     }
     tc::named_bar_sync(kBarEpi, kEpiThreads);
-    if (half == 0 && !bars->abort) {
+    if (grp == 0 && !bars->abort) {
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb) {
         if (mb >= a.nb1) break;
@@ -471,7 +489,7 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
         if (r >= a.R) continue;
         float M = m_run[mb];
         double L = l_run[mb];
-        merge_ml(M, L, sp.ex_m[mb * kTile + rl], sp.ex_l[mb * kTile + rl]);
+        for (int o = 0; o < kGroups - 1; ++o) merge_ml(M, L, sp.ex_m[o * 256 + mb * kTile + rl], sp.ex_l[o * 256 + mb * kTile + rl]);
         const size_t slot = ((size_t)g * a.max_chunks + wk.gid) * a.Rq + r;
         a.part_m[slot] = M;
         a.part_l[slot] = L;
@@ -617,74 +635,54 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
       tc::fence_proxy_async_smem();  // visible to the MMA's operand reads
       tc::mbar_arrive(&bars->bias_ready);
     }
-    // ---- epilogue: one key per thread; halves take alternate tiles.  The R
-    // columns of a tile come in groups of <= 64; the next group's TMEM load is
-    // in flight while the current one is reduced.
-    const int half = (warp - 2) >> 2;
+    // ---- epilogue: one key per thread; the groups take the tiles in turn and
+    // walk a tile's Rn row columns kCols at a time.
+    const int grp = (warp - 2) >> 2;
     const int q = warp & 3;
     const int kl = 32 * q + lane;  // key within the tile
     const int64_t first_window_key = wk.len - a.w;
-    const int ng = (a.Rn + 63) / 64;
-    for (int t = half; t < ntiles; t += 2) {
+    for (int t = grp; t < ntiles; t += kGroups) {
       const int buf = t % a.nbuf;
-      if (!tc::mbar_wait(&bars->tfull[buf], (t / a.nbuf) & 1, &bars->abort)) break;
+      if (!wait_filled(a, bars, t)) break;
       tc::tc_fence_after();
       const int tp = ntiles - 1 - t;                    // tiles are walked backwards
       const int64_t j = k0 + (int64_t)tp * kTile + kl;  // this thread's key (sequence-local)
       const bool masked = (k0 + (int64_t)tp * kTile + kTile - 1 > first_window_key);
+      // first row that sees key j: row r = i*G + h belongs to window query i,
+      // which sees keys up to first_window_key + i
+      const int64_t lim = j - first_window_key;
+      const int rmin = lim <= 0 ? 0 : (int)std::min<int64_t>(lim * a.G, a.Rn);
       const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * a.acc_stride);
-      float s8[8];
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      walk_columns(
+          base, a.Rn,
+          [&](int gi, uint32_t(&x)[kCols]) {
+            const int col0 = gi * kCols;
+            const int ncol = min(kCols, a.Rn - col0);
+            // columns past ncol (not loaded) and, on tiles reaching into the
+            // window, keys past a row's own position get -inf, i.e. probability
+            // 0.  Both are rare and warp-uniform, so they sit outside the math
+            // loop, which stays branch-free and lets the exponentials interleave.
+            if (ncol < kCols) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) s8[u] = 0.f;
-      auto release = [&]() {
-        tc::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bars->tempty[buf]);
-      };
-      auto ncol_of = [&](int gi) { return min(64, a.Rn - gi * 64); };
-      auto proc = [&](int gi, uint32_t(&x)[64]) {
-        const int col0 = gi * 64;
-        const int ncol = ncol_of(gi);
-        // columns past ncol (not loaded) and, on tiles reaching into the window,
-        // keys past a row's own position get -inf, i.e. probability 0.  Both
-        // are rare and warp-uniform, so they sit outside the math loop, which
-        // stays branch-free and lets the 64 exponentials interleave.
-        if (ncol < 64) {
+              for (int e = 0; e < kCols; ++e)
+                if (e >= ncol) x[e] = __float_as_uint(-INFINITY);
+            }
+            if (masked) {
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if (e >= ncol) x[e] = __float_as_uint(-INFINITY);
-        }
-        if (masked) {
-          const int64_t lim = j - first_window_key;  // row r visible iff r / G >= lim
+              for (int e = 0; e < kCols; ++e)
+                if (col0 + e < rmin) x[e] = __float_as_uint(-INFINITY);
+            }
 #pragma unroll
-          for (int e = 0; e < 64; ++e)
-            if ((int64_t)((col0 + e) / a.G) < lim) x[e] = __float_as_uint(-INFINITY);
-        }
-#pragma unroll
-        for (int e = 0; e < 64; ++e) s8[e & 7] += tc::ex2_approx(__uint_as_float(x[e]) * a.c);
-      };
-      uint32_t xa[64], xb[64];
-      tmem_ld_cols(base, xa, ncol_of(0));
-      KVC_TMEM_WAIT_LD64(xa);
-      if (ng > 1) tmem_ld_cols(base + 64, xb, ncol_of(1)); else release();
-      proc(0, xa);
-      if (ng > 1) {
-        KVC_TMEM_WAIT_LD64(xb);
-        if (ng > 2) tmem_ld_cols(base + 128, xa, ncol_of(2)); else release();
-        proc(1, xb);
-        if (ng > 2) {
-          KVC_TMEM_WAIT_LD64(xa);
-          if (ng > 3) tmem_ld_cols(base + 192, xb, ncol_of(3)); else release();
-          proc(2, xa);
-          if (ng > 3) {
-            KVC_TMEM_WAIT_LD64(xb);
-            release();
-            proc(3, xb);
-          }
-        }
-      }
+            for (int e = 0; e < kCols; ++e) s4[e & 3] += tc::ex2_approx(__uint_as_float(x[e]) * a.c);
+          },
+          [&]() {
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->tempty[buf]);
+          });
       if (j < k1) {
-        const float v = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+        const float v = (s4[0] + s4[1]) + (s4[2] + s4[3]);
         const int64_t o = (int64_t)g * a.total + wk.start + j;
         a.scores[o] = v;
         if (a.accum) a.accum[o] += v;
