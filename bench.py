@@ -40,10 +40,10 @@ def algorithmic_bytes(cfg) -> dict:
     N, Hkv, d, H, w = cfg.N, cfg.Hkv, cfg.d, cfg.H, cfg.w
     kk, kt, D = cfg.k_kv, cfg.k_tsp, cfg.hidden
     return {
-        "score": N * Hkv * d * 2 + w * H * d * 2 + Hkv * N * 4,      # K once, Q_win, scores out
+        "score": N * Hkv * d * 2 + w * H * d * 2 + Hkv * N * 4 + N * 4,  # K once, Q_win, scores + head sum out
         "select_kv": Hkv * N * 4 + Hkv * kk * 4,                     # scores in, indices out
         "gather_kv": 2 * 2 * Hkv * kk * d * 2 + Hkv * kk * 4,        # K,V rows in+out, indices
-        "select_tsp": Hkv * N * 4 + kt * 4,
+        "select_tsp": N * 4 + kt * 4,                                  # head-sum row in, indices out
         "gather_hidden": 2 * kt * D * 2 + kt * 4,
     }
 
@@ -51,7 +51,7 @@ def algorithmic_bytes(cfg) -> dict:
 def layer_bytes(cfg) -> int:
     """Algorithmic bytes of the whole step (scores written once and read once)."""
     b = algorithmic_bytes(cfg)
-    return (b["score"] + b["gather_kv"] + b["gather_hidden"] + cfg.Hkv * cfg.N * 4
+    return (b["score"] + b["gather_kv"] + b["gather_hidden"] + (cfg.Hkv + 1) * cfg.N * 4
             + (cfg.Hkv * cfg.k_kv + cfg.k_tsp) * 4)
 
 
@@ -275,17 +275,16 @@ def main() -> None:
             fn()
             if evs is not None:
                 evs[name][1].record(call_stream[name])
-        timed("score", lambda: kvc.kvc_score(q, k, scores=plan.scores, ws=plan.ws_score, dev_err=plan.dev_err,
-                                             stream=st))
+        timed("score", lambda: kvc.kvc_score(q, k, scores=plan.scores, tsp=plan.tsp, ws=plan.ws_score,
+                                             dev_err=plan.dev_err, stream=st))
         ev_scores.record(st)
+        timed("select_tsp", lambda: kvc.kvc_select_topk(plan.tsp, cfg.w, cfg.pool, cfg.k_tsp, idx=plan.idx_tsp,
+                                                        ws=plan.ws_sel_tsp, stream=st))
         side.wait_event(ev_scores)
         timed("select_kv", lambda: kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_kv, idx=plan.idx_kv,
                                                        ws=plan.ws_sel_kv, stream=side))
         timed("gather_kv", lambda: kvc.kvc_gather_kv(k, v, plan.idx_kv, k_out=plan.k_c, v_out=plan.v_c,
                                                      dev_err=plan.dev_err, stream=side))
-        timed("select_tsp", lambda: kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_tsp,
-                                                        row_group=cfg.Hkv, idx=plan.idx_tsp, ws=plan.ws_sel_tsp,
-                                                        stream=st))
         timed("gather_hidden", lambda: kvc.kvc_gather_hidden(x, plan.idx_tsp.view(-1), out=plan.x_c,
                                                              dev_err=plan.dev_err, stream=st))
         ev_side.record(side)

@@ -380,7 +380,9 @@ class LayerPlan:
         self.k_c = torch.empty((Hkv, min(k_kv, n), d), dtype=bf, device=device)
         self.v_c = torch.empty_like(self.k_c) if with_v else None
         self.dev_err = torch.zeros(1, dtype=i32, device=device)
+        self.tsp = None
         if k_tsp is not None:
+            self.tsp = torch.empty((1, n), dtype=f32, device=device)  # all-head score sums
             self.ws_sel_tsp = _workspace(select_workspace_size(1, 1, n), device)
             self.idx_tsp = torch.empty((1, min(k_tsp, n)), dtype=i32, device=device)
             self.x_c = (torch.empty((min(k_tsp, n), hidden), dtype=bf, device=device)
@@ -393,22 +395,27 @@ class LayerPlan:
         """Score -> per-KV-head top-k -> K/V gather; with a TSP budget also the
         all-head top-k -> hidden-state gather.
 
-        The two selection -> gather chains only share the scores, so the K/V
-        chain runs on a side stream concurrently with the TSP chain; both
-        join the calling stream before returning.  Nothing is synchronised
-        with the host; inputs must stay alive until the work completes."""
+        The scoring call also writes the all-head sum of the scores (one row),
+        which the TSP selection ranks.  The two selection -> gather chains only
+        share the scores, so the K/V chain runs on a side stream concurrently
+        with the TSP chain (enqueued first: it leads to the longer gather);
+        both join the calling stream before returning.  Nothing is
+        synchronised with the host; inputs must stay alive until the work
+        completes."""
         main = stream if stream is not None else torch.cuda.current_stream(self.scores.device)
-        kvc_score(q_win, k, scores=self.scores, ws=self.ws_score, dev_err=self.dev_err, stream=main)
+        kvc_score(q_win, k, scores=self.scores, tsp=self.tsp, ws=self.ws_score, dev_err=self.dev_err,
+                  stream=main)
         out = LayerOutputs(self.scores, self.idx_kv, self.k_c, self.v_c)
         if self.k_tsp is None:
             self._kv_chain(k, v, main)
             return out
         self._ev_scores.record(main)
+        kvc_select_topk(self.tsp, self.w, self.pool, self.k_tsp, idx=self.idx_tsp, ws=self.ws_sel_tsp,
+                        stream=main)
         self.side.wait_event(self._ev_scores)
         self._kv_chain(k, v, self.side)
-        kvc_select_topk(self.scores, self.w, self.pool, self.k_tsp, row_group=self.Hkv, idx=self.idx_tsp,
-                        ws=self.ws_sel_tsp, stream=main)
         out.idx_tsp = self.idx_tsp
+        out.tsp = self.tsp
         if x is not None and self.x_c is not None:
             kvc_gather_hidden(x, self.idx_tsp.view(-1), out=self.x_c, dev_err=self.dev_err, stream=main)
             out.x_c = self.x_c

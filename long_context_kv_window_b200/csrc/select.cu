@@ -6,14 +6,23 @@
 // StructKV (gist.science 2604.06746) section 2.B: attention entropy, sparsity
 // (here: mass of the top 1 % keys) and variance per layer.
 //
-// Design: one thread-block cluster of kCS CTAs per ranking row.  Each CTA owns
-// a contiguous segment of the row.  The exact k-th largest key is found by a
-// three-pass radix select (11 + 11 + 10 bits of an order-preserving uint32
-// image of the fp32 score); each pass builds a shared-memory histogram per
-// CTA and the cluster sums the kCS histograms through distributed shared
-// memory.  The final compaction walks each segment in index order with a
-// block-wide scan, so the output is ascending without a sort.  Ties at the
-// threshold go to the lowest positions.
+// Design: one thread-block cluster of kCS CTAs per ranking row.  Each CTA owns a contiguous segment of the row and keeps its pooled values in
+// shared memory.  Keys are an order-preserving uint32 image of the fp32 score.
+// The exact k-th largest key is found in three cluster steps:
+//   1. every CTA samples its pooled keys; the cluster's sorted sample brackets
+//      the k-th largest key with a key window (sample quantiles around k/L);
+//   2. a 1024-bin histogram over that window (one bin below, one above) is
+//      summed through distributed shared memory and gives the bin holding the
+//      k-th largest key -- typically a few dozen keys, however concentrated
+//      the scores are (a fixed-digit radix would see one bin hold most keys);
+//   3. those candidate keys, with their positions, are gathered into every
+//      CTA, which picks the threshold itself and, from the positions, knows
+//      how many selected keys precede each of its warps -- the
+//      order-preserving compaction (ascending positions) then needs no
+//      further exchange.  Ties at the threshold go to the lowest positions.
+// If the window misses (the k-th key lies outside it) or its bin holds more
+// than kCandMax keys (heavy ties), a plain radix select runs cluster-wide
+// instead (11 + 11 + 10 bits).
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -31,7 +40,10 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kCS = 8;          // CTAs per ranking row (portable cluster size)
 constexpr int kMaxHalf = 32;    // pool_kernel <= 65
 constexpr int kBins = 2048;     // radix bins of the first two passes
-constexpr int kPerTile = 4;     // elements per thread in the compaction tiles
+constexpr int kWinBins = 1024;  // bins of the windowed histogram
+constexpr int kWin = kWinBins - 2;  // its interior bins (bin 0: below the window; last: above)
+constexpr int kSampleTotal = 256;   // sampled keys per ranking row
+constexpr int kCandMax = 1024;      // largest threshold bin resolved from a candidate list
 
 __device__ __forceinline__ uint32_t order_key(float v) {
   const uint32_t b = __float_as_uint(v);
@@ -79,49 +91,20 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* warp_t
   return warp_tmp[warp] + x - v;
 }
 
-// Sum of this CTA's local hist[lo+1 .. nbins) (all threads get it).
-__device__ __forceinline__ uint32_t local_count_above(RadixShared& sh, int buf, int nbins, uint32_t lo) {
-  uint32_t mine = 0;
-  for (int b = threadIdx.x; b < nbins; b += kThreads)
-    if ((uint32_t)b > lo) mine += (uint32_t)sh.hist[buf][b];
-  uint32_t total;
-  block_excl_scan(mine, sh.warp_tmp, &total);
-  return total;
-}
-
-// After every CTA of the cluster filled hist[buf] (and a cluster barrier),
-// sum the kCS histograms and find the bin that holds the want-th largest
-// candidate: count(bins above) < want <= count(bins above) + tot[bin].
-// Bins are visited from the top.  Returns through sh.found_*.
-__device__ void cluster_find_bucket(cg::cluster_group& cluster, RadixShared& sh, int buf, int nbins,
-                                    uint32_t want) {
-  // 16-byte loads of every rank's histogram, all issued before the sum: one
-  // round trip through distributed shared memory
-  for (int v4 = threadIdx.x; v4 < nbins / 4; v4 += kThreads) {
-    int4 part[kCS];
-#pragma unroll
-    for (int c = 0; c < kCS; ++c) part[c] = reinterpret_cast<const int4*>(cluster.map_shared_rank(&sh.hist[buf][0], c))[v4];
-    int4 acc = part[0];
-#pragma unroll
-    for (int c = 1; c < kCS; ++c) {
-      acc.x += part[c].x;
-      acc.y += part[c].y;
-      acc.z += part[c].z;
-      acc.w += part[c].w;
-    }
-    reinterpret_cast<int4*>(sh.tot)[v4] = acc;
-  }
-  __syncthreads();
+// Bin of histogram h (nbins = 1024 or 2048, shared memory) that holds the
+// want-th largest key: count(bins above) < want <= count(bins above) + h[bin].
+// Bins are visited from the top.  Returns through sh.found_*; all threads call.
+__device__ void scan_find(RadixShared& sh, const int* h, int nbins, uint32_t want) {
   // thread t owns the group of bins (kThreads-1-t): higher t = lower bins
   const int per = nbins / kThreads;  // 1 or 2
   const int grp = kThreads - 1 - threadIdx.x;
   uint32_t mine = 0;
-  for (int q = 0; q < per; ++q) mine += sh.tot[grp * per + q];
+  for (int q = 0; q < per; ++q) mine += h[grp * per + q];
   uint32_t total;
   uint32_t above = block_excl_scan(mine, sh.warp_tmp, &total);
   for (int q = per - 1; q >= 0; --q) {
     const int bin = grp * per + q;
-    const uint32_t c = sh.tot[bin];
+    const uint32_t c = h[bin];
     if (above < want && want <= above + c) {
       sh.found_bucket = bin;
       sh.found_rem = want - above;
@@ -130,6 +113,57 @@ __device__ void cluster_find_bucket(cg::cluster_group& cluster, RadixShared& sh,
   }
   __syncthreads();
 }
+
+// After every CTA of the cluster filled hist[buf] (and a cluster barrier),
+// sum the CS histograms into tot and find the bin that holds the want-th
+// largest key of the cluster (scan_find).
+// 16 bytes of CTA `rank`'s shared memory at this CTA's shared address `local`.
+__device__ __forceinline__ int4 ld_dsmem_v4(uint32_t local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local), "r"(rank));
+  int4 v;
+  asm volatile("ld.shared::cluster.v4.s32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "r"(remote)
+               : "memory");
+  return v;
+}
+
+template <int CS>
+__device__ void cluster_find_bucket(cg::cluster_group& cluster, RadixShared& sh, int buf, int nbins,
+                                    uint32_t want) {
+  // 16-byte loads of every rank's histogram, all issued before the sum: one
+  // round trip through distributed shared memory
+  for (int v4 = threadIdx.x; v4 < nbins / 4; v4 += kThreads) {
+    int4 part[CS];
+    const uint32_t local = (uint32_t)__cvta_generic_to_shared(&sh.hist[buf][4 * v4]);
+#pragma unroll
+    for (int c = 0; c < CS; ++c) part[c] = ld_dsmem_v4(local, (uint32_t)c);
+    int4 acc = part[0];
+#pragma unroll
+    for (int c = 1; c < CS; ++c) {
+      acc.x += part[c].x;
+      acc.y += part[c].y;
+      acc.z += part[c].z;
+      acc.w += part[c].w;
+    }
+    reinterpret_cast<int4*>(sh.tot)[v4] = acc;
+  }
+  __syncthreads();
+  scan_find(sh, sh.tot, nbins, want);
+}
+
+__device__ __forceinline__ uint32_t warp_sum(uint32_t v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Split cluster barrier: arrive once this CTA reads no other CTA's shared
+// memory any more, wait before exiting (no CTA may leave while another still
+// reads its shared memory).
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // --------------------------------------------------------------------------
 // selection
@@ -151,36 +185,100 @@ struct SelArgs {
   bool vals_packed;        // vals_g indexed by packed token offset (varlen / workspace)
   bool smem_vals;          // keep this CTA's pooled segment in shared memory
   int64_t seg_cap;         // smem mode: longest segment the dynamic smem holds
+  int v_off;               // smem mode: words of dynamic smem before the pooled values
   int out_rows;
   int32_t* err;
 };
 
 struct SelShared {
   RadixShared rx;
-  uint32_t cnt_gt, cnt_eq;  // this CTA's counts for the output phase
+  uint2 cand[kCandMax];            // candidate list: (key, segment position), rank by rank
+  uint32_t sample[kSampleTotal];   // this CTA's sampled keys
+  uint32_t sall[kSampleTotal];     // the cluster's samples (rank order), then ...
+  uint32_t ssort[kSampleTotal];    // ... sorted, largest first
+  uint32_t ns;                     // this CTA's sample count
+  uint32_t soff[kCS + 1];      // sample slots per rank
+  uint32_t cand_off[kCS + 1];  // candidate slots per rank, total last
+  uint32_t cand_n;                 // candidate slots this CTA has taken
+  uint32_t above;                  // this CTA's keys in bins above the threshold bin
+  uint32_t T, need_eq;             // threshold resolved from the candidate list
+  uint32_t cnt_gt, cnt_eq;         // plain-radix path: this CTA's keys above / equal to the threshold
+  uint32_t g_prev, e_prev;         // plain-radix path: the same summed over the lower ranks
+  uint32_t warp_gt[kWarps], warp_eq[kWarps];
+  uint32_t red[2][kWarps];
 };
 
-// Histogram increment.  Contention is modest (a CTA's 16K keys spread over
-// tens of first-pass bins; later passes only see the keys of one bucket), so
-// plain shared-memory atomics beat warp-level match/aggregate here.
+// Histogram increment (shared-memory atomics; callers spread the lanes of a
+// warp over distant positions, whose keys rarely share a bin).
 __device__ __forceinline__ void hist_add(int* hist, uint32_t bin, bool active) {
   if (active) atomicAdd(&hist[bin], 1);
 }
 
-// Dynamic shared memory of the selection kernel: the staged row sums of the
-// segment plus halo, and the pooled values of the segment (smem mode).
-__host__ __device__ inline size_t sel_dyn_smem(int64_t seg, int half, bool smem_vals) {
-  return smem_vals ? (size_t)(2 * seg + 2 * half + 16) * sizeof(float) : 0;
+// Block-wide sums of two counters (all threads get both).
+__device__ __forceinline__ void block_sum2(uint32_t& x, uint32_t& y, uint32_t (*red)[kWarps]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  x = warp_sum(x);
+  y = warp_sum(y);
+  if (lane == 0) {
+    red[0][warp] = x;
+    red[1][warp] = y;
+  }
+  __syncthreads();
+  x = warp_sum(red[0][lane]);
+  y = warp_sum(red[1][lane]);
+  __syncthreads();
 }
 
-__global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kThreads, 1)
-select_kernel(const SelArgs a) {
+// Warp-wide exclusive prefix sum.
+__device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v) {
+  const int lane = threadIdx.x & 31;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  return x - v;
+}
+
+// Four consecutive pooled values v[p .. p+3] as order keys; positions at or
+// past `end` give 0 (the caller masks them).
+__device__ __forceinline__ void load_keys4(const float* v, int p, int end, bool vec, uint32_t (&key)[4]) {
+  if (vec && p + 4 <= end) {
+    const float4 f = *reinterpret_cast<const float4*>(v + p);
+    key[0] = order_key(f.x);
+    key[1] = order_key(f.y);
+    key[2] = order_key(f.z);
+    key[3] = order_key(f.w);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) key[q] = p + q < end ? order_key(v[p + q]) : 0u;
+  }
+}
+
+// The i-th position of a 1024-position block, spread so that the lanes of a
+// warp sit 32 positions apart (their keys rarely share a histogram bin).
+__device__ __forceinline__ int spread_index(int warp, int lane) { return lane * 32 + ((warp + lane) & 31); }
+
+// Dynamic shared memory of the selection kernel (words): [candidate list,
+// which first holds the staged row sums of the segment plus halo][pooled
+// values of the segment (smem mode)].
+__host__ __device__ inline int stage_halo(int half) { return (half + 3) & ~3; }
+inline size_t round4(int64_t x) { return (size_t)((x + 3) & ~int64_t(3)); }
+inline size_t sel_v_words(int64_t seg) { return round4(seg) + 4; }
+inline size_t sel_stage_words(int64_t seg, int half) { return round4(seg) + 2 * stage_halo(half) + 4; }
+// Positions per CTA: a multiple of 4, so that segments start 16-byte aligned.
+__host__ __device__ inline int64_t sel_segment(int64_t L, int cs) { return ((L + cs - 1) / cs + 3) & ~int64_t(3); }
+
+template <int CS>
+__global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
   __shared__ SelShared sh;
-  extern __shared__ float dyn[];
+  extern __shared__ __align__(16) float dyn[];
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
   const int o = blockIdx.y;
   const int b = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool varlen = a.cu != nullptr;
 
   int64_t start = 0, len = a.n;
@@ -190,7 +288,7 @@ select_kernel(const SelArgs a) {
     len = (int64_t)a.cu[b + 1] - start;
     bad = (start < 0 || len < a.w);
     // a sequence longer than the max_seqlen the launch was sized for
-    if (!bad && a.smem_vals && (len - a.w + kCS - 1) / kCS > a.seg_cap) bad = true;
+    if (!bad && a.smem_vals && sel_segment(len - a.w, CS) > a.seg_cap) bad = true;
   }
   const int64_t orow = varlen ? ((int64_t)b * a.out_rows + o) : o;
   int32_t* out = a.idx + orow * (varlen ? a.k : a.idx_row_stride);
@@ -201,30 +299,30 @@ select_kernel(const SelArgs a) {
       set_dev_err(a.err, KVC_DEV_ERR_SEQLENS);
       if (a.counts && o == 0) a.counts[b] = 0;
     }
-    for (int64_t t = (int64_t)crank * kThreads + threadIdx.x; t < kout; t += (int64_t)kCS * kThreads)
+    for (int64_t t = (int64_t)crank * kThreads + threadIdx.x; t < kout; t += (int64_t)CS * kThreads)
       out[t] = -1;
     return;
   }
   const int64_t m = a.k < len ? a.k : len;  // positions kept in this sequence
   if (varlen && a.counts && o == 0 && crank == 0 && threadIdx.x == 0) a.counts[b] = (int32_t)m;
   // padding of short sequences (varlen rows have k entries)
-  for (int64_t t = m + (int64_t)crank * kThreads + threadIdx.x; t < kout; t += (int64_t)kCS * kThreads)
+  for (int64_t t = m + (int64_t)crank * kThreads + threadIdx.x; t < kout; t += (int64_t)CS * kThreads)
     out[t] = -1;
 
   const int64_t L = len - a.w;
   const int64_t kk = a.k - a.w;
   if (a.k >= len) {  // keep everything
-    for (int64_t t = (int64_t)crank * kThreads + threadIdx.x; t < len; t += (int64_t)kCS * kThreads)
+    for (int64_t t = (int64_t)crank * kThreads + threadIdx.x; t < len; t += (int64_t)CS * kThreads)
       out[t] = (int32_t)t;
   } else {
-    for (int64_t t = (int64_t)crank * kThreads + threadIdx.x; t < a.w; t += (int64_t)kCS * kThreads)
+    for (int64_t t = (int64_t)crank * kThreads + threadIdx.x; t < a.w; t += (int64_t)CS * kThreads)
       out[kk + t] = (int32_t)(L + t);
   }
   const bool need_rank = (a.k < len) && kk > 0;
   if (!need_rank && a.vals_g == nullptr) return;  // nothing to rank, nothing to report
 
   // ---- segment of this CTA: row sums (+halo), then pooled values -------------
-  const int64_t seg = (L + kCS - 1) / kCS;
+  const int64_t seg = sel_segment(L, CS);
   const int64_t s0 = (int64_t)crank * seg < L ? (int64_t)crank * seg : L;
   const int64_t s1 = s0 + seg < L ? s0 + seg : L;
   const int nseg = (int)(s1 - s0);
@@ -233,89 +331,137 @@ select_kernel(const SelArgs a) {
   const float* rows0 = a.scores + (int64_t)o * a.row_group * a.row_stride + start;
   float* gvals = a.vals_g ? a.vals_g + (int64_t)o * a.vals_stride + (a.vals_packed ? start : 0) : nullptr;
   // pooled values of the segment, indexed 0..nseg-1 (shared or global memory)
-  float* v = a.smem_vals ? dyn + ((nseg + 2 * half + 8 + 3) & ~3) : gvals + s0;  // 16-B aligned in smem
+  float* v = a.smem_vals ? dyn + a.v_off : gvals + s0;
 
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[0][i] = 0;
-  __syncthreads();
+  if (threadIdx.x == 0) sh.cand_n = 0;
 
-  constexpr int kU = 4;
   if (a.smem_vals) {
-    float* stage = dyn;  // row sums over [s0 - half, s1 + half)
-    const int span = nseg + 2 * half;
-    for (int t0 = 0; t0 < span; t0 += kThreads * kU) {
-      float acc[kU];
+    // row sums R over [s0 - hs, s0 + nseg4 + hs + 4) into the stage, zero
+    // outside [0, L)
+    const int hs = stage_halo(half);
+    const int nseg4 = (nseg + 3) & ~3;
+    float* stage = dyn;
+    const int64_t p0 = s0 - hs;
+    const int span = nseg4 + 2 * hs + 4;
+    const bool vec_in = ((reinterpret_cast<uintptr_t>(rows0) & 15) == 0) && (a.row_stride & 3) == 0 && (p0 & 3) == 0;
+    if (vec_in) {
+      // 16-byte loads, four per thread and row in flight
+      float4* st4 = reinterpret_cast<float4*>(stage);
+      const int n4 = span / 4;
+      constexpr int kU = 4;
+      for (int i0 = threadIdx.x; i0 < n4; i0 += kThreads * kU) {
+        float4 acc[kU];
 #pragma unroll
-      for (int u = 0; u < kU; ++u) acc[u] = 0.f;
-      for (int r = 0; r < a.row_group; ++r) {
-        const float* row = rows0 + (int64_t)r * a.row_stride;
+        for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int r = 0; r < a.row_group; ++r) {
+          const float* row = rows0 + (int64_t)r * a.row_stride;
+          float4 x[kU];
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            const int i = i0 + u * kThreads;
+            const int64_t pos = p0 + 4 * (int64_t)i;
+            x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < n4 && pos >= 0 && pos + 4 <= L) {
+              x[u] = *reinterpret_cast<const float4*>(row + pos);
+            } else if (i < n4) {
+              if (pos + 0 >= 0 && pos + 0 < L) x[u].x = row[pos + 0];
+              if (pos + 1 >= 0 && pos + 1 < L) x[u].y = row[pos + 1];
+              if (pos + 2 >= 0 && pos + 2 < L) x[u].z = row[pos + 2];
+              if (pos + 3 >= 0 && pos + 3 < L) x[u].w = row[pos + 3];
+            }
+          }
+#pragma unroll
+          for (int u = 0; u < kU; ++u) {
+            acc[u].x += x[u].x;
+            acc[u].y += x[u].y;
+            acc[u].z += x[u].z;
+            acc[u].w += x[u].w;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+          if (i0 + u * kThreads < n4) st4[i0 + u * kThreads] = acc[u];
+      }
+    } else {
+      // unaligned rows: coalesced 4-byte loads, eight positions per thread in flight
+      constexpr int kU = 8;
+      for (int t0 = threadIdx.x; t0 < span; t0 += kThreads * kU) {
+        float acc[kU];
+        bool ok[kU];
 #pragma unroll
         for (int u = 0; u < kU; ++u) {
-          const int t = t0 + u * kThreads + threadIdx.x;
-          const int64_t pos = s0 - half + t;
-          if (t < span && pos >= 0 && pos < L) acc[u] += row[pos];
+          const int64_t pos = p0 + t0 + u * kThreads;
+          ok[u] = t0 + u * kThreads < span && pos >= 0 && pos < L;
+          acc[u] = 0.f;
         }
-      }
+        for (int r = 0; r < a.row_group; ++r) {
+          const float* row = rows0 + (int64_t)r * a.row_stride + p0 + t0;
 #pragma unroll
-      for (int u = 0; u < kU; ++u) {
-        const int t = t0 + u * kThreads + threadIdx.x;
-        if (t < span) stage[t] = acc[u];
+          for (int u = 0; u < kU; ++u)
+            if (ok[u]) acc[u] += row[u * kThreads];
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u)
+          if (t0 + u * kThreads < span) stage[t0 + u * kThreads] = acc[u];
       }
     }
     __syncthreads();
     // v[t] = sum of the p staged row sums around t.  Ranking uses this sum: the
     // average differs by the constant factor 1/p, a monotone map, so the order
     // (ties to the lower position) is the same; the average itself is only
-    // formed for the optional pooled output.  Four consecutive outputs per
-    // thread and round share one register window of 4 + 2*half staged values.
-    const int span_w = 4 + 2 * half;
-    for (int base = 0; base < nseg; base += 4 * kThreads) {
-      const int t0 = base + 4 * threadIdx.x;
-      float sums[4] = {0.f, 0.f, 0.f, 0.f};
-      if (half <= 8) {
-        float win[4 + 16];
+    // formed for the optional pooled output.  Each thread forms four
+    // consecutive outputs from 16-byte shared-memory loads (lanes 128
+    // positions apart: no bank conflicts).
+    const float4* st4 = reinterpret_cast<const float4*>(stage);
+    float4* v4 = reinterpret_cast<float4*>(v);
+    const int nv = nseg4 / 4;
+    for (int i = spread_index(warp, lane); i < nv; i += kThreads) {
+      float sums[4];
+      if (hs == 0) {
+        const float4 x = st4[i];
+        sums[0] = x.x;
+        sums[1] = x.y;
+        sums[2] = x.z;
+        sums[3] = x.w;
+      } else if (hs == 4) {
+        const float4 x0 = st4[i], x1 = st4[i + 1], x2 = st4[i + 2];
+        const float win[12] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w, x2.x, x2.y, x2.z, x2.w};
 #pragma unroll
-        for (int q = 0; q < 4 + 16; ++q) win[q] = (q < span_w && t0 + q < span) ? stage[t0 + q] : 0.f;
+        for (int u = 0; u < 4; ++u) {
+          float sum = 0.f;
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int q = 0; q < 17; ++q)
-            if (q <= 2 * half) sums[u] += win[u + q];
+          for (int q = 0; q <= 8; ++q)
+            if (q >= 4 - half && q <= 4 + half) sum += win[u + q];
+          sums[u] = sum;
+        }
       } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          for (int q = 0; q <= 2 * half; ++q)
-            if (t0 + u + q < span) sums[u] += stage[t0 + u + q];
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int t = t0 + u;
-        const bool in = t < nseg;
-        if (in) {
-          v[t] = sums[u];
-          if (gvals) gvals[s0 + t] = (a.pool == 1) ? sums[u] : sums[u] / pool_div;
+        for (int u = 0; u < 4; ++u) {
+          float sum = 0.f;
+          for (int q = -half; q <= half; ++q) sum += stage[4 * i + u + hs + q];
+          sums[u] = sum;
         }
-        if (need_rank) hist_add(sh.rx.hist[0], order_key(sums[u]) >> 21, in);
+      }
+      v4[i] = make_float4(sums[0], sums[1], sums[2], sums[3]);
+      if (gvals) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          if (4 * i + u < nseg) gvals[s0 + 4 * i + u] = (a.pool == 1) ? sums[u] : sums[u] / pool_div;
       }
     }
   } else {
     // long rows: pooled values go straight to global memory (L2-resident)
-    for (int base = 0; base < nseg; base += kThreads) {
-      const int t = base + threadIdx.x;
-      const bool in = t < nseg;
-      float val = 0.f;
-      if (in) {
-        float sum = 0.f;
-        for (int q = -half; q <= half; ++q) {
-          const int64_t pos = s0 + t + q;
-          if (pos < 0 || pos >= L) continue;
-          float rs = 0.f;
-          for (int r = 0; r < a.row_group; ++r) rs += rows0[(int64_t)r * a.row_stride + pos];
-          sum += rs;
-        }
-        val = sum;  // ranked as the pooled sum (see the shared-memory path)
-        v[t] = val;
+    for (int t = threadIdx.x; t < nseg; t += kThreads) {
+      float sum = 0.f;
+      for (int q = -half; q <= half; ++q) {
+        const int64_t pos = s0 + t + q;
+        if (pos < 0 || pos >= L) continue;
+        float rs = 0.f;
+        for (int r = 0; r < a.row_group; ++r) rs += rows0[(int64_t)r * a.row_stride + pos];
+        sum += rs;
       }
-      if (need_rank) hist_add(sh.rx.hist[0], order_key(val) >> 21, in);
+      v[t] = sum;  // ranked as the pooled sum (see the shared-memory path)
     }
   }
   // global-memory mode keeps the pooled sums in the caller's buffer while
@@ -330,128 +476,300 @@ select_kernel(const SelArgs a) {
     finish_gvals();
     return;
   }
+  __syncthreads();  // (global mode: each thread reads values other threads wrote)
 
-  // ---- radix passes ---------------------------------------------------------
+  // ---- 1. sample -> key window --------------------------------------------------
+  {
+    const int per = kSampleTotal / CS;
+    const int nsc = nseg < per ? nseg : per;
+    if (threadIdx.x < nsc) sh.sample[threadIdx.x] = order_key(v[((2 * (int64_t)threadIdx.x + 1) * nseg) / (2 * nsc)]);
+    if (threadIdx.x == 0) sh.ns = (uint32_t)nsc;
+  }
   cluster.sync();
-  cluster_find_bucket(cluster, sh.rx, 0, kBins, (uint32_t)kk);
-  const uint32_t b1 = sh.rx.found_bucket;
-  uint32_t want = sh.rx.found_rem;
-  // keys of this CTA above bucket b1 are selected whatever the finer bits
-  const uint32_t gt1 = local_count_above(sh.rx, 0, kBins, b1);
-
-  for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[1][i] = 0;
+  if (warp == 0) {
+    const uint32_t c = lane < CS ? cluster.map_shared_rank(&sh, lane)->ns : 0u;
+    const uint32_t ex = warp_excl_scan(c);
+    if (lane <= CS) sh.soff[lane] = ex;
+  }
   __syncthreads();
-  for (int base = 0; base < nseg; base += kThreads) {
-    const int t = base + threadIdx.x;
-    const uint32_t key = t < nseg ? order_key(v[t]) : 0u;
-    hist_add(sh.rx.hist[1], (key >> 10) & 2047u, t < nseg && (key >> 21) == b1);
+  const uint32_t ns = sh.soff[CS];
+  if (threadIdx.x < ns) {
+    int r = 0;
+#pragma unroll
+    for (int q = 1; q < CS; ++q) r += sh.soff[q] <= threadIdx.x;
+    sh.sall[threadIdx.x] = cluster.map_shared_rank(&sh, r)->sample[threadIdx.x - sh.soff[r]];
   }
-  cluster.sync();
-  cluster_find_bucket(cluster, sh.rx, 1, kBins, want);
-  const uint32_t b2 = sh.rx.found_bucket;
-  want = sh.rx.found_rem;
-  const uint32_t pre2 = (b1 << 11) | b2;
-  const uint32_t gt2 = local_count_above(sh.rx, 1, kBins, b2);
-
-  for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[0][i] = 0;
   __syncthreads();
-  for (int base = 0; base < nseg; base += kThreads) {
-    const int t = base + threadIdx.x;
-    const uint32_t key = t < nseg ? order_key(v[t]) : 0u;
-    hist_add(sh.rx.hist[0], key & 1023u, t < nseg && (key >> 10) == pre2);
+  {
+    // rank by counting (equal keys: lower slot first), four threads per sample
+    const uint32_t i = threadIdx.x >> 2, part = threadIdx.x & 3;
+    const uint32_t mine = i < ns ? sh.sall[i] : 0u;
+    uint32_t c = 0;
+    if (i < ns) {
+#pragma unroll 4
+      for (uint32_t j = part; j < ns; j += 4) {
+        const uint32_t x = sh.sall[j];
+        c += (x > mine) || (x == mine && j < i);
+      }
+    }
+    c += __shfl_xor_sync(0xffffffffu, c, 1);
+    c += __shfl_xor_sync(0xffffffffu, c, 2);
+    if (i < ns && part == 0) sh.ssort[c] = mine;
   }
-  cluster.sync();
-  cluster_find_bucket(cluster, sh.rx, 0, 1024, want);
-  const uint32_t b3 = sh.rx.found_bucket;
-  const uint32_t T = (pre2 << 10) | b3;
-  const uint32_t need_eq = sh.rx.found_rem;  // how many keys == T are taken (lowest positions)
+  __syncthreads();
+  // the kk-th largest key sits near sample index ns*kk/L; the window spans
+  // `margin` sample places to either side
+  const int64_t tr = (int64_t)ns * kk / L;
+  const int64_t margin = 4 + ns / 16;
+  const uint32_t hi_key = tr - margin >= 0 ? sh.ssort[tr - margin] : 0xFFFFFFFFu;
+  const uint32_t lo_key = tr + margin < (int64_t)ns ? sh.ssort[tr + margin] : 0u;
+  int wsh = 0;
+  while (((hi_key - lo_key) >> wsh) >= (uint32_t)kWin) ++wsh;
+  auto wbin = [&](uint32_t key) -> uint32_t {
+    if (key < lo_key) return 0u;
+    const uint32_t d = (key - lo_key) >> wsh;
+    return d >= (uint32_t)kWin ? (uint32_t)(kWinBins - 1) : d + 1u;
+  };
 
-  // ---- counts per CTA (from the local histograms), then cluster prefix ------
-  const uint32_t gt3 = local_count_above(sh.rx, 0, 1024, b3);
-  if (threadIdx.x == 0) {
-    sh.cnt_gt = gt1 + gt2 + gt3;
-    sh.cnt_eq = (uint32_t)sh.rx.hist[0][b3];
+  // ---- 2. windowed histogram, summed over the cluster --------------------------
+  for (int t0 = 0; t0 < nseg; t0 += kThreads) {
+    const int t = t0 + spread_index(warp, lane);
+    if (t < nseg) hist_add(sh.rx.hist[0], wbin(order_key(v[t])), true);
   }
   cluster.sync();
-  uint32_t out_base = 0, eq_seen = 0;
-  if (threadIdx.x < 32) {
-    // lanes c < crank hold rank c's counts; a warp scan gives this CTA's offset
-    const int lane = threadIdx.x;
-    uint32_t cg_ = 0, ce = 0;
-    if (lane < crank) {
-      const SelShared* r = cluster.map_shared_rank(&sh, lane);
-      cg_ = r->cnt_gt;
-      ce = r->cnt_eq;
+  cluster_find_bucket<CS>(cluster, sh.rx, 0, kWinBins, (uint32_t)kk);
+  const uint32_t b1 = sh.rx.found_bucket & (kWinBins - 1);
+  const uint32_t nc = (uint32_t)sh.rx.tot[b1];
+  const bool listed = b1 != 0u && b1 != (uint32_t)(kWinBins - 1) && nc <= (uint32_t)kCandMax;  // uniform
+
+  // compaction layout: warp w owns positions [w*sub, (w+1)*sub) of the
+  // segment, four consecutive positions per lane and step
+  const int sub = (nseg + kThreads * 4 - 1) / (kThreads * 4) * 128;
+  const int w0 = min(nseg, warp * sub), w1 = min(nseg, w0 + sub);
+  const bool vec = a.smem_vals;  // 16-byte aligned pooled values
+
+  uint32_t T, need_eq;              // threshold key; how many keys == T are taken
+  uint32_t g_prev = 0, e_prev = 0;  // keys > T / == T in the lower ranks
+  if (listed) {
+    // ---- 3. candidates (keys of bin b1) with positions, rank by rank ----------
+    if (warp == 0) {
+      const uint32_t c = lane < CS ? (uint32_t)cluster.map_shared_rank(&sh.rx.hist[0][0], lane)[b1] : 0u;
+      const uint32_t ex = warp_excl_scan(c);
+      if (lane <= CS) sh.cand_off[lane] = ex;
     }
-    // equal keys are taken by rank order: rank c takes min(ce, quota left)
-    uint32_t ce_before = ce;
+    __syncthreads();
+    const uint32_t off = sh.cand_off[crank];
+    uint32_t above_w = 0;  // keys of this warp's range in bins above b1
+    for (int p = w0 + 4 * lane; p - 4 * lane < w1; p += 128) {
+      uint32_t key[4];
+      load_keys4(v, p, w1, vec, key);
+      uint32_t nmine = 0;
+      bool is[4];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, ce_before, o);
-      if (lane >= o) ce_before += y;
+      for (int q = 0; q < 4; ++q) {
+        const uint32_t bin = wbin(key[q]);
+        const bool in = p + q < w1;
+        above_w += in && bin > b1;
+        is[q] = in && bin == b1;
+        nmine += is[q];
+      }
+      if (__any_sync(0xffffffffu, nmine != 0)) {  // candidates are rare: most steps skip this
+        const uint32_t ex = warp_excl_scan(nmine);
+        const uint32_t tot = __shfl_sync(0xffffffffu, ex + nmine, 31);
+        uint32_t base = 0;
+        if (lane == 0) base = atomicAdd(&sh.cand_n, tot);
+        base = __shfl_sync(0xffffffffu, base, 0) + off + ex;
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (is[q]) sh.cand[base++] = make_uint2(key[q], (uint32_t)(p + q));
+      }
     }
-    ce_before -= ce;  // exclusive
-    const uint32_t take = ce_before < need_eq ? min(need_eq - ce_before, ce) : 0u;
-    uint32_t sum = cg_ + take;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-    uint32_t eqs = ce;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) eqs += __shfl_xor_sync(0xffffffffu, eqs, o);
+    above_w = warp_sum(above_w);
     if (lane == 0) {
-      sh.rx.found_bucket = sum;  // reused as scratch: output offset of this CTA
-      sh.rx.found_rem = eqs;     // equal keys in earlier ranks
+      sh.warp_gt[warp] = above_w;
+      sh.warp_eq[warp] = 0;
     }
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t t = warp_sum(sh.warp_gt[lane]);
+      if (lane == 0) sh.above = t;
+    }
+    cluster.sync();  // every rank's candidates and `above` are published
+    // gather the other ranks' candidates
+    const uint32_t own_n = sh.cand_off[crank + 1] - off;
+    for (uint32_t i = threadIdx.x; i < nc; i += kThreads) {
+      if (i >= off && i < off + own_n) continue;
+      int r = 0;
+#pragma unroll
+      for (int q = 1; q < CS; ++q) r += sh.cand_off[q] <= i;
+      sh.cand[i] = cluster.map_shared_rank(&sh.cand[0], r)[i];
+    }
+    uint32_t above_prev = 0;
+    if (warp == 0) above_prev = warp_sum(lane < crank ? cluster.map_shared_rank(&sh, lane)->above : 0u);
+    __syncthreads();
+    // the want-th largest candidate: rank by counting, four threads per
+    // candidate (nc <= kCandMax = kThreads)
+    {
+      const uint32_t want = sh.rx.found_rem;
+      for (uint32_t i0 = 0; i0 < nc; i0 += kThreads / 4) {
+        const uint32_t i = i0 + (threadIdx.x >> 2), part = threadIdx.x & 3;
+        const uint32_t mine = i < nc ? sh.cand[i].x : 0u;
+        uint32_t gt = 0, eq = 0;
+        if (i < nc) {
+#pragma unroll 4
+          for (uint32_t j = part; j < nc; j += 4) {
+            const uint32_t x = sh.cand[j].x;
+            gt += x > mine;
+            eq += x == mine;
+          }
+        }
+        gt += __shfl_xor_sync(0xffffffffu, gt, 1);
+        gt += __shfl_xor_sync(0xffffffffu, gt, 2);
+        eq += __shfl_xor_sync(0xffffffffu, eq, 1);
+        eq += __shfl_xor_sync(0xffffffffu, eq, 2);
+        if (i < nc && part == 0 && gt < want && want <= gt + eq) {
+          sh.T = mine;
+          sh.need_eq = want - gt;
+        }
+      }
+    }
+    __syncthreads();
+    T = sh.T;
+    need_eq = sh.need_eq;
+    // this CTA's candidates per compaction warp; the lower ranks' candidates
+    for (uint32_t i = off + threadIdx.x; i < off + own_n; i += kThreads) {
+      const uint2 c = sh.cand[i];
+      const int w = sub > 0 ? (int)c.y / sub : 0;
+      if (c.x > T) atomicAdd(&sh.warp_gt[w], 1u);
+      if (c.x == T) atomicAdd(&sh.warp_eq[w], 1u);
+    }
+    uint32_t gt = threadIdx.x == 0 ? above_prev : 0u, eq = 0;
+    for (uint32_t i = threadIdx.x; i < off; i += kThreads) {
+      const uint32_t x = sh.cand[i].x;
+      gt += x > T;
+      eq += x == T;
+    }
+    block_sum2(gt, eq, sh.red);  // (also completes the per-warp atomics)
+    g_prev = gt;
+    e_prev = eq;
+  } else {
+    // ---- the window missed, or heavy ties: plain radix select, cluster-wide ----
+    // (hist[1] and hist[0] alternate: a CTA rewrites a histogram only after the
+    // cluster barrier that follows every rank's last read of it)
+    uint32_t want = (uint32_t)kk;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[1][i] = 0;
+    __syncthreads();
+    for (int t0 = 0; t0 < nseg; t0 += kThreads) {
+      const int t = t0 + spread_index(warp, lane);
+      if (t < nseg) hist_add(sh.rx.hist[1], order_key(v[t]) >> 21, true);
+    }
+    cluster.sync();
+    cluster_find_bucket<CS>(cluster, sh.rx, 1, kBins, want);
+    const uint32_t r1 = sh.rx.found_bucket & (kBins - 1);
+    want = sh.rx.found_rem;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[0][i] = 0;
+    __syncthreads();
+    for (int t0 = 0; t0 < nseg; t0 += kThreads) {
+      const int t = t0 + spread_index(warp, lane);
+      const uint32_t key = t < nseg ? order_key(v[t]) : 0u;
+      hist_add(sh.rx.hist[0], (key >> 10) & 2047u, t < nseg && (key >> 21) == r1);
+    }
+    cluster.sync();
+    cluster_find_bucket<CS>(cluster, sh.rx, 0, kBins, want);
+    const uint32_t pre2 = (r1 << 11) | (sh.rx.found_bucket & (kBins - 1));
+    want = sh.rx.found_rem;
+    for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[1][i] = 0;
+    __syncthreads();
+    for (int t0 = 0; t0 < nseg; t0 += kThreads) {
+      const int t = t0 + spread_index(warp, lane);
+      const uint32_t key = t < nseg ? order_key(v[t]) : 0u;
+      hist_add(sh.rx.hist[1], key & 1023u, t < nseg && (key >> 10) == pre2);
+    }
+    cluster.sync();
+    cluster_find_bucket<CS>(cluster, sh.rx, 1, 1024, want);
+    T = (pre2 << 10) | (sh.rx.found_bucket & 1023u);
+    need_eq = sh.rx.found_rem;
+    // per-warp counts, then the per-CTA totals through the cluster
+    {
+      uint32_t gt = 0, eq = 0;
+      for (int p = w0 + 4 * lane; p < w1; p += 128) {
+        uint32_t key[4];
+        load_keys4(v, p, w1, vec, key);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          gt += p + q < w1 && key[q] > T;
+          eq += p + q < w1 && key[q] == T;
+        }
+      }
+      gt = warp_sum(gt);
+      eq = warp_sum(eq);
+      if (lane == 0) {
+        sh.warp_gt[warp] = gt;
+        sh.warp_eq[warp] = eq;
+      }
+    }
+    __syncthreads();
+    if (warp == 0) {
+      const uint32_t tg = warp_sum(sh.warp_gt[lane]), te = warp_sum(sh.warp_eq[lane]);
+      if (lane == 0) {
+        sh.cnt_gt = tg;
+        sh.cnt_eq = te;
+      }
+    }
+    cluster.sync();
+    if (warp == 0) {
+      uint32_t g = 0, e = 0;
+      if (lane < crank) {
+        const SelShared* r = cluster.map_shared_rank(&sh, lane);
+        g = r->cnt_gt;
+        e = r->cnt_eq;
+      }
+      g = warp_sum(g);
+      e = warp_sum(e);
+      if (lane == 0) {
+        sh.g_prev = g;
+        sh.e_prev = e;
+      }
+    }
+    __syncthreads();
+    g_prev = sh.g_prev;
+    e_prev = sh.e_prev;
   }
-  __syncthreads();
-  out_base = sh.rx.found_bucket;
-  eq_seen = sh.rx.found_rem;
+  cluster_arrive();  // no reads of other CTAs' shared memory from here on
 
-  // ---- order-preserving compaction -----------------------------------------
-  for (int t0 = 0; t0 < nseg; t0 += kThreads * kPerTile) {
-    const int tb = t0 + threadIdx.x * kPerTile;
-    uint32_t keys[kPerTile];
-    uint32_t my_gt = 0, my_eq = 0;
-    if (a.smem_vals && tb + kPerTile <= nseg) {
-      const float4 f = *reinterpret_cast<const float4*>(v + tb);  // conflict-free 16-B loads
-      keys[0] = order_key(f.x);
-      keys[1] = order_key(f.y);
-      keys[2] = order_key(f.z);
-      keys[3] = order_key(f.w);
-    } else {
+  // ---- order-preserving compaction ---------------------------------------------
+  {
+    uint32_t run_g = g_prev + warp_sum(lane < warp ? sh.warp_gt[lane] : 0u);
+    uint32_t run_e = e_prev + warp_sum(lane < warp ? sh.warp_eq[lane] : 0u);
+    const uint32_t kk32 = (uint32_t)kk;  // output slots of the ranked part (bounds guard)
+    for (int p = w0 + 4 * lane; p - 4 * lane < w1; p += 128) {
+      uint32_t key[4];
+      load_keys4(v, p, w1, vec, key);
+      uint32_t ng = 0, ne = 0;
 #pragma unroll
-      for (int q = 0; q < kPerTile; ++q) keys[q] = (tb + q < nseg) ? order_key(v[tb + q]) : 0u;
-    }
-#pragma unroll
-    for (int q = 0; q < kPerTile; ++q) {
-      if (tb + q < nseg) {
-        my_gt += keys[q] > T;
-        my_eq += keys[q] == T;
+      for (int q = 0; q < 4; ++q) {
+        ng += p + q < w1 && key[q] > T;
+        ne += p + q < w1 && key[q] == T;
       }
-    }
-    uint32_t tile_tot;
-    const uint32_t pref = block_excl_scan((my_eq << 16) | my_gt, sh.rx.warp_tmp, &tile_tot);
-    uint32_t g_before = pref & 0xffffu, e_before = pref >> 16;
-    const uint32_t quota = eq_seen < need_eq ? need_eq - eq_seen : 0u;
+      const uint32_t packed = warp_excl_scan(ng | (ne << 16));
+      uint32_t gb = run_g + (packed & 0xffffu);  // keys > T before this lane's first
+      uint32_t eb = run_e + (packed >> 16);      // keys == T before it
+      const uint32_t tot = __shfl_sync(0xffffffffu, packed + (ng | (ne << 16)), 31);
 #pragma unroll
-    for (int q = 0; q < kPerTile; ++q) {
-      const int t = tb + q;
-      if (t >= nseg) break;
-      const int32_t j = (int32_t)(s0 + t);
-      if (keys[q] > T) {
-        out[out_base + g_before + (e_before < quota ? e_before : quota)] = j;
-        ++g_before;
-      } else if (keys[q] == T) {
-        if (e_before < quota) out[out_base + g_before + e_before] = j;
-        ++e_before;
+      for (int q = 0; q < 4; ++q) {
+        const bool in = p + q < w1;
+        const bool g = in && key[q] > T, e = in && key[q] == T;
+        const uint32_t slot = gb + min(eb, need_eq);
+        if ((g || (e && eb < need_eq)) && slot < kk32) out[slot] = (int32_t)(s0 + p + q);
+        gb += g;
+        eb += e;
       }
+      run_g += tot & 0xffffu;
+      run_e += tot >> 16;
     }
-    const uint32_t tg = tile_tot & 0xffffu, te = tile_tot >> 16;
-    out_base += tg + (te < quota ? te : quota);
-    eq_seen += te;
   }
   finish_gvals();
-  cluster.sync();  // remote reads of sh are over before any CTA exits
+  cluster_wait();  // other CTAs' reads of this CTA's shared memory are over
 }
 
 // --------------------------------------------------------------------------
@@ -520,7 +838,7 @@ stats_kernel(const StatArgs a) {
   }
   const float mean = (float)(tsum / (double)a.n);
 
-  cluster_find_bucket(cluster, sh.rx, 0, kBins, (uint32_t)m);
+  cluster_find_bucket<kCS>(cluster, sh.rx, 0, kBins, (uint32_t)m);
   const uint32_t b1 = sh.rx.found_bucket;
   uint32_t want = sh.rx.found_rem;
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[1][i] = 0;
@@ -530,7 +848,7 @@ stats_kernel(const StatArgs a) {
     if ((key >> 21) == b1) atomicAdd(&sh.rx.hist[1][(key >> 10) & 2047u], 1);
   }
   cluster.sync();
-  cluster_find_bucket(cluster, sh.rx, 1, kBins, want);
+  cluster_find_bucket<kCS>(cluster, sh.rx, 1, kBins, want);
   const uint32_t pre2 = (b1 << 11) | sh.rx.found_bucket;
   want = sh.rx.found_rem;
   for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[0][i] = 0;
@@ -540,7 +858,7 @@ stats_kernel(const StatArgs a) {
     if ((key >> 10) == pre2) atomicAdd(&sh.rx.hist[0][key & 1023u], 1);
   }
   cluster.sync();
-  cluster_find_bucket(cluster, sh.rx, 0, 1024, want);
+  cluster_find_bucket<kCS>(cluster, sh.rx, 0, 1024, want);
   const uint32_t T = (pre2 << 10) | sh.rx.found_bucket;
   const uint32_t need_eq = sh.rx.found_rem;
 
@@ -576,10 +894,16 @@ stats_kernel(const StatArgs a) {
   cluster.sync();
 }
 
-constexpr size_t kSelDynMax = 180 * 1024;  // dynamic smem budget for pooled segments
+constexpr size_t kSelDynMax = 184 * 1024;  // dynamic smem of the selection kernel
 
-kvc_status launch_select(const SelArgs& a, int out_rows, int batch, int64_t seg, cudaStream_t st) {
-  const size_t dyn = sel_dyn_smem(seg, a.pool / 2, a.smem_vals);
+// pooled segment (and its staged row sums) of `seg` positions fit in shared memory
+bool sel_fits_smem(int64_t seg, int half) {
+  return (sel_v_words(seg) + sel_stage_words(seg, half)) * sizeof(float) <= kSelDynMax;
+}
+
+// Launch: kCS-CTA clusters, one per (sequence, output row).
+kvc_status launch_select(SelArgs a, int out_rows, int batch, cudaStream_t st) {
+  a.v_off = a.smem_vals ? (int)sel_stage_words(a.seg_cap, a.pool / 2) : 0;
   static std::mutex mu;
   static uint64_t done = 0;
   int dev = 0;
@@ -587,15 +911,25 @@ kvc_status launch_select(const SelArgs& a, int out_rows, int batch, int64_t seg,
   {
     std::lock_guard<std::mutex> lk(mu);
     if (dev >= 64 || !((done >> dev) & 1)) {
-      KVC_CUDA_TRY(cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+      KVC_CUDA_TRY(cudaFuncSetAttribute(select_kernel<kCS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                         (int)kSelDynMax));
       if (dev < 64) done |= (uint64_t)1 << dev;
     }
   }
-  dim3 grid(kCS, out_rows, batch);
-  select_kernel<<<grid, kThreads, dyn, st>>>(a);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kCS, out_rows, batch);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSelDynMax;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kCS;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  KVC_CUDA_TRY(cudaLaunchKernelEx(&cfg, select_kernel<kCS>, a));
   count_launch();
-  KVC_CUDA_TRY(cudaGetLastError());
   return KVC_OK;
 }
 
@@ -653,8 +987,8 @@ extern "C" kvc_status kvc_select_topk(const float* scores, int32_t rows, int64_t
   a.counts = nullptr;
   a.out_rows = out_rows;
   a.err = nullptr;
-  const int64_t seg = (n - window + kCS - 1) / kCS;
-  a.smem_vals = sel_dyn_smem(seg, pool_kernel / 2, true) <= kSelDynMax;
+  const int64_t seg = sel_segment(n - window, kCS);
+  a.smem_vals = sel_fits_smem(seg, pool_kernel / 2);
   a.seg_cap = seg;
   if (pooled) {
     a.vals_g = pooled;
@@ -671,7 +1005,7 @@ extern "C" kvc_status kvc_select_topk(const float* scores, int32_t rows, int64_t
     a.vals_stride = n;
     a.vals_packed = true;
   }
-  return launch_select(a, out_rows, 1, seg, (cudaStream_t)stream);
+  return launch_select(a, out_rows, 1, (cudaStream_t)stream);
 }
 
 extern "C" kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, int64_t row_stride,
@@ -690,8 +1024,8 @@ extern "C" kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, 
   const int out_rows = rows / row_group;
   size_t need = 0;
   kvc_select_workspace_size(out_rows, batch, total, &need);
-  const int64_t seg_max = (std::max<int64_t>(max_seqlen, window) - window + kCS - 1) / kCS;
-  if (sel_dyn_smem(seg_max, pool_kernel / 2, true) > kSelDynMax &&
+  const int64_t seg_max = sel_segment(std::max<int64_t>(max_seqlen, window) - window, kCS);
+  if (!sel_fits_smem(seg_max, pool_kernel / 2) &&
       (!ws || ws_bytes < need || !aligned(ws, kWsAlign)))
     return fail(KVC_ERR_WORKSPACE, "select workspace missing, too small or not 256-B aligned");
   SelArgs a{};
@@ -711,11 +1045,10 @@ extern "C" kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, 
   a.vals_packed = true;
   a.out_rows = out_rows;
   a.err = dev_err;
-  const int64_t seg = (std::max<int64_t>(max_seqlen, window) - window + kCS - 1) / kCS;
-  a.smem_vals = sel_dyn_smem(seg, pool_kernel / 2, true) <= kSelDynMax;
-  a.seg_cap = seg;
+  a.smem_vals = sel_fits_smem(seg_max, pool_kernel / 2);
+  a.seg_cap = seg_max;
   if (!a.smem_vals) a.vals_g = static_cast<float*>(ws);
-  return launch_select(a, out_rows, batch, seg, (cudaStream_t)stream);
+  return launch_select(a, out_rows, batch, (cudaStream_t)stream);
 }
 
 extern "C" kvc_status kvc_stats_workspace_size(int32_t rows, int64_t n, size_t* bytes) {

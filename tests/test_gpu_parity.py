@@ -82,17 +82,47 @@ def test_gather_hidden_bit_exact(D):
 # --------------------------------------------------------------------------- #
 # selection on given scores
 # --------------------------------------------------------------------------- #
-@pytest.mark.parametrize("n,w,k", [(50, 5, 12), (1000, 8, 64), (4097, 32, 1000), (20000, 32, 2048),
-                                   (300, 10, 10), (300, 10, 300), (300, 10, 1000), (131072, 32, 13107)])
-def test_select_exact_on_given_scores_no_pool(n, w, k):
+@pytest.mark.parametrize("n,w,k,levels", [(50, 5, 12, 50), (1000, 8, 64, 50), (4097, 32, 1000, 50),
+                                          (20000, 32, 2048, 50), (300, 10, 10, 50), (300, 10, 300, 50),
+                                          (300, 10, 1000, 50), (131072, 32, 13107, 50),
+                                          (131072, 32, 13107, 3), (131072, 32, 70000, 1)])
+def test_select_exact_on_given_scores_no_pool(n, w, k, levels):
     """Without pooling the GPU ranks exactly the values the oracle ranks: the
-    sets must be identical (ties included: many repeated values)."""
+    sets must be identical (ties included: many repeated values).  With 3 or 1
+    distinct values the threshold bin of the first radix digit holds tens of
+    thousands of keys, more than the candidate list takes, so the remaining
+    digits run cluster-wide."""
     rng = np.random.default_rng(n + k)
-    S = rng.integers(0, 50, size=(3, n)).astype(np.float32) * 0.25
+    S = rng.integers(0, levels, size=(3, n)).astype(np.float32) * 0.25
     idx = kvc.kvc_select_topk(torch.from_numpy(S).cuda(), w, 1, k).cpu().numpy()
     orc = oracle.get()
     for r in range(3):
         ref = orc.select_topk(S[r, : n - w].astype(np.float64), n, w, k)
+        assert np.array_equal(idx[r], ref), f"row {r}"
+
+
+def test_select_window_miss_falls_back_to_plain_radix():
+    """The selection brackets the k-th largest key with a window taken from
+    a sample of each CTA's keys (evenly spaced positions).  Here exactly the
+    sampled positions hold large values and everything else small ones, so the
+    window lands far above the true threshold; the result must still be exact
+    (the kernel then ranks with a plain radix select)."""
+    n, w, k, rows = 200000, 32, 20000, 4
+    L = n - w
+    cs = 8
+    seg = ((L + cs - 1) // cs + 3) & ~3
+    rng = np.random.default_rng(11)
+    S = rng.random((rows, n)).astype(np.float32)
+    for c in range(cs):
+        s0 = min(c * seg, L)
+        nseg = min(seg, L - s0)
+        nsc = min(256 // cs, nseg)
+        pos = s0 + ((2 * np.arange(nsc) + 1) * nseg) // (2 * nsc)
+        S[:, pos] = 100.0 + rng.random((rows, nsc)).astype(np.float32)
+    idx = kvc.kvc_select_topk(torch.from_numpy(S).cuda(), w, 1, k).cpu().numpy()
+    orc = oracle.get()
+    for r in range(rows):
+        ref = orc.select_topk(S[r, :L].astype(np.float64), n, w, k)
         assert np.array_equal(idx[r], ref), f"row {r}"
 
 
@@ -114,7 +144,7 @@ def test_select_long_row_global_memory_mode(n, pool):
         parity.assert_selection_matches(idx[r], orc.select_topk(Sp, n, w, k), Sp, n, w, k)
 
 
-@pytest.mark.parametrize("pool", [3, 7])
+@pytest.mark.parametrize("pool", [1, 3, 7, 9, 11, 65])
 def test_select_pooled_and_grouped(pool):
     rng = np.random.default_rng(pool)
     n, w, k, rows, grp = 9000, 16, 700, 8, 4
@@ -326,3 +356,31 @@ def test_varlen_select_rejects_sequences_longer_than_max_seqlen():
             Sp = orc.rank_scores(S[r, cu_np[b]:cu_np[b + 1]], lens[b], 16, 3)
             ref = orc.select_topk(Sp, lens[b], 16, 100)
             parity.assert_selection_matches(idx[b, r].cpu().numpy(), ref, Sp, lens[b], 16, 100)
+
+
+def test_layer_plan_matches_the_single_calls():
+    """LayerPlan ranks the TSP set on the head-sum row that scoring writes;
+    that row sums the heads in the same order and precision as the grouped
+    selection, so both index sets are identical.  The K/V chain runs on a
+    side stream; its results equal the direct calls."""
+    cfg = workloads.shrink(workloads.C3, N=20000, k_kv=2000, k_tsp=4000, hidden=512)
+    lay = workloads.make_layer(cfg)
+    q, kd, vd, xd = dev_bf16(lay.q), dev_bf16(lay.k), dev_bf16(lay.v), dev_bf16(lay.x)
+    plan = kvc.LayerPlan(cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden, True, "cuda",
+                         pool_kernel=cfg.pool)
+    out = plan.run(q, kd, vd, xd)
+    torch.cuda.synchronize()
+    scores = kvc.kvc_score(q, kd)
+    assert torch.equal(out.scores, scores)
+    ref_tsp = scores[0].clone()
+    for g in range(1, cfg.Hkv):
+        ref_tsp += scores[g]
+    assert torch.equal(out.tsp[0], ref_tsp)
+    it = kvc.kvc_select_topk(scores, cfg.w, cfg.pool, cfg.k_tsp, row_group=cfg.Hkv)
+    assert torch.equal(out.idx_tsp, it)
+    ik = kvc.kvc_select_topk(scores, cfg.w, cfg.pool, cfg.k_kv)
+    assert torch.equal(out.idx_kv, ik)
+    ko, vo = kvc.kvc_gather_kv(kd, vd, ik)
+    assert torch.equal(out.k_c, ko) and torch.equal(out.v_c, vo)
+    assert torch.equal(out.x_c, kvc.kvc_gather_hidden(xd, it.view(-1)))
+    assert plan.dev_err.item() == 0
