@@ -42,7 +42,7 @@ constexpr int kMaxHalf = 32;    // pool_kernel <= 65
 constexpr int kBins = 2048;     // radix bins of the first two passes
 constexpr int kWinBins = 1024;  // bins of the windowed histogram
 constexpr int kWin = kWinBins - 2;  // its interior bins (bin 0: below the window; last: above)
-constexpr int kSampleTotal = 256;   // sampled keys per ranking row
+constexpr int kSampleTotal = 128;   // sampled keys per ranking row
 constexpr int kCandMax = 1024;      // largest threshold bin resolved from a candidate list
 
 __device__ __forceinline__ uint32_t order_key(float v) {
@@ -196,7 +196,6 @@ struct SelShared {
   uint32_t sample[kSampleTotal];   // this CTA's sampled keys
   uint32_t sall[kSampleTotal];     // the cluster's samples (rank order), then ...
   uint32_t ssort[kSampleTotal];    // ... sorted, largest first
-  uint32_t ns;                     // this CTA's sample count
   uint32_t soff[kCS + 1];      // sample slots per rank
   uint32_t cand_off[kCS + 1];  // candidate slots per rank, total last
   uint32_t cand_n;                 // candidate slots this CTA has taken
@@ -241,20 +240,26 @@ __device__ __forceinline__ uint32_t warp_excl_scan(uint32_t v) {
   return x - v;
 }
 
-// Four consecutive pooled values v[p .. p+3] as order keys; positions at or
-// past `end` give 0 (the caller masks them).
-__device__ __forceinline__ void load_keys4(const float* v, int p, int end, bool vec, uint32_t (&key)[4]) {
-  if (vec && p + 4 <= end) {
-    const float4 f = *reinterpret_cast<const float4*>(v + p);
-    key[0] = order_key(f.x);
-    key[1] = order_key(f.y);
-    key[2] = order_key(f.z);
-    key[3] = order_key(f.w);
-  } else {
+// Order key of pooled value t: shared-memory mode stores the keys
+// themselves, global-memory mode the fp32 sums.
+struct PooledKeys {
+  const uint32_t* keys;  // shared-memory mode (16-byte aligned), else nullptr
+  const float* vals;     // global-memory mode
+  __device__ __forceinline__ uint32_t at(int t) const { return keys ? keys[t] : order_key(vals[t]); }
+  // keys of positions p .. p+3; positions at or past `end` give 0 (the caller masks them)
+  __device__ __forceinline__ void four(int p, int end, uint32_t (&key)[4]) const {
+    if (keys && p + 4 <= end) {
+      const uint4 k4 = *reinterpret_cast<const uint4*>(keys + p);
+      key[0] = k4.x;
+      key[1] = k4.y;
+      key[2] = k4.z;
+      key[3] = k4.w;
+    } else {
 #pragma unroll
-    for (int q = 0; q < 4; ++q) key[q] = p + q < end ? order_key(v[p + q]) : 0u;
+      for (int q = 0; q < 4; ++q) key[q] = p + q < end ? at(p + q) : 0u;
+    }
   }
-}
+};
 
 // The i-th position of a 1024-position block, spread so that the lanes of a
 // warp sit 32 positions apart (their keys rarely share a histogram bin).
@@ -407,15 +412,51 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
       }
     }
     __syncthreads();
-    // v[t] = sum of the p staged row sums around t.  Ranking uses this sum: the
-    // average differs by the constant factor 1/p, a monotone map, so the order
-    // (ties to the lower position) is the same; the average itself is only
-    // formed for the optional pooled output.  Each thread forms four
-    // consecutive outputs from 16-byte shared-memory loads (lanes 128
-    // positions apart: no bank conflicts).
+  } else {
+    // long rows: pooled values go straight to global memory (L2-resident)
+    for (int t = threadIdx.x; t < nseg; t += kThreads) {
+      float sum = 0.f;
+      for (int q = -half; q <= half; ++q) {
+        const int64_t pos = s0 + t + q;
+        if (pos < 0 || pos >= L) continue;
+        float rs = 0.f;
+        for (int r = 0; r < a.row_group; ++r) rs += rows0[(int64_t)r * a.row_stride + pos];
+        sum += rs;
+      }
+      v[t] = sum;  // ranked as the pooled sum (see the shared-memory path)
+    }
+    __syncthreads();
+  }
+  // global-memory mode keeps the pooled sums in the caller's buffer while
+  // ranking; it holds the averages once this CTA no longer reads them
+  auto finish_gvals = [&]() {
+    if (!a.smem_vals && gvals && a.pool > 1) {
+      __syncthreads();
+      for (int t = threadIdx.x; t < nseg; t += kThreads) v[t] = v[t] / pool_div;
+    }
+  };
+  const PooledKeys pk{a.smem_vals ? reinterpret_cast<const uint32_t*>(v) : nullptr, v};
+  const int hs = stage_halo(half);
+  const float* stage = dyn;
+  // Pooled sum of position t from the staged row sums (ascending order, the
+  // same as the pooling pass below).
+  auto pooled_at = [&](int t) {
+    float sum = 0.f;
+    for (int q = -half; q <= half; ++q) sum += stage[t + hs + q];
+    return sum;
+  };
+  // Shared-memory mode: the pooling pass.  v holds order keys of the sums p*S
+  // (ranking uses the sum: the average differs by the constant factor 1/p, a
+  // monotone map, so the order -- ties to the lower position -- is the same;
+  // the average itself is only formed for the optional pooled output).  Each
+  // thread forms four consecutive outputs from 16-byte shared-memory loads
+  // (lanes 128 positions apart: no bank conflicts, and neighbouring -- similar
+  // -- values rarely hit one histogram bin in the same instruction); `bin`
+  // maps keys to histogram bins, or is null.
+  auto pool_pass = [&](auto&& bin, bool with_hist) {
     const float4* st4 = reinterpret_cast<const float4*>(stage);
-    float4* v4 = reinterpret_cast<float4*>(v);
-    const int nv = nseg4 / 4;
+    uint4* v4 = reinterpret_cast<uint4*>(v);
+    const int nv = ((nseg + 3) & ~3) / 4;
     for (int i = spread_index(warp, lane); i < nv; i += kThreads) {
       float sums[4];
       if (hs == 0) {
@@ -437,61 +478,48 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
         }
       } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          float sum = 0.f;
-          for (int q = -half; q <= half; ++q) sum += stage[4 * i + u + hs + q];
-          sums[u] = sum;
-        }
+        for (int u = 0; u < 4; ++u) sums[u] = pooled_at(4 * i + u);
       }
-      v4[i] = make_float4(sums[0], sums[1], sums[2], sums[3]);
-      if (gvals) {
+      uint32_t key[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u)
-          if (4 * i + u < nseg) gvals[s0 + 4 * i + u] = (a.pool == 1) ? sums[u] : sums[u] / pool_div;
+      for (int u = 0; u < 4; ++u) key[u] = order_key(sums[u]);
+      v4[i] = make_uint4(key[0], key[1], key[2], key[3]);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const bool in = 4 * i + u < nseg;
+        if (in && gvals) gvals[s0 + 4 * i + u] = (a.pool == 1) ? sums[u] : sums[u] / pool_div;
+        if (with_hist) hist_add(sh.rx.hist[0], bin(key[u]), in);
       }
-    }
-  } else {
-    // long rows: pooled values go straight to global memory (L2-resident)
-    for (int t = threadIdx.x; t < nseg; t += kThreads) {
-      float sum = 0.f;
-      for (int q = -half; q <= half; ++q) {
-        const int64_t pos = s0 + t + q;
-        if (pos < 0 || pos >= L) continue;
-        float rs = 0.f;
-        for (int r = 0; r < a.row_group; ++r) rs += rows0[(int64_t)r * a.row_stride + pos];
-        sum += rs;
-      }
-      v[t] = sum;  // ranked as the pooled sum (see the shared-memory path)
-    }
-  }
-  // global-memory mode keeps the pooled sums in the caller's buffer while
-  // ranking; it holds the averages once this CTA no longer reads them
-  auto finish_gvals = [&]() {
-    if (!a.smem_vals && gvals && a.pool > 1) {
-      __syncthreads();
-      for (int t = threadIdx.x; t < nseg; t += kThreads) v[t] = v[t] / pool_div;
     }
   };
   if (!need_rank) {
+    if (a.smem_vals) pool_pass([](uint32_t) { return 0u; }, false);
     finish_gvals();
     return;
   }
-  __syncthreads();  // (global mode: each thread reads values other threads wrote)
 
   // ---- 1. sample -> key window --------------------------------------------------
-  {
-    const int per = kSampleTotal / CS;
-    const int nsc = nseg < per ? nseg : per;
-    if (threadIdx.x < nsc) sh.sample[threadIdx.x] = order_key(v[((2 * (int64_t)threadIdx.x + 1) * nseg) / (2 * nsc)]);
-    if (threadIdx.x == 0) sh.ns = (uint32_t)nsc;
-  }
-  cluster.sync();
+  // every CTA samples evenly spaced pooled values of its segment; the sample
+  // counts per rank follow from the segment lengths, so each CTA knows them
+  constexpr int kPer = kSampleTotal / CS;
   if (warp == 0) {
-    const uint32_t c = lane < CS ? cluster.map_shared_rank(&sh, lane)->ns : 0u;
+    uint32_t c = 0;
+    if (lane < CS) {
+      const int64_t r0 = (int64_t)lane * seg < L ? (int64_t)lane * seg : L;
+      const int64_t nr = L - r0 < seg ? L - r0 : seg;
+      c = (uint32_t)(nr < kPer ? nr : kPer);
+    }
     const uint32_t ex = warp_excl_scan(c);
     if (lane <= CS) sh.soff[lane] = ex;
   }
-  __syncthreads();
+  {
+    const int nsc = nseg < kPer ? nseg : kPer;
+    if (threadIdx.x < nsc) {
+      const int t = (int)(((2 * (int64_t)threadIdx.x + 1) * nseg) / (2 * nsc));
+      sh.sample[threadIdx.x] = a.smem_vals ? order_key(pooled_at(t)) : order_key(v[t]);
+    }
+  }
+  cluster.sync();
   const uint32_t ns = sh.soff[CS];
   if (threadIdx.x < ns) {
     int r = 0;
@@ -501,40 +529,45 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
   }
   __syncthreads();
   {
-    // rank by counting (equal keys: lower slot first), four threads per sample
-    const uint32_t i = threadIdx.x >> 2, part = threadIdx.x & 3;
+    // rank by counting (equal keys: lower slot first), eight threads per sample
+    const uint32_t i = threadIdx.x >> 3, part = threadIdx.x & 7;
     const uint32_t mine = i < ns ? sh.sall[i] : 0u;
     uint32_t c = 0;
     if (i < ns) {
 #pragma unroll 4
-      for (uint32_t j = part; j < ns; j += 4) {
+      for (uint32_t j = part; j < ns; j += 8) {
         const uint32_t x = sh.sall[j];
         c += (x > mine) || (x == mine && j < i);
       }
     }
     c += __shfl_xor_sync(0xffffffffu, c, 1);
     c += __shfl_xor_sync(0xffffffffu, c, 2);
+    c += __shfl_xor_sync(0xffffffffu, c, 4);
     if (i < ns && part == 0) sh.ssort[c] = mine;
   }
   __syncthreads();
   // the kk-th largest key sits near sample index ns*kk/L; the window spans
   // `margin` sample places to either side
-  const int64_t tr = (int64_t)ns * kk / L;
-  const int64_t margin = 4 + ns / 16;
+  const int tr = min((int)ns - 1, (int)((float)ns * ((float)kk / (float)L)));
+  const int margin = 4 + (int)ns / 16;
   const uint32_t hi_key = tr - margin >= 0 ? sh.ssort[tr - margin] : 0xFFFFFFFFu;
-  const uint32_t lo_key = tr + margin < (int64_t)ns ? sh.ssort[tr + margin] : 0u;
-  int wsh = 0;
-  while (((hi_key - lo_key) >> wsh) >= (uint32_t)kWin) ++wsh;
+  const uint32_t lo_key = tr + margin < (int)ns ? sh.ssort[tr + margin] : 0u;
+  const uint32_t wdt = hi_key - lo_key;
+  const int wsh = wdt < (uint32_t)kWin ? 0 : 32 - __clz(wdt / (uint32_t)kWin);  // (wdt >> wsh) < kWin
   auto wbin = [&](uint32_t key) -> uint32_t {
     if (key < lo_key) return 0u;
     const uint32_t d = (key - lo_key) >> wsh;
     return d >= (uint32_t)kWin ? (uint32_t)(kWinBins - 1) : d + 1u;
   };
 
-  // ---- 2. windowed histogram, summed over the cluster --------------------------
-  for (int t0 = 0; t0 < nseg; t0 += kThreads) {
-    const int t = t0 + spread_index(warp, lane);
-    if (t < nseg) hist_add(sh.rx.hist[0], wbin(order_key(v[t])), true);
+  // ---- 2. windowed histogram (with the pooling pass), summed over the cluster --
+  if (a.smem_vals) {
+    pool_pass(wbin, true);
+  } else {
+    for (int t0 = 0; t0 < nseg; t0 += kThreads) {
+      const int t = t0 + spread_index(warp, lane);
+      if (t < nseg) hist_add(sh.rx.hist[0], wbin(pk.at(t)), true);
+    }
   }
   cluster.sync();
   cluster_find_bucket<CS>(cluster, sh.rx, 0, kWinBins, (uint32_t)kk);
@@ -546,7 +579,6 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
   // segment, four consecutive positions per lane and step
   const int sub = (nseg + kThreads * 4 - 1) / (kThreads * 4) * 128;
   const int w0 = min(nseg, warp * sub), w1 = min(nseg, w0 + sub);
-  const bool vec = a.smem_vals;  // 16-byte aligned pooled values
 
   uint32_t T, need_eq;              // threshold key; how many keys == T are taken
   uint32_t g_prev = 0, e_prev = 0;  // keys > T / == T in the lower ranks
@@ -562,7 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
     uint32_t above_w = 0;  // keys of this warp's range in bins above b1
     for (int p = w0 + 4 * lane; p - 4 * lane < w1; p += 128) {
       uint32_t key[4];
-      load_keys4(v, p, w1, vec, key);
+      pk.four(p, w1, key);
       uint32_t nmine = 0;
       bool is[4];
 #pragma unroll
@@ -661,7 +693,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
     __syncthreads();
     for (int t0 = 0; t0 < nseg; t0 += kThreads) {
       const int t = t0 + spread_index(warp, lane);
-      if (t < nseg) hist_add(sh.rx.hist[1], order_key(v[t]) >> 21, true);
+      if (t < nseg) hist_add(sh.rx.hist[1], pk.at(t) >> 21, true);
     }
     cluster.sync();
     cluster_find_bucket<CS>(cluster, sh.rx, 1, kBins, want);
@@ -671,7 +703,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
     __syncthreads();
     for (int t0 = 0; t0 < nseg; t0 += kThreads) {
       const int t = t0 + spread_index(warp, lane);
-      const uint32_t key = t < nseg ? order_key(v[t]) : 0u;
+      const uint32_t key = t < nseg ? pk.at(t) : 0u;
       hist_add(sh.rx.hist[0], (key >> 10) & 2047u, t < nseg && (key >> 21) == r1);
     }
     cluster.sync();
@@ -682,7 +714,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
     __syncthreads();
     for (int t0 = 0; t0 < nseg; t0 += kThreads) {
       const int t = t0 + spread_index(warp, lane);
-      const uint32_t key = t < nseg ? order_key(v[t]) : 0u;
+      const uint32_t key = t < nseg ? pk.at(t) : 0u;
       hist_add(sh.rx.hist[1], key & 1023u, t < nseg && (key >> 10) == pre2);
     }
     cluster.sync();
@@ -694,7 +726,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
       uint32_t gt = 0, eq = 0;
       for (int p = w0 + 4 * lane; p < w1; p += 128) {
         uint32_t key[4];
-        load_keys4(v, p, w1, vec, key);
+        pk.four(p, w1, key);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           gt += p + q < w1 && key[q] > T;
@@ -744,7 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
     const uint32_t kk32 = (uint32_t)kk;  // output slots of the ranked part (bounds guard)
     for (int p = w0 + 4 * lane; p - 4 * lane < w1; p += 128) {
       uint32_t key[4];
-      load_keys4(v, p, w1, vec, key);
+      pk.four(p, w1, key);
       uint32_t ng = 0, ne = 0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
