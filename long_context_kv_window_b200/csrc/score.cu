@@ -133,18 +133,21 @@ struct Barriers {
 };
 
 // Shared memory: [Q rows, swizzled][pass 2: ones | bias block][K stage ring]
-// [barriers | exchange of the pass-1 group partials].  The pass-2 blocks hold one extra K-step of
-// the MMA: a [128 keys x 16] block of (1, 1, 1, 0, ...) and a [Rq x 16] block
-// of each row's (h1, h2, h3, 0, ...) with h1 + h2 + h3 = -bias / c (three
-// bf16 parts of an fp32-accurate value), laid out like the K tiles.
+// [barriers].  The pass-2 blocks hold one extra K-step of the MMA: a
+// [128 keys x 16] block of (1, 1, 1, 0, ...) and a [Rq x 16] block of each
+// row's (h1, h2, h3, 0, ...) with h1 + h2 + h3 = -bias / c (three bf16 parts
+// of an fp32-accurate value), 32-byte rows with the 32-byte swizzle.  Pass 1
+// exchanges its group partials through the K ring once every tile is done.
 template <int D>
 struct Smem {
   static constexpr int kChunks = D / 64;  // 64-element (128 B) swizzle columns
   static constexpr int kStageBytes = kChunks * kTile * 128;
-  static constexpr size_t kOnesBytes = (size_t)kTile * 128;
-  static constexpr size_t kTail = 512 /*barriers*/ + (size_t)(kGroups - 1) * 256 * (4 + 8) /*exchange*/;
+  static constexpr size_t kOnesBytes = (size_t)kTile * 32;
+  static constexpr size_t kTail = 512;  // barriers
+  static constexpr size_t kExchangeBytes = (size_t)(kGroups - 1) * 256 * (4 + 8);
+  static_assert(kExchangeBytes <= (size_t)kStageBytes * 2, "pass-1 exchange must fit in two stages");
   __host__ __device__ static size_t q_bytes(int Rq) { return (size_t)kChunks * Rq * 128; }
-  __host__ __device__ static size_t fold_bytes(int Rq, int fold) { return fold ? kOnesBytes + (size_t)Rq * 128 : 0; }
+  __host__ __device__ static size_t fold_bytes(int Rq, int fold) { return fold ? kOnesBytes + (size_t)Rq * 32 : 0; }
   __host__ __device__ static size_t total(int Rq, int stages, int fold) {
     return 1024 /*alignment slack*/ + q_bytes(Rq) + fold_bytes(Rq, fold) + (size_t)stages * kStageBytes + kTail;
   }
@@ -157,7 +160,7 @@ struct SmemPtrs {
   uint8_t* qb;    // pass 2 only
   uint8_t* kst;
   Barriers* bars;
-  float* ex_m;   // [kGroups - 1][256]
+  float* ex_m;   // [kGroups - 1][256], in the K ring (pass 1, after the last tile)
   double* ex_l;  // [kGroups - 1][256]
   __device__ SmemPtrs(uint8_t* raw, const ScoreArgs& a) {
     uint8_t* s = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
@@ -166,7 +169,7 @@ struct SmemPtrs {
     qb = ones + Smem<D>::kOnesBytes;
     kst = qs + Smem<D>::q_bytes(a.Rq) + Smem<D>::fold_bytes(a.Rq, a.fold);
     bars = reinterpret_cast<Barriers*>(kst + (size_t)a.stages * Smem<D>::kStageBytes);
-    ex_m = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 512);
+    ex_m = reinterpret_cast<float*>(kst);
     ex_l = reinterpret_cast<double*>(ex_m + (kGroups - 1) * 256);
   }
 };
@@ -253,8 +256,8 @@ __device__ __forceinline__ void issue_mmas(const ScoreArgs& a, Barriers* bars, u
   constexpr int kChunks = D / 64;
   const uint32_t idesc = kRowsOnM ? tc::idesc_bf16_f32(128, kTile) : tc::idesc_bf16_f32(128, a.Rn);
   const uint32_t qbase = tc::smem_u32(qs), kbase = tc::smem_u32(kst);
-  const uint64_t ones_desc = tc::desc_k_sw128(tc::smem_u32(ones));
-  const uint64_t qb_desc = tc::desc_k_sw128(tc::smem_u32(qb));
+  const uint64_t ones_desc = tc::desc_k_sw32(tc::smem_u32(ones));
+  const uint64_t qb_desc = tc::desc_k_sw32(tc::smem_u32(qb));
   int issued = 0;
   const bool go = kRowsOnM || tc::mbar_wait(&bars->bias_ready, 0, &bars->abort);
   for (int t = 0; go && t < ntiles; ++t) {
@@ -602,14 +605,14 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   }
   {
     // constant operands of the extra K-step: ones block (keys) and a zeroed
-    // bias block (rows); row r's 16-byte chunk 0 sits at chunk (r & 7)
+    // bias block (rows); row r's 16-byte chunk 0 sits at chunk (r >> 2) & 1
     uint4* ones4 = reinterpret_cast<uint4*>(sp.ones);
     for (int v = threadIdx.x; v < (int)(Smem<D>::kOnesBytes / 16); v += blockDim.x) {
-      const int r = v >> 3, ch = v & 7;
-      ones4[v] = (ch == (r & 7)) ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+      const int r = v >> 1, ch = v & 1;
+      ones4[v] = (ch == ((r >> 2) & 1)) ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
     }
     uint4* qb4 = reinterpret_cast<uint4*>(sp.qb);
-    for (int v = threadIdx.x; v < a.Rq * 8; v += blockDim.x) qb4[v] = make_uint4(0u, 0u, 0u, 0u);
+    for (int v = threadIdx.x; v < a.Rq * 2; v += blockDim.x) qb4[v] = make_uint4(0u, 0u, 0u, 0u);
   }
   load_q_swizzled<D>(a, wk.b, g, sp.qs);
   tc::tc_fence_before();
@@ -630,7 +633,7 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
       const int r = threadIdx.x - 64;
       if (r < a.Rn) {
         const uint2 wv = a.qsplit[((size_t)wk.b * a.Hkv + g) * a.Rq + r];
-        *reinterpret_cast<uint4*>(sp.qb + (size_t)r * 128 + (size_t)(r & 7) * 16) = make_uint4(wv.x, wv.y, 0u, 0u);
+        *reinterpret_cast<uint4*>(sp.qb + (size_t)r * 32 + (size_t)((r >> 2) & 1) * 16) = make_uint4(wv.x, wv.y, 0u, 0u);
       }
       tc::fence_proxy_async_smem();  // visible to the MMA's operand reads
       tc::mbar_arrive(&bars->bias_ready);

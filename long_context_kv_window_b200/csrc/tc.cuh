@@ -149,6 +149,20 @@ __device__ __forceinline__ uint64_t desc_k_sw128(uint32_t smem_addr) {
   return d;
 }
 
+// The same for a K-major bf16 operand of exactly one MMA K-step (16
+// elements = 32 B per row) stored with the 32-byte swizzle: 8-row atoms of
+// 256 B, the two 16-byte halves of row r swapped when bit 2 of r is set.
+// Stride byte offset 256 B between 8-row groups; layout SWIZZLE_32B (= 6).
+__device__ __forceinline__ uint64_t desc_k_sw32(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(256 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)6 << 61;
+  return d;
+}
+
 // Instruction descriptor, kind::f16: D fp32, A and B bf16, both K-major,
 // dense, no negation; N >> 3 in [17,23), M >> 4 in [24,29).
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
