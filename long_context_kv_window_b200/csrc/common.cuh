@@ -60,7 +60,49 @@ struct WsCursor {
     if (!(cond)) return ::kvc::fail(KVC_ERR_INVALID_ARG, msg); \
   } while (0)
 
+// ------------------------------------------------ programmatic dependent launch
+// Every kernel of the library is launched with programmatic stream
+// serialization: its CTAs may start once every CTA of the previous kernel in
+// the stream has called pdl_trigger() (or exited), i.e. while that kernel
+// still runs.  A kernel calls pdl_wait() -- which returns once the previous
+// kernel has completed and its memory is visible -- before it touches global
+// memory that an earlier kernel of the stream writes or reads, and calls
+// pdl_trigger() after its own pdl_wait(): then whatever a kernel reads
+// before its pdl_wait() (inputs of the library call) was complete before the
+// previous kernel passed its own wait.
+struct Launch {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  Launch(dim3 grid, dim3 block, size_t smem, cudaStream_t st) : cfg{}, attr{} {
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  }
+  Launch(const Launch&) = delete;
+  Launch& operator=(const Launch&) = delete;
+  // thread-block clusters of x CTAs along the grid's x axis
+  void cluster_x(unsigned x) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  template <class... K, class... A>
+  cudaError_t run(void (*kernel)(K...), A&&... args) const {
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<A&&>(args)...);
+  }
+};
+
 // -------------------------------------------------------------- device side
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void set_dev_err(int32_t* err, int32_t bit) {
   if (err) atomicOr(err, bit);
 }

@@ -24,6 +24,8 @@ gather_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int64
                  const int32_t* __restrict__ cu, int64_t n, int Hkv, const int32_t* __restrict__ idx,
                  int64_t idx_row_stride, int64_t kk, uint4* __restrict__ k_out,
                  uint4* __restrict__ v_out, int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
   // blockIdx.y = b * Hkv + g ; blockIdx.x covers kk * VPR items of that head
   const int bg = blockIdx.y;
   const int g = bg % Hkv;
@@ -71,6 +73,8 @@ __global__ void __launch_bounds__(kGatherThreads)
 gather_hidden_kernel(const uint4* __restrict__ x, int64_t sn_v, int64_t n, int64_t vpr,
                      const int32_t* __restrict__ idx, int64_t kk, uint4* __restrict__ out,
                      int32_t* err) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (kGatherThreads / 32);
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
@@ -114,14 +118,13 @@ kvc_status launch_gather_kv(const uint16_t* k, const uint16_t* v, int64_t sn, in
   auto vp = reinterpret_cast<const uint4*>(v);
   auto ko = reinterpret_cast<uint4*>(k_out);
   auto vo = reinterpret_cast<uint4*>(v_out);
+  const Launch l(grid, dim3(kGatherThreads), 0, st);
+  const int64_t sn8 = sn / 8, sh8 = sh / 8;
   if (vpr == 16)
-    gather_kv_kernel<16><<<grid, kGatherThreads, 0, st>>>(kp, vp, sn / 8, sh / 8, cu, n, Hkv, idx,
-                                                           idx_row_stride, kk, ko, vo, err);
+    KVC_CUDA_TRY(l.run(gather_kv_kernel<16>, kp, vp, sn8, sh8, cu, n, Hkv, idx, idx_row_stride, kk, ko, vo, err));
   else
-    gather_kv_kernel<8><<<grid, kGatherThreads, 0, st>>>(kp, vp, sn / 8, sh / 8, cu, n, Hkv, idx,
-                                                          idx_row_stride, kk, ko, vo, err);
+    KVC_CUDA_TRY(l.run(gather_kv_kernel<8>, kp, vp, sn8, sh8, cu, n, Hkv, idx, idx_row_stride, kk, ko, vo, err));
   count_launch();
-  KVC_CUDA_TRY(cudaGetLastError());
   return KVC_OK;
 }
 
@@ -192,10 +195,9 @@ extern "C" kvc_status kvc_gather_hidden(const uint16_t* x, int64_t stride_n, int
   int64_t blocks = (kk + warps_per_block - 1) / warps_per_block;
   const int64_t cap = (int64_t)num_sms() * 8;
   if (blocks > cap) blocks = cap;
-  gather_hidden_kernel<<<(unsigned)blocks, kGatherThreads, 0, (cudaStream_t)stream>>>(
-      reinterpret_cast<const uint4*>(x), stride_n / 8, n, hidden / 8, idx, kk,
-      reinterpret_cast<uint4*>(out), dev_err);
+  const Launch l(dim3((unsigned)blocks), dim3(kGatherThreads), 0, (cudaStream_t)stream);
+  KVC_CUDA_TRY(l.run(gather_hidden_kernel, reinterpret_cast<const uint4*>(x), stride_n / 8, n, hidden / 8, idx, kk,
+                     reinterpret_cast<uint4*>(out), dev_err));
   count_launch();
-  KVC_CUDA_TRY(cudaGetLastError());
   return KVC_OK;
 }

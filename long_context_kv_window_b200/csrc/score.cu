@@ -400,6 +400,8 @@ __device__ __forceinline__ void pass1_group(uint32_t (&x)[kCols], float c, float
 template <int D>
 __global__ void __launch_bounds__(kThreadsScore, 1)
 score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) {
+  pdl_wait();
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   const SmemPtrs<D> sp(smem_raw, a);
   Barriers* bars = sp.bars;
@@ -515,6 +517,10 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
 // one).  Pass 2 multiplies them by ones in one extra MMA K-step.
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) score_combine_kernel(const ScoreArgs a) {
+  // pass 2 may launch now: its prologue (barriers, TMEM, Q, first K tiles)
+  // reads only the inputs and overlaps pass 1's tail and this kernel
+  pdl_trigger();
+  pdl_wait();
   const int g = blockIdx.x, b = blockIdx.y;
   int gid0 = 0, nch = 0;
   bool bad = false;
@@ -579,6 +585,10 @@ __global__ void __launch_bounds__(256) score_combine_kernel(const ScoreArgs a) {
 template <int D>
 __global__ void __launch_bounds__(kThreadsScore, 1)
 score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) {
+  // Before pdl_wait() this kernel reads only the call's inputs (Q, K, the
+  // sequence offsets) and shared memory; the combined biases and every global
+  // write come after it.
+  pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   const SmemPtrs<D> sp(smem_raw, a);
   Barriers* bars = sp.bars;
@@ -588,6 +598,7 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   const Work wk = map_work(a, blockIdx.x, true);
   if (!wk.valid) return;
   if (wk.bad) {
+    pdl_wait();
     // leave nothing stale behind: zero whatever part of the row is addressable
     if (wk.start >= 0 && wk.len > 0 && wk.start + wk.len <= a.total)
       for (int64_t j = threadIdx.x; j < wk.len; j += blockDim.x) a.scores[(int64_t)g * a.total + wk.start + j] = 0.f;
@@ -630,6 +641,7 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
     // x - b_r / c.  TMA fills the pipeline meanwhile; the MMA waits for
     // bias_ready.
     {
+      pdl_wait();  // the combined biases (previous kernel)
       const int r = threadIdx.x - 64;
       if (r < a.Rn) {
         const uint2 wv = a.qsplit[((size_t)wk.b * a.Hkv + g) * a.Rq + r];
@@ -702,6 +714,8 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
 
 // TSP aggregate: tsp[j] = sum_g scores[g][j] (all heads, one row).
 __global__ void tsp_sum_kernel(const float* __restrict__ scores, int Hkv, int64_t total, float* __restrict__ tsp) {
+  pdl_wait();
+  pdl_trigger();
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < total; j += (int64_t)gridDim.x * blockDim.x) {
     float s = 0.f;
     for (int g = 0; g < Hkv; ++g) s += scores[(int64_t)g * total + j];
@@ -816,18 +830,24 @@ kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, 
     a.tmem_cols = gm.cols1;
     a.stages = stages[0];
     a.fold = 0;
-    score_pass1_kernel<D><<<grid, kThreadsScore, smem[0], st>>>(kmap, a);
-    KVC_CUDA_TRY(cudaGetLastError());
-    score_combine_kernel<<<dim3(a.Hkv, a.B), 256, 0, st>>>(a);
-    KVC_CUDA_TRY(cudaGetLastError());
+    {
+      const Launch l(grid, dim3(kThreadsScore), smem[0], st);
+      KVC_CUDA_TRY(l.run(score_pass1_kernel<D>, kmap, a));
+    }
+    {
+      const Launch l(dim3(a.Hkv, a.B), dim3(256), 0, st);
+      KVC_CUDA_TRY(l.run(score_combine_kernel, a));
+    }
     count_launch();
     a.acc_stride = gm.stride2;
     a.nbuf = gm.nbuf2;
     a.tmem_cols = gm.cols2;
     a.stages = stages[1];
     a.fold = 1;
-    score_pass2_kernel<D><<<grid, kThreadsScore, smem[1], st>>>(kmap, a);
-    KVC_CUDA_TRY(cudaGetLastError());
+    {
+      const Launch l(grid, dim3(kThreadsScore), smem[1], st);
+      KVC_CUDA_TRY(l.run(score_pass2_kernel<D>, kmap, a));
+    }
     count_launch(2);
   }
   return KVC_OK;
@@ -924,9 +944,9 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
   if (tsp) {
     const int threads = 256;
     const int64_t blocks = std::min<int64_t>((total + threads - 1) / threads, (int64_t)sms * 8);
-    tsp_sum_kernel<<<(unsigned)blocks, threads, 0, st>>>(scores, Hkv, total, tsp);
+    const Launch l(dim3((unsigned)blocks), dim3(threads), 0, st);
+    KVC_CUDA_TRY(l.run(tsp_sum_kernel, (const float*)scores, Hkv, total, tsp));
     count_launch();
-    KVC_CUDA_TRY(cudaGetLastError());
   }
   return KVC_OK;
 }

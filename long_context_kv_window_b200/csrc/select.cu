@@ -277,6 +277,8 @@ __host__ __device__ inline int64_t sel_segment(int64_t L, int cs) { return ((L +
 
 template <int CS>
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ SelShared sh;
   extern __shared__ __align__(16) float dyn[];
   cg::cluster_group cluster = cg::this_cluster();
@@ -836,6 +838,8 @@ __device__ double block_sum(double v, double* red) {
 
 __global__ void __cluster_dims__(kCS, 1, 1) __launch_bounds__(kThreads, 1)
 stats_kernel(const StatArgs a) {
+  pdl_wait();
+  pdl_trigger();
   __shared__ StatShared sh;
   cg::cluster_group cluster = cg::this_cluster();
   const int crank = (int)cluster.block_rank();
@@ -948,19 +952,9 @@ kvc_status launch_select(SelArgs a, int out_rows, int batch, cudaStream_t st) {
       if (dev < 64) done |= (uint64_t)1 << dev;
     }
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kCS, out_rows, batch);
-  cfg.blockDim = dim3(kThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSelDynMax;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kCS;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  KVC_CUDA_TRY(cudaLaunchKernelEx(&cfg, select_kernel<kCS>, a));
+  Launch l(dim3(kCS, out_rows, batch), dim3(kThreads), kSelDynMax, st);
+  l.cluster_x(kCS);
+  KVC_CUDA_TRY(l.run(select_kernel<kCS>, a));
   count_launch();
   return KVC_OK;
 }
@@ -1102,8 +1096,8 @@ extern "C" kvc_status kvc_layer_stats(const float* scores, int32_t rows, int64_t
   KVC_CHECK_ARG(mass_norm > 0.f, "mass_norm must be > 0");
   StatArgs a{scores, row_stride, n, 1.0f / mass_norm, out};
   dim3 grid(kCS, rows, 1);
-  stats_kernel<<<grid, kThreads, 0, (cudaStream_t)stream>>>(a);
+  const Launch l(grid, dim3(kThreads), 0, (cudaStream_t)stream);
+  KVC_CUDA_TRY(l.run(stats_kernel, a));
   count_launch();
-  KVC_CUDA_TRY(cudaGetLastError());
   return KVC_OK;
 }
