@@ -641,29 +641,72 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
     uint32_t above_prev = 0;
     if (warp == 0) above_prev = warp_sum(lane < crank ? cluster.map_shared_rank(&sh, lane)->above : 0u);
     __syncthreads();
-    // the want-th largest candidate: rank by counting, four threads per
-    // candidate (nc <= kCandMax = kThreads)
+    // the want-th largest candidate.  Every candidate lies in bin b1, i.e.
+    // its key is base + off with off < 2^wsh.  Up to two 11-bit histogram
+    // levels over off narrow a long list down to the keys that agree above
+    // the last `rest` bits; those are ranked by counting (four threads per
+    // key).  Lists alternate between hist[0] and tot (free by now: no CTA
+    // reads this CTA's histograms after the last cluster barrier).
     {
-      const uint32_t want = sh.rx.found_rem;
-      for (uint32_t i0 = 0; i0 < nc; i0 += kThreads / 4) {
-        const uint32_t i = i0 + (threadIdx.x >> 2), part = threadIdx.x & 3;
-        const uint32_t mine = i < nc ? sh.cand[i].x : 0u;
-        uint32_t gt = 0, eq = 0;
-        if (i < nc) {
-#pragma unroll 4
-          for (uint32_t j = part; j < nc; j += 4) {
-            const uint32_t x = sh.cand[j].x;
-            gt += x > mine;
-            eq += x == mine;
-          }
+      uint32_t want = sh.rx.found_rem;
+      const uint32_t base = lo_key + ((b1 - 1u) << wsh);
+      uint32_t* lst = reinterpret_cast<uint32_t*>(sh.rx.hist[0]);
+      uint32_t* nxt = reinterpret_cast<uint32_t*>(sh.rx.tot);
+      for (uint32_t i = threadIdx.x; i < nc; i += kThreads) lst[i] = sh.cand[i].x - base;
+      if (threadIdx.x == 0) sh.cand_n = 0;
+      __syncthreads();
+      uint32_t n = nc;
+      int rest = wsh;
+      for (int level = 0; level < 2 && n > 64 && rest > 0; ++level) {
+        const int sb = rest < 11 ? rest : 11;
+        const int shf = rest - sb;
+        const uint32_t mask = (1u << sb) - 1u;
+        for (int i = threadIdx.x; i < kBins; i += kThreads) sh.rx.hist[1][i] = 0;
+        __syncthreads();
+        for (uint32_t i = threadIdx.x; i < n; i += kThreads) atomicAdd(&sh.rx.hist[1][(lst[i] >> shf) & mask], 1);
+        __syncthreads();
+        scan_find(sh.rx, sh.rx.hist[1], kBins, want);
+        const uint32_t sbin = sh.rx.found_bucket & mask;
+        want = sh.rx.found_rem;
+        for (uint32_t i = threadIdx.x; i < n; i += kThreads) {
+          const uint32_t x = lst[i];
+          if (((x >> shf) & mask) == sbin) nxt[atomicAdd(&sh.cand_n, 1u)] = x;
         }
-        gt += __shfl_xor_sync(0xffffffffu, gt, 1);
-        gt += __shfl_xor_sync(0xffffffffu, gt, 2);
-        eq += __shfl_xor_sync(0xffffffffu, eq, 1);
-        eq += __shfl_xor_sync(0xffffffffu, eq, 2);
-        if (i < nc && part == 0 && gt < want && want <= gt + eq) {
-          sh.T = mine;
-          sh.need_eq = want - gt;
+        __syncthreads();
+        n = sh.cand_n;
+        __syncthreads();
+        if (threadIdx.x == 0) sh.cand_n = 0;
+        uint32_t* t = lst;
+        lst = nxt;
+        nxt = t;
+        rest = shf;
+      }
+      if (rest == 0) {  // the survivors are all equal
+        if (threadIdx.x == 0) {
+          sh.T = base + lst[0];
+          sh.need_eq = want;
+        }
+      } else {
+        for (uint32_t i0 = 0; i0 < n; i0 += kThreads / 4) {
+          const uint32_t i = i0 + (threadIdx.x >> 2), part = threadIdx.x & 3;
+          const uint32_t mine = i < n ? lst[i] : 0u;
+          uint32_t gt = 0, eq = 0;
+          if (i < n) {
+#pragma unroll 4
+            for (uint32_t j = part; j < n; j += 4) {
+              const uint32_t x = lst[j];
+              gt += x > mine;
+              eq += x == mine;
+            }
+          }
+          gt += __shfl_xor_sync(0xffffffffu, gt, 1);
+          gt += __shfl_xor_sync(0xffffffffu, gt, 2);
+          eq += __shfl_xor_sync(0xffffffffu, eq, 1);
+          eq += __shfl_xor_sync(0xffffffffu, eq, 2);
+          if (i < n && part == 0 && gt < want && want <= gt + eq) {
+            sh.T = base + mine;
+            sh.need_eq = want - gt;
+          }
         }
       }
     }

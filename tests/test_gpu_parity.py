@@ -384,3 +384,18 @@ def test_layer_plan_matches_the_single_calls():
     assert torch.equal(out.k_c, ko) and torch.equal(out.v_c, vo)
     assert torch.equal(out.x_c, kvc.kvc_gather_hidden(xd, it.view(-1)))
     assert plan.dev_err.item() == 0
+
+
+@pytest.mark.parametrize("sigma,pool,k", [(3.0, 7, 13107), (1.0, 7, 26214), (3.0, 1, 4000)])
+def test_select_heavy_tailed_rows(sigma, pool, k):
+    """Log-normal rows: a long upper tail stretches the sampled key window, so
+    the threshold bin holds hundreds of keys and the kernel narrows them with
+    histogram levels before ranking the survivors."""
+    n, w, rows = 131072, 32, 4
+    rng = np.random.default_rng(int(sigma * 10) + pool + k)
+    S = np.exp(sigma * rng.standard_normal((rows, n))).astype(np.float32)
+    idx = kvc.kvc_select_topk(torch.from_numpy(S).cuda(), w, pool, k).cpu().numpy()
+    orc = oracle.get()
+    for r in range(rows):
+        Sp = orc.rank_scores(S[r].astype(np.float64), n, w, pool)
+        parity.assert_selection_matches(idx[r], orc.select_topk(Sp, n, w, k), Sp, n, w, k)
