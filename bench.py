@@ -297,27 +297,28 @@ def main() -> None:
         raise RuntimeError(f"device error word {plan.dev_err.item()}")
 
     # ---- timed region ----------------------------------------------------------
-    # per-call events; "external" so that, recorded inside a CUDA graph, they
-    # stay readable (timing) after the replay
-    evs = [{c: (torch.cuda.Event(enable_timing=True, external=not args.no_graph),
-                torch.cuda.Event(enable_timing=True, external=not args.no_graph)) for c in calls}
-           for _ in range(args.steps)]
-    t_start = torch.cuda.Event(enable_timing=True)
-    t_end = torch.cuda.Event(enable_timing=True)
-    sampler = ClockSampler(local)
-    launches0 = kvc.launch_count()
-    graph = None
-    if not args.no_graph:
-        # the K steps (with their per-call events) are captured once and
-        # replayed as one CUDA graph: no host launch overhead between kernels
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph):
-            cap = torch.cuda.current_stream(dev)
-            for s in range(args.steps):
-                step(evs[s], main=cap)
-        torch.cuda.synchronize(dev)
-    launches = kvc.launch_count() - launches0
-    with sampler:
+    def timed_run(with_events: bool):
+        """K steps, captured once as a CUDA graph (unless --no-graph) and
+        replayed; device time per step, and per-call times when the steps
+        carry per-call events.  The headline run carries none: an event
+        recorded between two kernels of a stream also cuts the programmatic
+        (early-launch) dependency between them."""
+        evs = [{c: (torch.cuda.Event(enable_timing=True, external=not args.no_graph),
+                    torch.cuda.Event(enable_timing=True, external=not args.no_graph)) for c in calls}
+               if with_events else None for _ in range(args.steps)]
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        launches0 = kvc.launch_count()
+        graph = None
+        if not args.no_graph:
+            # no host launch overhead between kernels
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                cap = torch.cuda.current_stream(dev)
+                for s_ in range(args.steps):
+                    step(evs[s_], main=cap)
+            torch.cuda.synchronize(dev)
+        launches = kvc.launch_count() - launches0
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
@@ -325,18 +326,25 @@ def main() -> None:
         if graph is not None:
             graph.replay()
         else:
-            for s in range(args.steps):
-                step(evs[s], main=st)
+            for s_ in range(args.steps):
+                step(evs[s_], main=st)
         t_end.record(st)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-    if graph is None:
-        launches = kvc.launch_count() - launches0
-    ms_total = shard.max_over_ranks(t_start.elapsed_time(t_end), dist, dev)
-    ms_step = ms_total / args.steps
-    per_call = {c: sum(evs[s][c][0].elapsed_time(evs[s][c][1]) for s in range(args.steps)) / args.steps
-                for c in calls}
+        if graph is None:
+            launches = kvc.launch_count() - launches0
+        ms = shard.max_over_ranks(t_start.elapsed_time(t_end), dist, dev) / args.steps
+        per_call = None
+        if with_events:
+            per_call = {c: sum(evs[s_][c][0].elapsed_time(evs[s_][c][1]) for s_ in range(args.steps)) / args.steps
+                        for c in calls}
+        return ms, per_call, launches
+
+    sampler = ClockSampler(local)
+    with sampler:
+        ms_step, _, launches = timed_run(with_events=False)
+    ms_step_events, per_call, _ = timed_run(with_events=True)
 
     # ---- end to end through the public API with host buffers ------------------
     hq, hk, hv, hx = (workloads.torch_bf16(a).pin_memory() for a in (lay.q, lay.k, lay.v, lay.x))
@@ -390,10 +398,11 @@ def main() -> None:
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
                          "traffic": load_traffic(dom)},
             "calls": breakdown,
+            "ms_per_step_with_call_events": ms_step_events,
             "e2e": {"value": world * cfg.N / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},
             "gpu_launches": launches,
-            "graph": graph is not None,
+            "graph": not args.no_graph,
             "clocks": sampler.summary(),
             "cpu_baseline": cpu,
         }
