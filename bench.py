@@ -208,6 +208,124 @@ def run_reference(args, cfg, rank: int) -> None:
 
 
 # --------------------------------------------------------------------------- #
+# the other configurations (per-layer time; the headline is the 128K layer)
+# --------------------------------------------------------------------------- #
+def other_bytes(cfg, total: int) -> int:
+    """Algorithmic HBM bytes of one layer of cfg (K once, Q_win, scores written
+    and read once, the K/V gather's rows in and out; the head-sum row when a
+    TSP budget is given)."""
+    B = cfg.batch
+    b = total * cfg.Hkv * cfg.d * 2 + B * cfg.w * cfg.H * cfg.d * 2 + 2 * cfg.Hkv * total * 4
+    kv_rows = cfg.Hkv * B * min(cfg.k_kv, cfg.N)
+    b += (2 if cfg.with_v else 1) * 2 * kv_rows * cfg.d * 2
+    if cfg.k_tsp:
+        b += 2 * total * 4
+    return b
+
+
+def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
+    """Per-layer time of configuration cfg on one GPU: score (with the head-sum
+    row and C_global accumulation where cfg has them) -> per-KV-head top-k ->
+    K(/V) gather, plus the TSP top-k and the layer statistics for the
+    16-layer configuration; ragged batches through the varlen calls."""
+    layers = ([workloads.make_layer(cfg, layer=l) for l in range(1, cfg.layers + 1)] if cfg.layers > 1
+              else [workloads.make_layer(cfg)])
+    lay0 = layers[0]
+    B, total = lay0.batch, lay0.total
+    max_len = int(lay0.lengths().max())
+    qs = [workloads.torch_bf16(l.q, dev).view(B, cfg.w, cfg.H, cfg.d) if B > 1 else workloads.torch_bf16(l.q, dev)
+          for l in layers]
+    ks = [workloads.torch_bf16(l.k, dev) for l in layers]
+    vs = [workloads.torch_bf16(l.v, dev) if cfg.with_v else None for l in layers]
+    cu = torch.from_numpy(lay0.cu_seqlens).to(dev)
+    kk = min(cfg.k_kv, cfg.N)
+    scores = torch.empty((cfg.Hkv, total), dtype=torch.float32, device=dev)
+    tsp = torch.empty((1, total), dtype=torch.float32, device=dev) if cfg.k_tsp else None
+    accum = torch.zeros((cfg.Hkv, total), dtype=torch.float32, device=dev) if cfg.layers > 1 else None
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    p = kvc.score_params(cfg.H, cfg.Hkv, cfg.d, cfg.w)
+    ws_s = torch.empty(kvc.score_workspace_size(p, B, total), dtype=torch.uint8, device=dev)
+    ws_k = torch.empty(kvc.select_workspace_size(cfg.Hkv, B, total), dtype=torch.uint8, device=dev)
+    ws_t = torch.empty(kvc.select_workspace_size(1, B, total), dtype=torch.uint8, device=dev)
+    if B > 1:
+        idx = torch.empty((B, cfg.Hkv, cfg.k_kv), dtype=torch.int32, device=dev)
+        counts = torch.empty((B,), dtype=torch.int32, device=dev)
+        k_c = torch.empty((B, cfg.Hkv, cfg.k_kv, cfg.d), dtype=torch.bfloat16, device=dev)
+    else:
+        idx = torch.empty((cfg.Hkv, kk), dtype=torch.int32, device=dev)
+        k_c = torch.empty((cfg.Hkv, kk, cfg.d), dtype=torch.bfloat16, device=dev)
+    v_c = torch.empty_like(k_c) if cfg.with_v else None
+    idx_t = torch.empty((1, min(cfg.k_tsp, cfg.N)), dtype=torch.int32, device=dev) if cfg.k_tsp else None
+    stats = torch.empty((cfg.Hkv, 3), dtype=torch.float32, device=dev) if cfg.layers > 1 else None
+
+    def step(l: int, st):
+        q, k, v = qs[l], ks[l], vs[l]
+        if B > 1:
+            kvc.kvc_score_varlen(q, k, cu, max_len, scores=scores, tsp=tsp, accum=accum, ws=ws_s, dev_err=err,
+                                 stream=st)
+            kvc.kvc_select_topk_varlen(scores, cu, max_len, cfg.w, cfg.pool, cfg.k_kv, idx=idx, counts=counts,
+                                       ws=ws_k, dev_err=err, stream=st)
+            kvc.kvc_gather_kv_varlen(k, v, cu, idx, k_out=k_c, v_out=v_c, dev_err=err, stream=st)
+            return
+        kvc.kvc_score(q, k, scores=scores, tsp=tsp, accum=accum, ws=ws_s, dev_err=err, stream=st)
+        if cfg.k_tsp:
+            kvc.kvc_select_topk(tsp, cfg.w, cfg.pool, cfg.k_tsp, idx=idx_t, ws=ws_t, stream=st)
+        kvc.kvc_select_topk(scores, cfg.w, cfg.pool, cfg.k_kv, idx=idx, ws=ws_k, stream=st)
+        kvc.kvc_gather_kv(k, v, idx, k_out=k_c, v_out=v_c, dev_err=err, stream=st)
+        if stats is not None:
+            kvc.kvc_layer_stats(scores, float(cfg.w * cfg.G), out=stats, stream=st)
+
+    st = torch.cuda.current_stream(dev)
+    for i in range(args.warmup):
+        step(i % cfg.layers, st)
+    torch.cuda.synchronize(dev)
+    if err.item() != 0:
+        raise RuntimeError(f"device error word {err.item()}")
+    nsteps = args.steps
+    launches0 = kvc.launch_count()
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream(dev)
+            for i in range(nsteps):
+                step(i % cfg.layers, cap)
+        torch.cuda.synchronize(dev)
+    launches = kvc.launch_count() - launches0
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev.index)
+    with sampler:
+        torch.cuda.synchronize(dev)
+        t0.record(st)
+        if graph is not None:
+            graph.replay()
+        else:
+            for i in range(nsteps):
+                step(i % cfg.layers, st)
+        t1.record(st)
+        torch.cuda.synchronize(dev)
+    if graph is None:
+        launches = kvc.launch_count() - launches0
+    if err.item() != 0:
+        raise RuntimeError(f"device error word {err.item()} after the timed region")
+    ms = t0.elapsed_time(t1) / nsteps
+    alg = other_bytes(cfg, total)
+    peak, peak_kind = measured_peaks()
+    gbs = alg / (ms * 1e-3) / 1e9
+    line = {"metric": "context tokens scored+compressed/s per layer", "value": total / (ms * 1e-3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": nsteps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": cfg.name, "tokens_per_layer": total, "batch": B, "layers_cycled": cfg.layers,
+                       "N": cfg.N, "H": cfg.H, "Hkv": cfg.Hkv, "d": cfg.d, "w": cfg.w, "pool": cfg.pool,
+                       "k_kv": cfg.k_kv, "k_tsp": cfg.k_tsp, "with_v": cfg.with_v},
+            "hbm": {"alg_bytes_per_layer": alg, "achieved_gbs": round(gbs, 1), "peak": peak,
+                    "peak_kind": peak_kind, "frac": round(gbs / peak, 4)},
+            "gpu_launches": launches, "graph": graph is not None, "clocks": sampler.summary()}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- #
 # CUDA arm
 # --------------------------------------------------------------------------- #
 def main() -> None:
@@ -220,6 +338,8 @@ def main() -> None:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed steps one by one instead of replaying a CUDA graph")
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5"],
+                    help="c3 (the 128K layer) is the headline; the others print their per-layer time")
     ap.add_argument("--tokens", type=int, default=None,
                     help="same layer structure at another N (small cases for profiling)")
     args = ap.parse_args()
@@ -239,6 +359,13 @@ def main() -> None:
 
     if args.impl == "reference":
         run_reference(args, cfg, rank)
+        return
+    if args.workload != "c3":
+        import torch
+        import long_context_kv_window_b200 as kvc
+        torch.cuda.set_device(local)
+        run_other(args, getattr(workloads, args.workload.upper()), torch, kvc, workloads,
+                  torch.device("cuda", local))
         return
 
     import torch
@@ -345,6 +472,8 @@ def main() -> None:
     with sampler:
         ms_step, _, launches = timed_run(with_events=False)
     ms_step_events, per_call, _ = timed_run(with_events=True)
+    if plan.dev_err.item() != 0:
+        raise RuntimeError(f"device error word {plan.dev_err.item()} after the timed region")
 
     # ---- end to end through the public API with host buffers ------------------
     hq, hk, hv, hx = (workloads.torch_bf16(a).pin_memory() for a in (lay.q, lay.k, lay.v, lay.x))

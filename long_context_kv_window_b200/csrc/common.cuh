@@ -67,9 +67,14 @@ struct WsCursor {
 // still runs.  A kernel calls pdl_wait() -- which returns once the previous
 // kernel has completed and its memory is visible -- before it touches global
 // memory that an earlier kernel of the stream writes or reads, and calls
-// pdl_trigger() after its own pdl_wait(): then whatever a kernel reads
-// before its pdl_wait() (inputs of the library call) was complete before the
-// previous kernel passed its own wait.
+// pdl_trigger() (if at all) only after its own pdl_wait(): then whatever a
+// kernel reads before its pdl_wait() (inputs of the library call) was
+// complete before the previous kernel passed its own wait, and a kernel is
+// never started while the kernel two places before it still runs.  Only
+// kernels whose grid is resident at once and whose dependents cannot hold
+// the SMs their own unscheduled CTAs would need trigger early (scoring pass 1,
+// the bias combine, the statistics); the others let their dependents launch
+// at completion.
 struct Launch {
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[2];

@@ -25,7 +25,6 @@ gather_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int64
                  int64_t idx_row_stride, int64_t kk, uint4* __restrict__ k_out,
                  uint4* __restrict__ v_out, int32_t* err) {
   pdl_wait();
-  pdl_trigger();
   // blockIdx.y = b * Hkv + g ; blockIdx.x covers kk * VPR items of that head
   const int bg = blockIdx.y;
   const int g = bg % Hkv;
@@ -74,7 +73,6 @@ gather_hidden_kernel(const uint4* __restrict__ x, int64_t sn_v, int64_t n, int64
                      const int32_t* __restrict__ idx, int64_t kk, uint4* __restrict__ out,
                      int32_t* err) {
   pdl_wait();
-  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t warps = (int64_t)gridDim.x * (kGatherThreads / 32);
   const uint4 zero = make_uint4(0u, 0u, 0u, 0u);

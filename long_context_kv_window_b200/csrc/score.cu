@@ -128,6 +128,7 @@ struct Barriers {
   uint64_t tfull[kMaxBufs];
   uint64_t tempty[kMaxBufs];
   uint64_t bias_ready;  // pass 2: the epilogue wrote the bias block
+  uint64_t gsync[kGroups];  // per epilogue group: its warps finished their previous tile
   uint32_t tmem_base;
   int abort;
 };
@@ -208,6 +209,7 @@ __device__ __forceinline__ void init_barriers(Barriers* bars, int stages, int nb
     tc::mbar_init(&bars->tempty[s], kEpiWarps / kGroups);
   }
   tc::mbar_init(&bars->bias_ready, kEpiThreads);
+  for (int g = 0; g < kGroups; ++g) tc::mbar_init(&bars->gsync[g], kEpiWarps / kGroups);
   bars->abort = 0;
   tc::fence_mbar_init();
 }
@@ -294,14 +296,26 @@ __device__ __forceinline__ void issue_mmas(const ScoreArgs& a, Barriers* bars, u
 
 __device__ __forceinline__ void record_timeout(int32_t* err) { set_dev_err(err, KVC_DEV_ERR_TIMEOUT); }
 
-// Epilogue group: wait until the accumulator of tile t is filled.  An
-// mbarrier wait only tells phases apart by parity, so with fewer buffers than
-// groups (a group then skips uses of its buffer) it first waits for the
-// release of the buffer's previous use, by another group: after that the
-// buffer's tfull barrier is at most one phase behind this use.
-__device__ __forceinline__ bool wait_filled(const ScoreArgs& a, Barriers* bars, int t) {
+// Epilogue warp of group grp, at its it-th tile t: wait until the tile's
+// accumulator is filled.  An mbarrier wait tells phases apart by parity
+// only, so a waiter must never be two phases away from the barrier.  With one
+// buffer per group that holds by construction.  With fewer buffers than
+// groups (a group then skips uses of its buffer):
+//  * the group's warps first meet (gsync): all four have released their
+//    previous tile, so that use's release phase is complete -- otherwise a
+//    fast warp could see a later phase's parity as already passed;
+//  * then each waits for the release of the buffer's previous use, by
+//    another group: after that the buffer's fill barrier is at most one phase
+//    behind this use.
+__device__ __forceinline__ bool wait_filled(const ScoreArgs& a, Barriers* bars, int t, int grp, int it, int lane) {
   const int buf = t % a.nbuf, ub = t / a.nbuf;
-  if (a.nbuf < kGroups && ub > 0 && !tc::mbar_wait(&bars->tempty[buf], (ub - 1) & 1, &bars->abort)) return false;
+  if (a.nbuf < kGroups) {
+    if (it > 0) {
+      if (lane == 0) tc::mbar_arrive(&bars->gsync[grp]);
+      if (!tc::mbar_wait(&bars->gsync[grp], (it - 1) & 1, &bars->abort)) return false;
+    }
+    if (ub > 0 && !tc::mbar_wait(&bars->tempty[buf], (ub - 1) & 1, &bars->abort)) return false;
+  }
   return tc::mbar_wait(&bars->tfull[buf], ub & 1, &bars->abort);
 }
 
@@ -322,6 +336,7 @@ __device__ __forceinline__ void merge_ml(float& M, double& L, float m2, double l
 // Load `ncol` (16 or 32) fp32 columns of this warp's 32 TMEM lanes starting
 // at taddr into x[0..ncol).  Completion: KVC_TMEM_WAIT_LD32(x).
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&x)[kCols], int ncol) {
+  __syncwarp();  // .sync.aligned: the whole warp, converged
   if (ncol == 32) {
     KVC_TMEM_LD32(taddr, x);
   } else {
@@ -339,6 +354,7 @@ __device__ __forceinline__ void walk_columns(uint32_t base, int ncols, Proc&& pr
   const int ng = (ncols + kCols - 1) / kCols;
   tmem_ld_cols(base, xa, min(kCols, ncols));
   for (int gi = 0; gi < ng; gi += 2) {
+    __syncwarp();  // proc() may branch per thread; the TMEM wait and loads need the warp converged
     KVC_TMEM_WAIT_LD32(xa);
     if (gi + 1 < ng)
       tmem_ld_cols(base + (uint32_t)((gi + 1) * kCols), xb, min(kCols, ncols - (gi + 1) * kCols));
@@ -346,6 +362,7 @@ __device__ __forceinline__ void walk_columns(uint32_t base, int ncols, Proc&& pr
       release();
     proc(gi, xa);
     if (gi + 1 < ng) {
+      __syncwarp();
       KVC_TMEM_WAIT_LD32(xb);
       if (gi + 2 < ng)
         tmem_ld_cols(base + (uint32_t)((gi + 2) * kCols), xa, min(kCols, ncols - (gi + 2) * kCols));
@@ -383,7 +400,7 @@ __device__ __forceinline__ float max_cols(const uint32_t (&x)[kCols]) {
 // running sum rescaled.
 __device__ __forceinline__ void pass1_group(uint32_t (&x)[kCols], float c, float& ref, double& l) {
   float s = sum_ex2(x, c, -ref);
-  if (!(s < 0x1p100f)) {  // overflow, or NaN from ref = -inf
+  if (!(s < 0x1p100f)) {  // overflow, or NaN from ref = -inf (a per-thread branch)
     const float hmax = max_cols(x);
     if (hmax == -INFINITY) return;  // every key masked
     const float nr = fmaxf(ref, hmax * c);
@@ -444,9 +461,9 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
     float m_run[2] = {-INFINITY, -INFINITY};
     double l_run[2] = {0.0, 0.0};
     const int64_t first_window_key = wk.len - a.w;  // earliest window row sees keys <= this
-    for (int t = grp; t < ntiles; t += kGroups) {
+    for (int t = grp, it = 0; t < ntiles; t += kGroups, ++it) {
       const int buf = t % a.nbuf;
-      if (!wait_filled(a, bars, t)) break;
+      if (!wait_filled(a, bars, t, grp, it, lane)) break;
       tc::tc_fence_after();
       const int64_t j0 = k0 + (int64_t)t * kTile;  // first key of the tile (sequence-local)
       const bool masked = (j0 + kTile - 1 > first_window_key);
@@ -517,10 +534,10 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
 // one).  Pass 2 multiplies them by ones in one extra MMA K-step.
 // --------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) score_combine_kernel(const ScoreArgs a) {
-  // pass 2 may launch now: its prologue (barriers, TMEM, Q, first K tiles)
-  // reads only the inputs and overlaps pass 1's tail and this kernel
-  pdl_trigger();
+  // pass 2 may launch once pass 1 is complete: its prologue (barriers, TMEM,
+  // Q, first K tiles) then overlaps this kernel
   pdl_wait();
+  pdl_trigger();
   const int g = blockIdx.x, b = blockIdx.y;
   int gid0 = 0, nch = 0;
   bool bad = false;
@@ -587,8 +604,9 @@ __global__ void __launch_bounds__(kThreadsScore, 1)
 score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) {
   // Before pdl_wait() this kernel reads only the call's inputs (Q, K, the
   // sequence offsets) and shared memory; the combined biases and every global
-  // write come after it.
-  pdl_trigger();
+  // write come after it.  Its own dependents may launch only once it is
+  // complete (no early trigger: a dependent resident early could hold the SM
+  // a not yet scheduled CTA of this grid needs).
   extern __shared__ uint8_t smem_raw[];
   const SmemPtrs<D> sp(smem_raw, a);
   Barriers* bars = sp.bars;
@@ -656,9 +674,9 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
     const int q = warp & 3;
     const int kl = 32 * q + lane;  // key within the tile
     const int64_t first_window_key = wk.len - a.w;
-    for (int t = grp; t < ntiles; t += kGroups) {
+    for (int t = grp, it = 0; t < ntiles; t += kGroups, ++it) {
       const int buf = t % a.nbuf;
-      if (!wait_filled(a, bars, t)) break;
+      if (!wait_filled(a, bars, t, grp, it, lane)) break;
       tc::tc_fence_after();
       const int tp = ntiles - 1 - t;                    // tiles are walked backwards
       const int64_t j = k0 + (int64_t)tp * kTile + kl;  // this thread's key (sequence-local)
@@ -715,7 +733,6 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
 // TSP aggregate: tsp[j] = sum_g scores[g][j] (all heads, one row).
 __global__ void tsp_sum_kernel(const float* __restrict__ scores, int Hkv, int64_t total, float* __restrict__ tsp) {
   pdl_wait();
-  pdl_trigger();
   for (int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; j < total; j += (int64_t)gridDim.x * blockDim.x) {
     float s = 0.f;
     for (int g = 0; g < Hkv; ++g) s += scores[(int64_t)g * total + j];
@@ -821,7 +838,9 @@ kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, 
   }
   kvc_status s = set_smem_attrs<D>(std::max(smem[0], smem[1]));
   if (s != KVC_OK) return s;
-  const int grid_x = (int)((a.total + a.chunk_keys - 1) / a.chunk_keys) + a.B;
+  // chunks of all sequences: a bound (every sequence adds at most one partial
+  // chunk); a single sequence needs exactly ceil(total / chunk)
+  const int grid_x = (int)((a.total + a.chunk_keys - 1) / a.chunk_keys) + (a.cu ? a.B : 0);
   for (int g0 = 0; g0 < a.Hkv; g0 += hp) {
     a.g0 = g0;
     dim3 grid(grid_x, std::min(hp, a.Hkv - g0));

@@ -278,7 +278,6 @@ __host__ __device__ inline int64_t sel_segment(int64_t L, int cs) { return ((L +
 template <int CS>
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
   pdl_wait();
-  pdl_trigger();
   __shared__ SelShared sh;
   extern __shared__ __align__(16) float dyn[];
   cg::cluster_group cluster = cg::this_cluster();
