@@ -336,7 +336,6 @@ __device__ __forceinline__ void merge_ml(float& M, double& L, float m2, double l
 // Load `ncol` (16 or 32) fp32 columns of this warp's 32 TMEM lanes starting
 // at taddr into x[0..ncol).  Completion: KVC_TMEM_WAIT_LD32(x).
 __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&x)[kCols], int ncol) {
-  __syncwarp();  // .sync.aligned: the whole warp, converged
   if (ncol == 32) {
     KVC_TMEM_LD32(taddr, x);
   } else {
@@ -348,27 +347,32 @@ __device__ __forceinline__ void tmem_ld_cols(uint32_t taddr, uint32_t (&x)[kCols
 // groups of kCols: the next group's TMEM load is in flight while the current
 // one is processed (proc(gi, x)); release() runs as soon as the last load has
 // landed, so the MMA may refill the buffer during the last group's math.
-template <class Proc, class Release>
+// The TMEM loads and waits are warp-collective (.sync.aligned): the warp is
+// reconverged before the first one, and, when proc() branches or returns per
+// lane (kDiverges), after every proc() call -- the one point every lane of the
+// warp always reaches.
+template <bool kDiverges, class Proc, class Release>
 __device__ __forceinline__ void walk_columns(uint32_t base, int ncols, Proc&& proc, Release&& release) {
   uint32_t xa[kCols], xb[kCols];
   const int ng = (ncols + kCols - 1) / kCols;
+  __syncwarp();
   tmem_ld_cols(base, xa, min(kCols, ncols));
   for (int gi = 0; gi < ng; gi += 2) {
-    __syncwarp();  // proc() may branch per thread; the TMEM wait and loads need the warp converged
     KVC_TMEM_WAIT_LD32(xa);
     if (gi + 1 < ng)
       tmem_ld_cols(base + (uint32_t)((gi + 1) * kCols), xb, min(kCols, ncols - (gi + 1) * kCols));
     else
       release();
     proc(gi, xa);
+    if (kDiverges) __syncwarp();
     if (gi + 1 < ng) {
-      __syncwarp();
       KVC_TMEM_WAIT_LD32(xb);
       if (gi + 2 < ng)
         tmem_ld_cols(base + (uint32_t)((gi + 2) * kCols), xa, min(kCols, ncols - (gi + 2) * kCols));
       else
         release();
       proc(gi + 1, xb);
+      if (kDiverges) __syncwarp();
     }
   }
 }
@@ -468,7 +472,7 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
       const int64_t j0 = k0 + (int64_t)t * kTile;  // first key of the tile (sequence-local)
       const bool masked = (j0 + kTile - 1 > first_window_key);
       const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * a.acc_stride);
-      walk_columns(
+      walk_columns<true>(
           base, a.nb1 * kTile,
           [&](int gi, uint32_t(&x)[kCols]) {
             const int mb = gi / kPerBlock;
@@ -687,7 +691,7 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
       const int rmin = lim <= 0 ? 0 : (int)std::min<int64_t>(lim * a.G, a.Rn);
       const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * a.acc_stride);
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
-      walk_columns(
+      walk_columns<false>(
           base, a.Rn,
           [&](int gi, uint32_t(&x)[kCols]) {
             const int col0 = gi * kCols;
