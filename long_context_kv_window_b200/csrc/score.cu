@@ -26,12 +26,13 @@
 // tiles pass 1 read last, which are still in L2.
 //
 // Warp roles per CTA: warp 0 issues TMA, warp 1 allocates TMEM and issues
-// MMAs, warps 2..17 drain TMEM (epilogue: four groups of four warps, one warp
-// per TMEM lane quarter; the groups take the tiles in turn, so four warps per
-// SM sub-partition hide each other's TMEM-load and MUFU latencies).  Every
-// wait is bounded; on a
-// timeout the CTA records KVC_DEV_ERR_TIMEOUT, lets in-flight copies and MMAs
-// land, frees TMEM and exits.
+// MMAs, the rest drain TMEM (epilogue: one group of four warps, one warp per
+// TMEM lane quarter, for each accumulator buffer -- four buffers of 128
+// columns in the common case, fewer when the accumulator is wider; the groups
+// take the tiles in turn, so up to four warps per SM sub-partition hide each
+// other's TMEM-load and MUFU latencies).  Every wait is bounded; on a timeout
+// the CTA records KVC_DEV_ERR_TIMEOUT, lets in-flight copies and MMAs land,
+// frees TMEM and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -49,14 +50,22 @@ namespace {
 constexpr int kTile = 128;       // keys per tile
 constexpr int kMaxStages = 8;    // TMA ring depth bound (the host picks what fits)
 constexpr int kMaxBufs = 4;      // TMEM accumulator buffers
-constexpr int kEpiWarps = 16;    // groups of four, one warp per TMEM lane quarter
-constexpr int kGroups = kEpiWarps / 4;  // the groups take the tiles in turn
 constexpr int kCols = 32;        // accumulator columns per TMEM load
-constexpr int kThreadsScore = 64 + 32 * kEpiWarps;
-constexpr int kEpiThreads = 32 * kEpiWarps;
 constexpr int kMinChunkTiles = 4;
 constexpr int kBarEpi = 1;       // named barrier of all epilogue warps
 constexpr double kLog2e = 1.4426950408889634;
+
+// Block layout of both passes: warp 0 TMA producer, warp 1 MMA issuer, then
+// one epilogue group of four warps (one per TMEM lane quarter) for each of the
+// NB accumulator buffers.  Group i drains buffer i, i.e. tiles i, i + NB, ...
+// Four groups hide each other's TMEM-load and exponential latencies; with
+// fewer buffers (wide accumulators) a group per buffer beats groups that share
+// one.
+template <int NB>
+struct Epi {
+  static constexpr int kThreads = 128 * NB;
+  static constexpr int kBlock = 64 + kThreads;
+};
 
 struct ScoreArgs {
   const uint16_t* q;
@@ -67,7 +76,7 @@ struct ScoreArgs {
   int Hkv, G, w, R, Rq, Rn;  // rows per KV head, rows in smem, MMA N (pass 2)
   int nb1;                   // 128-row blocks in pass 1
   int acc_stride;            // TMEM columns between accumulator buffers (this pass)
-  int nbuf;                  // TMEM accumulator buffers (this pass): 2 or 4
+  int nbuf;                  // TMEM accumulator buffers = epilogue groups (this pass): 2, 3 or 4
   int stages;                // TMA ring depth
   int fold;                  // pass 2: the row bias rides in one extra MMA K-step
   float keep_frac;           // pass 1: trailing fraction of each chunk left at normal L2 priority
@@ -128,7 +137,6 @@ struct Barriers {
   uint64_t tfull[kMaxBufs];
   uint64_t tempty[kMaxBufs];
   uint64_t bias_ready;  // pass 2: the epilogue wrote the bias block
-  uint64_t gsync[kGroups];  // per epilogue group: its warps finished their previous tile
   uint32_t tmem_base;
   int abort;
 };
@@ -145,7 +153,7 @@ struct Smem {
   static constexpr int kStageBytes = kChunks * kTile * 128;
   static constexpr size_t kOnesBytes = (size_t)kTile * 32;
   static constexpr size_t kTail = 512;  // barriers
-  static constexpr size_t kExchangeBytes = (size_t)(kGroups - 1) * 256 * (4 + 8);
+  static constexpr size_t kExchangeBytes = (size_t)(kMaxBufs - 1) * 256 * (4 + 8);
   static_assert(kExchangeBytes <= (size_t)kStageBytes * 2, "pass-1 exchange must fit in two stages");
   __host__ __device__ static size_t q_bytes(int Rq) { return (size_t)kChunks * Rq * 128; }
   __host__ __device__ static size_t fold_bytes(int Rq, int fold) { return fold ? kOnesBytes + (size_t)Rq * 32 : 0; }
@@ -161,8 +169,8 @@ struct SmemPtrs {
   uint8_t* qb;    // pass 2 only
   uint8_t* kst;
   Barriers* bars;
-  float* ex_m;   // [kGroups - 1][256], in the K ring (pass 1, after the last tile)
-  double* ex_l;  // [kGroups - 1][256]
+  float* ex_m;   // [groups - 1][256], in the K ring (pass 1, after the last tile)
+  double* ex_l;  // [groups - 1][256]
   __device__ SmemPtrs(uint8_t* raw, const ScoreArgs& a) {
     uint8_t* s = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(raw) + 1023) & ~uintptr_t(1023));
     qs = s;
@@ -171,7 +179,7 @@ struct SmemPtrs {
     kst = qs + Smem<D>::q_bytes(a.Rq) + Smem<D>::fold_bytes(a.Rq, a.fold);
     bars = reinterpret_cast<Barriers*>(kst + (size_t)a.stages * Smem<D>::kStageBytes);
     ex_m = reinterpret_cast<float*>(kst);
-    ex_l = reinterpret_cast<double*>(ex_m + (kGroups - 1) * 256);
+    ex_l = reinterpret_cast<double*>(ex_m + (kMaxBufs - 1) * 256);
   }
 };
 
@@ -198,18 +206,17 @@ __device__ __forceinline__ void load_q_swizzled(const ScoreArgs& a, int b, int g
 }
 
 // Barrier init (one thread) for the stage ring and the TMEM buffers.  Each
-// use of a buffer is drained by the four warps of one epilogue group.
-__device__ __forceinline__ void init_barriers(Barriers* bars, int stages, int nbuf) {
+// use of a buffer is drained by the four warps of its epilogue group.
+__device__ __forceinline__ void init_barriers(Barriers* bars, int stages, int nbuf, int epi_threads) {
   for (int s = 0; s < stages; ++s) {
     tc::mbar_init(&bars->full[s], 1);
     tc::mbar_init(&bars->empty[s], 1);
   }
   for (int s = 0; s < nbuf; ++s) {
     tc::mbar_init(&bars->tfull[s], 1);
-    tc::mbar_init(&bars->tempty[s], kEpiWarps / kGroups);
+    tc::mbar_init(&bars->tempty[s], 4);
   }
-  tc::mbar_init(&bars->bias_ready, kEpiThreads);
-  for (int g = 0; g < kGroups; ++g) tc::mbar_init(&bars->gsync[g], kEpiWarps / kGroups);
+  tc::mbar_init(&bars->bias_ready, epi_threads);
   bars->abort = 0;
   tc::fence_mbar_init();
 }
@@ -296,27 +303,15 @@ __device__ __forceinline__ void issue_mmas(const ScoreArgs& a, Barriers* bars, u
 
 __device__ __forceinline__ void record_timeout(int32_t* err) { set_dev_err(err, KVC_DEV_ERR_TIMEOUT); }
 
-// Epilogue warp of group grp, at its it-th tile t: wait until the tile's
-// accumulator is filled.  An mbarrier wait tells phases apart by parity
-// only, so a waiter must never be two phases away from the barrier.  With one
-// buffer per group that holds by construction.  With fewer buffers than
-// groups (a group then skips uses of its buffer):
-//  * the group's warps first meet (gsync): all four have released their
-//    previous tile, so that use's release phase is complete -- otherwise a
-//    fast warp could see a later phase's parity as already passed;
-//  * then each waits for the release of the buffer's previous use, by
-//    another group: after that the buffer's fill barrier is at most one phase
-//    behind this use.
-__device__ __forceinline__ bool wait_filled(const ScoreArgs& a, Barriers* bars, int t, int grp, int it, int lane) {
-  const int buf = t % a.nbuf, ub = t / a.nbuf;
-  if (a.nbuf < kGroups) {
-    if (it > 0) {
-      if (lane == 0) tc::mbar_arrive(&bars->gsync[grp]);
-      if (!tc::mbar_wait(&bars->gsync[grp], (it - 1) & 1, &bars->abort)) return false;
-    }
-    if (ub > 0 && !tc::mbar_wait(&bars->tempty[buf], (ub - 1) & 1, &bars->abort)) return false;
-  }
-  return tc::mbar_wait(&bars->tfull[buf], ub & 1, &bars->abort);
+// Epilogue warp, at tile t of its group: wait until the tile's accumulator is
+// filled.  An mbarrier wait tells phases apart by parity only, so a waiter
+// must never be two phases away from the barrier.  Every group owns one
+// buffer: the buffer's previous use (tile t - nbuf) was this group's own
+// previous tile, filled before and released by this warp, and the MMA cannot
+// refill the buffer again before the group releases tile t -- so the fill
+// barrier is exactly one phase behind this use.
+__device__ __forceinline__ bool wait_filled(const ScoreArgs& a, Barriers* bars, int t) {
+  return tc::mbar_wait(&bars->tfull[t % a.nbuf], (t / a.nbuf) & 1, &bars->abort);
 }
 
 // Online merge of (m, l) pairs in the log2 domain: l * 2^(m - M) summed.
@@ -418,8 +413,8 @@ __device__ __forceinline__ void pass1_group(uint32_t (&x)[kCols], float c, float
 // --------------------------------------------------------------------------
 // pass 1: per-row max / sum over a chunk of keys
 // --------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(kThreadsScore, 1)
+template <int D, int NB>
+__global__ void __launch_bounds__(Epi<NB>::kBlock, 1)
 score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -439,7 +434,7 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   const int64_t k1 = std::min<int64_t>(wk.len, k0 + a.chunk_keys);
   const int ntiles = (int)((k1 - k0 + kTile - 1) / kTile);
 
-  if (threadIdx.x == 0) init_barriers(bars, a.stages, a.nbuf);
+  if (threadIdx.x == 0) init_barriers(bars, a.stages, a.nbuf, Epi<NB>::kThreads);
   if (warp == 0 && lane == 0) tc::prefetch_tmap(&kmap);
   if (warp == 1) {
     tc::tmem_alloc(&bars->tmem_base, a.tmem_cols);
@@ -465,9 +460,9 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
     float m_run[2] = {-INFINITY, -INFINITY};
     double l_run[2] = {0.0, 0.0};
     const int64_t first_window_key = wk.len - a.w;  // earliest window row sees keys <= this
-    for (int t = grp, it = 0; t < ntiles; t += kGroups, ++it) {
+    for (int t = grp; t < ntiles; t += NB) {
       const int buf = t % a.nbuf;
-      if (!wait_filled(a, bars, t, grp, it, lane)) break;
+      if (!wait_filled(a, bars, t)) break;
       tc::tc_fence_after();
       const int64_t j0 = k0 + (int64_t)t * kTile;  // first key of the tile (sequence-local)
       const bool masked = (j0 + kTile - 1 > first_window_key);
@@ -497,7 +492,7 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
           });
     }
     // ---- merge the groups, then one chunk partial per row (combined later)
-    tc::named_bar_sync(kBarEpi, kEpiThreads);
+    tc::named_bar_sync(kBarEpi, Epi<NB>::kThreads);
     if (grp > 0) {
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb) {
@@ -506,7 +501,7 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
         sp.ex_l[(grp - 1) * 256 + mb * kTile + rl] = l_run[mb];
       }
     }
-    tc::named_bar_sync(kBarEpi, kEpiThreads);
+    tc::named_bar_sync(kBarEpi, Epi<NB>::kThreads);
     if (grp == 0 && !bars->abort) {
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb) {
@@ -515,7 +510,7 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
         if (r >= a.R) continue;
         float M = m_run[mb];
         double L = l_run[mb];
-        for (int o = 0; o < kGroups - 1; ++o) merge_ml(M, L, sp.ex_m[o * 256 + mb * kTile + rl], sp.ex_l[o * 256 + mb * kTile + rl]);
+        for (int o = 0; o < NB - 1; ++o) merge_ml(M, L, sp.ex_m[o * 256 + mb * kTile + rl], sp.ex_l[o * 256 + mb * kTile + rl]);
         const size_t slot = ((size_t)g * a.max_chunks + wk.gid) * a.Rq + r;
         a.part_m[slot] = M;
         a.part_l[slot] = L;
@@ -603,8 +598,8 @@ __global__ void __launch_bounds__(256) score_combine_kernel(const ScoreArgs a) {
 // --------------------------------------------------------------------------
 // pass 2: per-key sum of normalised probabilities over the window rows
 // --------------------------------------------------------------------------
-template <int D>
-__global__ void __launch_bounds__(kThreadsScore, 1)
+template <int D, int NB>
+__global__ void __launch_bounds__(Epi<NB>::kBlock, 1)
 score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) {
   // Before pdl_wait() this kernel reads only the call's inputs (Q, K, the
   // sequence offsets) and shared memory; the combined biases and every global
@@ -630,7 +625,7 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   const int64_t k1 = std::min<int64_t>(wk.len, k0 + a.chunk_keys);
   const int ntiles = (int)((k1 - k0 + kTile - 1) / kTile);
 
-  if (threadIdx.x == 0) init_barriers(bars, a.stages, a.nbuf);
+  if (threadIdx.x == 0) init_barriers(bars, a.stages, a.nbuf, Epi<NB>::kThreads);
   if (warp == 0 && lane == 0) tc::prefetch_tmap(&kmap);
   if (warp == 1) {
     tc::tmem_alloc(&bars->tmem_base, a.tmem_cols);
@@ -678,9 +673,9 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
     const int q = warp & 3;
     const int kl = 32 * q + lane;  // key within the tile
     const int64_t first_window_key = wk.len - a.w;
-    for (int t = grp, it = 0; t < ntiles; t += kGroups, ++it) {
+    for (int t = grp; t < ntiles; t += NB) {
       const int buf = t % a.nbuf;
-      if (!wait_filled(a, bars, t, grp, it, lane)) break;
+      if (!wait_filled(a, bars, t)) break;
       tc::tc_fence_after();
       const int tp = ntiles - 1 - t;                    // tiles are walked backwards
       const int64_t j = k0 + (int64_t)tp * kTile + kl;  // this thread's key (sequence-local)
@@ -778,11 +773,12 @@ Geometry geometry(const kvc_score_params* p) {
   g.Rn = (g.R + 15) / 16 * 16;
   g.nb1 = (g.R + kTile - 1) / kTile;
   g.Rq = std::max(g.nb1 * kTile, g.Rn);
-  // as many accumulator buffers (4, else 2) as the 512 TMEM columns allow
+  // as many accumulator buffers (at most 4) as the 512 TMEM columns allow:
+  // pass 1 4 or 2 (one or two 128-row blocks), pass 2 4, 3 or 2 (Rn <= 256)
   g.stride1 = g.nb1 * kTile;
-  g.nbuf1 = (kMaxBufs * g.stride1 <= 512) ? kMaxBufs : 2;
+  g.nbuf1 = std::min(kMaxBufs, 512 / g.stride1);
   g.stride2 = (g.Rn + 31) / 32 * 32;
-  g.nbuf2 = (kMaxBufs * g.stride2 <= 512) ? kMaxBufs : 2;
+  g.nbuf2 = std::min(kMaxBufs, 512 / g.stride2);
   g.cols1 = pow2_cols(g.nbuf1 * g.stride1);
   g.cols2 = pow2_cols(g.nbuf2 * g.stride2);
   return g;
@@ -822,8 +818,11 @@ kvc_status set_smem_attrs(size_t bytes) {
   KVC_CUDA_TRY(cudaGetDevice(&dev));
   std::lock_guard<std::mutex> lk(mu);
   if (dev < 64 && (done >> dev) & 1) return KVC_OK;
-  KVC_CUDA_TRY(cudaFuncSetAttribute(score_pass1_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-  KVC_CUDA_TRY(cudaFuncSetAttribute(score_pass2_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+  const void* fns[] = {(const void*)score_pass1_kernel<D, 2>, (const void*)score_pass1_kernel<D, 4>,
+                       (const void*)score_pass2_kernel<D, 2>, (const void*)score_pass2_kernel<D, 3>,
+                       (const void*)score_pass2_kernel<D, 4>};
+  for (const void* f : fns)
+    KVC_CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
   if (dev < 64) done |= (uint64_t)1 << dev;
   return KVC_OK;
 }
@@ -840,6 +839,9 @@ kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, 
     if (stages[pass] < 2) return fail(KVC_ERR_UNSUPPORTED, "score kernel: shared memory too small for 2 stages");
     smem[pass] = Smem<D>::total(a.Rq, stages[pass], pass);
   }
+  // one epilogue group per buffer: only these block shapes are instantiated
+  if ((gm.nbuf1 != 2 && gm.nbuf1 != 4) || gm.nbuf2 < 2 || gm.nbuf2 > 4)
+    return fail(KVC_ERR_UNSUPPORTED, "score kernel: no block shape for this accumulator width");
   kvc_status s = set_smem_attrs<D>(std::max(smem[0], smem[1]));
   if (s != KVC_OK) return s;
   // chunks of all sequences: a bound (every sequence adds at most one partial
@@ -854,8 +856,11 @@ kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, 
     a.stages = stages[0];
     a.fold = 0;
     {
-      const Launch l(grid, dim3(kThreadsScore), smem[0], st);
-      KVC_CUDA_TRY(l.run(score_pass1_kernel<D>, kmap, a));
+      const Launch l(grid, dim3(64 + 128 * a.nbuf), smem[0], st);
+      if (a.nbuf == 4)
+        KVC_CUDA_TRY(l.run(score_pass1_kernel<D, 4>, kmap, a));
+      else
+        KVC_CUDA_TRY(l.run(score_pass1_kernel<D, 2>, kmap, a));
     }
     {
       const Launch l(dim3(a.Hkv, a.B), dim3(256), 0, st);
@@ -868,8 +873,13 @@ kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, 
     a.stages = stages[1];
     a.fold = 1;
     {
-      const Launch l(grid, dim3(kThreadsScore), smem[1], st);
-      KVC_CUDA_TRY(l.run(score_pass2_kernel<D>, kmap, a));
+      const Launch l(grid, dim3(64 + 128 * a.nbuf), smem[1], st);
+      if (a.nbuf == 4)
+        KVC_CUDA_TRY(l.run(score_pass2_kernel<D, 4>, kmap, a));
+      else if (a.nbuf == 3)
+        KVC_CUDA_TRY(l.run(score_pass2_kernel<D, 3>, kmap, a));
+      else
+        KVC_CUDA_TRY(l.run(score_pass2_kernel<D, 2>, kmap, a));
     }
     count_launch(2);
   }
