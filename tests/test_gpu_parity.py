@@ -218,6 +218,25 @@ def test_d128_shapes(N, H, Hkv, w, pool, k):
     check_layer(lay, cfg, g["scores"], g["idx"], what=f"H={H} Hkv={Hkv} N={N}")
 
 
+@pytest.mark.parametrize("base,N,H,Hkv,w,pool,k", [
+    ("C2", 3000, 68, 4, 8, 7, 500),   # R = 136: pass 2 three 160-column buffers, 144-row MMA (16-column tail)
+    ("C2", 2500, 48, 8, 32, 3, 400),  # R = 192: two 192-column buffers in pass 2, two 256 in pass 1
+    ("C2", 2000, 64, 8, 32, 1, 300),  # R = 256: the widest accumulator, 512 TMEM columns in both passes
+    ("C2", 1500, 10, 2, 8, 5, 200),   # R = 40: four 64-column buffers, 48-row MMA
+    ("C1", 2000, 34, 2, 8, 7, 300),   # d = 64, R = 136
+])
+def test_wide_window_rows(base, N, H, Hkv, w, pool, k):
+    """Window row counts past one 128-row block and ragged MMA widths: the
+    accumulator widths that leave room for fewer TMEM buffers (one epilogue
+    group per buffer) and the 16-column tail of the column walk."""
+    cfg = workloads.shrink(getattr(workloads, base), N=N, H=H, Hkv=Hkv, w=w, pool=pool, k_kv=k,
+                           n_sinks=4, n_hitters=8, seed=5000 + H)
+    lay = workloads.make_layer(cfg)
+    g = _run_layer(lay, cfg)
+    assert g["err"] == 0
+    check_layer(lay, cfg, g["scores"], g["idx"], what=f"{base} H={H} Hkv={Hkv} w={w}")
+
+
 def test_llama_32k_full_size():
     cfg = workloads.C2
     lay = workloads.make_layer(cfg)
