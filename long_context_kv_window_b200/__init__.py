@@ -111,24 +111,86 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream: Optional[torch.cuda.Stream]):
-    s = stream if stream is not None else torch.cuda.current_stream()
+def _stream(stream: Optional[torch.cuda.Stream], dev: torch.device):
+    """The launch stream: the given one, else the current stream of `dev`
+    (the device every tensor of the call lives on)."""
+    s = stream if stream is not None else torch.cuda.current_stream(dev)
+    if s.device != dev:
+        raise ValueError(f"stream is on {s.device}, the tensors on {dev}")
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _bf16(t: torch.Tensor, name: str) -> torch.Tensor:
-    if t.dtype not in (torch.bfloat16, torch.int16, torch.uint16):
-        raise TypeError(f"{name} must hold bf16 values (bfloat16 or int16/uint16 bits)")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor")
-    if t.stride(-1) != 1:
-        raise ValueError(f"{name} must be contiguous in its last dimension")
+def _call(dev: torch.device, fn, *args) -> int:
+    """Run one libkvc entry point with `dev` current (kernel launches and the
+    per-device function attributes refer to the current device)."""
+    with torch.cuda.device(dev):
+        return fn(*args)
+
+
+# The C entry points take raw pointers and sizes and cannot see a tensor's
+# extent; the checks below make every pointer passed cover what the call
+# reads or writes through it.
+_BF16_BITS = (torch.bfloat16, torch.int16, torch.uint16)  # 2-byte storage of bf16 values
+
+
+def _dense(t: torch.Tensor, name: str, shape, dtype, dev: torch.device) -> torch.Tensor:
+    """A caller-supplied output the kernels address densely: exact shape,
+    contiguous.  dtype: one dtype, or a tuple of accepted ones."""
+    ok = t.dtype in dtype if isinstance(dtype, tuple) else t.dtype == dtype
+    if not ok or t.device != dev:
+        raise TypeError(f"{name} must be a {dtype} tensor on {dev}")
+    if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous tensor of shape {tuple(shape)}, got {tuple(t.shape)}")
     return t
 
 
-def _dev(t: torch.Tensor, name: str, dtype: torch.dtype) -> torch.Tensor:
-    if t.dtype != dtype or not t.is_cuda:
-        raise TypeError(f"{name} must be a CUDA {dtype} tensor")
+def _vector(t: Optional[torch.Tensor], name: str, numel: int, dtype: torch.dtype, dev: torch.device):
+    """An optional contiguous array of exactly `numel` elements (any shape)."""
+    if t is None:
+        return None
+    if t.dtype != dtype or t.device != dev:
+        raise TypeError(f"{name} must be a {dtype} tensor on {dev}")
+    if t.numel() != numel or not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous with {numel} elements, got shape {tuple(t.shape)}")
+    return t
+
+
+def _rows(t: torch.Tensor, name: str, rows: int, min_cols: int, dtype: torch.dtype, dev: torch.device):
+    """A [rows][>= min_cols] matrix addressed by its row stride (unit column stride)."""
+    if t.dtype != dtype or t.device != dev:
+        raise TypeError(f"{name} must be a {dtype} tensor on {dev}")
+    if t.dim() != 2 or t.shape[0] != rows or t.shape[1] < min_cols or (t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be [{rows}][>= {min_cols}] with unit column stride, got {tuple(t.shape)}")
+    return t
+
+
+def _err_word(t: Optional[torch.Tensor], dev: torch.device):
+    if t is not None and (t.dtype != torch.int32 or t.device != dev or t.numel() < 1):
+        raise TypeError(f"dev_err must be an int32 tensor on {dev} with at least one element")
+    return t
+
+
+def _ws_bytes(t: torch.Tensor, dev: torch.device) -> int:
+    if t.device != dev or not t.is_contiguous():
+        raise ValueError(f"ws must be a contiguous tensor on {dev}")
+    return t.numel() * t.element_size()
+
+
+def _same_device(dev: torch.device, **ts) -> None:
+    for name, t in ts.items():
+        if t is not None and t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the other inputs on {dev}")
+
+
+def _bf16(t: torch.Tensor, name: str, dim: int) -> torch.Tensor:
+    if t.dtype not in _BF16_BITS:
+        raise TypeError(f"{name} must hold bf16 values (bfloat16 or int16/uint16 bits)")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dim() != dim:
+        raise ValueError(f"{name} must have {dim} dimensions, got shape {tuple(t.shape)}")
+    if t.stride(-1) != 1:
+        raise ValueError(f"{name} must be contiguous in its last dimension")
     return t
 
 
@@ -150,25 +212,37 @@ def score_workspace_size(p: ScoreParams, batch: int, total: int) -> int:
     return int(out.value)
 
 
+def _score_outputs(dev, Hkv: int, total: int, scores, tsp, accum, dev_err):
+    if scores is None:
+        scores = torch.empty((Hkv, total), dtype=torch.float32, device=dev)
+    _dense(scores, "scores", (Hkv, total), torch.float32, dev)
+    _vector(tsp, "tsp", total, torch.float32, dev)
+    if accum is not None:
+        _dense(accum, "accum", (Hkv, total), torch.float32, dev)
+    _err_word(dev_err, dev)
+    return scores
+
+
 def kvc_score(q_win: torch.Tensor, k: torch.Tensor, scale: Optional[float] = None,
               scores: Optional[torch.Tensor] = None, tsp: Optional[torch.Tensor] = None,
               accum: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
               dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Window-attention aggregate A [Hkv][n] (fp32) of q_win [w][H][d] over k [n][Hkv][d]."""
-    _bf16(q_win, "q_win")
-    _bf16(k, "k")
+    _bf16(q_win, "q_win", 3)
+    _bf16(k, "k", 3)
+    dev = k.device
+    _same_device(dev, q_win=q_win)
     w, H, d = q_win.shape
     n, Hkv, dk = k.shape
     if dk != d:
         raise ValueError("head_dim of q_win and k differ")
     p = score_params(H, Hkv, d, w, scale)
-    if scores is None:
-        scores = torch.empty((Hkv, n), dtype=torch.float32, device=k.device)
+    scores = _score_outputs(dev, Hkv, n, scores, tsp, accum, dev_err)
     if ws is None:
-        ws = _workspace(score_workspace_size(p, 1, n), k.device)
-    _check(lib().kvc_score(_ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k), k.stride(0), k.stride(1),
-                           n, ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum), _ptr(ws),
-                           ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)), "kvc_score")
+        ws = _workspace(score_workspace_size(p, 1, n), dev)
+    _check(_call(dev, lib().kvc_score, _ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k), k.stride(0),
+                 k.stride(1), n, ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum), _ptr(ws),
+                 _ws_bytes(ws, dev), _ptr(dev_err), _stream(stream, dev)), "kvc_score")
     return scores
 
 
@@ -180,16 +254,19 @@ def kvc_score_noalloc(q_win: torch.Tensor, k: torch.Tensor, scale: Optional[floa
     scratch is used instead (for callers that cannot allocate; calls that
     overlap on the GPU race on that scratch).  Pass `scores` to avoid even the
     output allocation here."""
-    _bf16(q_win, "q_win")
-    _bf16(k, "k")
+    _bf16(q_win, "q_win", 3)
+    _bf16(k, "k", 3)
+    dev = k.device
+    _same_device(dev, q_win=q_win)
     w, H, d = q_win.shape
-    n, Hkv, _ = k.shape
+    n, Hkv, dk = k.shape
+    if dk != d:
+        raise ValueError("head_dim of q_win and k differ")
     p = score_params(H, Hkv, d, w, scale)
-    if scores is None:
-        scores = torch.empty((Hkv, n), dtype=torch.float32, device=k.device)
-    _check(lib().kvc_score_noalloc(_ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k), k.stride(0),
-                                   k.stride(1), n, ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum),
-                                   _ptr(dev_err), _stream(stream)), "kvc_score_noalloc")
+    scores = _score_outputs(dev, Hkv, n, scores, tsp, accum, dev_err)
+    _check(_call(dev, lib().kvc_score_noalloc, _ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k),
+                 k.stride(0), k.stride(1), n, ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum),
+                 _ptr(dev_err), _stream(stream, dev)), "kvc_score_noalloc")
     return scores
 
 
@@ -199,21 +276,23 @@ def kvc_score_varlen(q_win: torch.Tensor, k: torch.Tensor, cu_seqlens: torch.Ten
                      ws: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
                      stream=None) -> torch.Tensor:
     """Ragged batch: q_win [B][w][H][d], k [total][Hkv][d] packed, cu_seqlens int32 [B+1]."""
-    _bf16(q_win, "q_win")
-    _bf16(k, "k")
-    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    _bf16(q_win, "q_win", 4)
+    _bf16(k, "k", 3)
+    dev = k.device
+    _same_device(dev, q_win=q_win)
     B, w, H, d = q_win.shape
-    total, Hkv, _ = k.shape
+    total, Hkv, dk = k.shape
+    if dk != d:
+        raise ValueError("head_dim of q_win and k differ")
+    _vector(cu_seqlens, "cu_seqlens", B + 1, torch.int32, dev)
     p = score_params(H, Hkv, d, w, scale)
-    if scores is None:
-        scores = torch.empty((Hkv, total), dtype=torch.float32, device=k.device)
+    scores = _score_outputs(dev, Hkv, total, scores, tsp, accum, dev_err)
     if ws is None:
-        ws = _workspace(score_workspace_size(p, B, total), k.device)
-    _check(lib().kvc_score_varlen(_ptr(q_win), q_win.stride(0), q_win.stride(1), q_win.stride(2), _ptr(k),
-                                  k.stride(0), k.stride(1), _ptr(cu_seqlens), B, total, int(max_seqlen),
-                                  ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum), _ptr(ws),
-                                  ws.numel() * ws.element_size(), _ptr(dev_err), _stream(stream)),
-           "kvc_score_varlen")
+        ws = _workspace(score_workspace_size(p, B, total), dev)
+    _check(_call(dev, lib().kvc_score_varlen, _ptr(q_win), q_win.stride(0), q_win.stride(1), q_win.stride(2),
+                 _ptr(k), k.stride(0), k.stride(1), _ptr(cu_seqlens), B, total, int(max_seqlen),
+                 ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum), _ptr(ws), _ws_bytes(ws, dev),
+                 _ptr(dev_err), _stream(stream, dev)), "kvc_score_varlen")
     return scores
 
 
@@ -227,24 +306,36 @@ def select_workspace_size(out_rows: int, batch: int, total: int) -> int:
     return int(out.value)
 
 
+def _out_rows(rows: int, row_group: int) -> int:
+    if row_group < 1 or rows % row_group:
+        raise ValueError(f"row_group {row_group} must divide the {rows} score rows")
+    return rows // row_group
+
+
 def kvc_select_topk(scores: torch.Tensor, window: int, pool_kernel: int, k: int, row_group: int = 1,
                     n: Optional[int] = None, idx: Optional[torch.Tensor] = None,
                     pooled: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                     stream=None) -> torch.Tensor:
     """Per output row: the k - window best (pooled) prefix positions plus the
     window, ascending.  scores [rows][>= n] fp32; returns int32 [rows/row_group][min(k, n)]."""
-    _dev(scores, "scores", torch.float32)
+    dev = scores.device
+    if scores.dim() != 2:
+        raise ValueError(f"scores must be [rows][n], got shape {tuple(scores.shape)}")
     rows = scores.shape[0]
-    n = scores.shape[1] if n is None else n
-    out_rows = rows // row_group
+    n = scores.shape[1] if n is None else int(n)
+    _rows(scores, "scores", rows, n, torch.float32, dev)
+    out_rows = _out_rows(rows, row_group)
     kout = min(k, n)
     if idx is None:
-        idx = torch.empty((out_rows, kout), dtype=torch.int32, device=scores.device)
+        idx = torch.empty((out_rows, kout), dtype=torch.int32, device=dev)
+    _rows(idx, "idx", out_rows, kout, torch.int32, dev)
+    if pooled is not None:
+        _dense(pooled, "pooled", (out_rows, n - window), torch.float32, dev)
     if ws is None and pooled is None:
-        ws = _workspace(select_workspace_size(out_rows, 1, n), scores.device)
-    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
-    _check(lib().kvc_select_topk(_ptr(scores), rows, scores.stride(0), row_group, n, window, pool_kernel, k,
-                                 _ptr(idx), idx.stride(0), _ptr(pooled), _ptr(ws), nbytes, _stream(stream)),
+        ws = _workspace(select_workspace_size(out_rows, 1, n), dev)
+    nbytes = 0 if ws is None else _ws_bytes(ws, dev)
+    _check(_call(dev, lib().kvc_select_topk, _ptr(scores), rows, scores.stride(0), row_group, n, window,
+                 pool_kernel, k, _ptr(idx), idx.stride(0), _ptr(pooled), _ptr(ws), nbytes, _stream(stream, dev)),
            "kvc_select_topk")
     return idx
 
@@ -256,47 +347,64 @@ def kvc_select_topk_varlen(scores: torch.Tensor, cu_seqlens: torch.Tensor, max_s
                            stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
     """Ragged batch; returns (idx int32 [B][rows/row_group][k] local positions, -1 padded,
     counts int32 [B])."""
-    _dev(scores, "scores", torch.float32)
-    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    dev = scores.device
+    if scores.dim() != 2:
+        raise ValueError(f"scores must be [rows][total], got shape {tuple(scores.shape)}")
     rows, total = scores.shape[0], scores.shape[1]
+    _rows(scores, "scores", rows, total, torch.float32, dev)
     B = cu_seqlens.numel() - 1
-    out_rows = rows // row_group
+    _vector(cu_seqlens, "cu_seqlens", B + 1, torch.int32, dev)
+    out_rows = _out_rows(rows, row_group)
     if idx is None:
-        idx = torch.empty((B, out_rows, k), dtype=torch.int32, device=scores.device)
+        idx = torch.empty((B, out_rows, k), dtype=torch.int32, device=dev)
+    _dense(idx, "idx", (B, out_rows, k), torch.int32, dev)
     if counts is None:
-        counts = torch.empty((B,), dtype=torch.int32, device=scores.device)
+        counts = torch.empty((B,), dtype=torch.int32, device=dev)
+    _vector(counts, "counts", B, torch.int32, dev)
+    _err_word(dev_err, dev)
     if ws is None:
-        ws = _workspace(select_workspace_size(out_rows, B, total), scores.device)
-    _check(lib().kvc_select_topk_varlen(_ptr(scores), rows, scores.stride(0), row_group, _ptr(cu_seqlens), B,
-                                        total, int(max_seqlen), window, pool_kernel, k, _ptr(idx),
-                                        _ptr(counts), _ptr(ws), ws.numel() * ws.element_size(),
-                                        _ptr(dev_err), _stream(stream)), "kvc_select_topk_varlen")
+        ws = _workspace(select_workspace_size(out_rows, B, total), dev)
+    _check(_call(dev, lib().kvc_select_topk_varlen, _ptr(scores), rows, scores.stride(0), row_group,
+                 _ptr(cu_seqlens), B, total, int(max_seqlen), window, pool_kernel, k, _ptr(idx), _ptr(counts),
+                 _ptr(ws), _ws_bytes(ws, dev), _ptr(dev_err), _stream(stream, dev)), "kvc_select_topk_varlen")
     return idx, counts
 
 
 # --------------------------------------------------------------------------- #
 # gathers
 # --------------------------------------------------------------------------- #
+def _kv_pair(k: torch.Tensor, v: Optional[torch.Tensor]) -> torch.device:
+    _bf16(k, "k", 3)
+    if v is not None:
+        _bf16(v, "v", 3)
+        _same_device(k.device, v=v)
+        if v.stride() != k.stride() or v.shape != k.shape:
+            raise ValueError("k and v must have the same shape and strides")
+    return k.device
+
+
 def kvc_gather_kv(k: torch.Tensor, v: Optional[torch.Tensor], idx: torch.Tensor,
                   k_out: Optional[torch.Tensor] = None, v_out: Optional[torch.Tensor] = None,
                   dev_err: Optional[torch.Tensor] = None, stream=None):
     """k, v [n][Hkv][d]; idx int32 [Hkv][kk] (or [1][kk] broadcast) -> k_out, v_out [Hkv][kk][d]."""
-    _bf16(k, "k")
-    if v is not None:
-        _bf16(v, "v")
-        if v.stride() != k.stride() or v.shape != k.shape:
-            raise ValueError("k and v must have the same shape and strides")
-    _dev(idx, "idx", torch.int32)
+    dev = _kv_pair(k, v)
     n, Hkv, d = k.shape
-    kk = idx.shape[-1]
+    if idx.dim() != 2 or idx.shape[0] not in (1, Hkv):
+        raise ValueError(f"idx must be [{Hkv}][kk] or [1][kk], got shape {tuple(idx.shape)}")
+    kk = idx.shape[1]
+    _rows(idx, "idx", idx.shape[0], kk, torch.int32, dev)
     irs = 0 if idx.shape[0] == 1 and Hkv > 1 else idx.stride(0)
     if k_out is None:
-        k_out = torch.empty((Hkv, kk, d), dtype=k.dtype, device=k.device)
-    if v is not None and v_out is None:
-        v_out = torch.empty((Hkv, kk, d), dtype=v.dtype, device=v.device)
-    _check(lib().kvc_gather_kv(_ptr(k), _ptr(v), k.stride(0), k.stride(1), n, Hkv, d, _ptr(idx), irs, kk,
-                               _ptr(k_out), _ptr(v_out if v is not None else None), _ptr(dev_err),
-                               _stream(stream)), "kvc_gather_kv")
+        k_out = torch.empty((Hkv, kk, d), dtype=k.dtype, device=dev)
+    _dense(k_out, "k_out", (Hkv, kk, d), _BF16_BITS, dev)
+    if v is not None:
+        if v_out is None:
+            v_out = torch.empty((Hkv, kk, d), dtype=v.dtype, device=dev)
+        _dense(v_out, "v_out", (Hkv, kk, d), _BF16_BITS, dev)
+    _err_word(dev_err, dev)
+    _check(_call(dev, lib().kvc_gather_kv, _ptr(k), _ptr(v), k.stride(0), k.stride(1), n, Hkv, d, _ptr(idx),
+                 irs, kk, _ptr(k_out), _ptr(v_out if v is not None else None), _ptr(dev_err),
+                 _stream(stream, dev)), "kvc_gather_kv")
     return k_out, v_out
 
 
@@ -305,32 +413,41 @@ def kvc_gather_kv_varlen(k: torch.Tensor, v: Optional[torch.Tensor], cu_seqlens:
                          v_out: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
                          stream=None):
     """k, v [total][Hkv][d]; idx int32 [B][Hkv][kk] local positions -> [B][Hkv][kk][d]."""
-    _bf16(k, "k")
-    _dev(idx, "idx", torch.int32)
-    _dev(cu_seqlens, "cu_seqlens", torch.int32)
+    dev = _kv_pair(k, v)
     total, Hkv, d = k.shape
+    if idx.dim() != 3 or idx.shape[1] != Hkv:
+        raise ValueError(f"idx must be [B][{Hkv}][kk], got shape {tuple(idx.shape)}")
     B, _, kk = idx.shape
+    _dense(idx, "idx", (B, Hkv, kk), torch.int32, dev)
+    _vector(cu_seqlens, "cu_seqlens", B + 1, torch.int32, dev)
     if k_out is None:
-        k_out = torch.empty((B, Hkv, kk, d), dtype=k.dtype, device=k.device)
-    if v is not None and v_out is None:
-        v_out = torch.empty((B, Hkv, kk, d), dtype=v.dtype, device=v.device)
-    _check(lib().kvc_gather_kv_varlen(_ptr(k), _ptr(v), k.stride(0), k.stride(1), _ptr(cu_seqlens), B, total,
-                                      Hkv, d, _ptr(idx), kk, _ptr(k_out), _ptr(v_out if v is not None else None),
-                                      _ptr(dev_err), _stream(stream)), "kvc_gather_kv_varlen")
+        k_out = torch.empty((B, Hkv, kk, d), dtype=k.dtype, device=dev)
+    _dense(k_out, "k_out", (B, Hkv, kk, d), _BF16_BITS, dev)
+    if v is not None:
+        if v_out is None:
+            v_out = torch.empty((B, Hkv, kk, d), dtype=v.dtype, device=dev)
+        _dense(v_out, "v_out", (B, Hkv, kk, d), _BF16_BITS, dev)
+    _err_word(dev_err, dev)
+    _check(_call(dev, lib().kvc_gather_kv_varlen, _ptr(k), _ptr(v), k.stride(0), k.stride(1), _ptr(cu_seqlens),
+                 B, total, Hkv, d, _ptr(idx), kk, _ptr(k_out), _ptr(v_out if v is not None else None),
+                 _ptr(dev_err), _stream(stream, dev)), "kvc_gather_kv_varlen")
     return k_out, v_out
 
 
 def kvc_gather_hidden(x: torch.Tensor, idx: torch.Tensor, out: Optional[torch.Tensor] = None,
                       dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """x [n][D] -> out [kk][D] = x[idx]."""
-    _bf16(x, "x")
-    _dev(idx, "idx", torch.int32)
+    _bf16(x, "x", 2)
+    dev = x.device
     n, D = x.shape
     kk = idx.numel()
+    _vector(idx, "idx", kk, torch.int32, dev)
     if out is None:
-        out = torch.empty((kk, D), dtype=x.dtype, device=x.device)
-    _check(lib().kvc_gather_hidden(_ptr(x), x.stride(0), n, D, _ptr(idx), kk, _ptr(out), _ptr(dev_err),
-                                   _stream(stream)), "kvc_gather_hidden")
+        out = torch.empty((kk, D), dtype=x.dtype, device=dev)
+    _dense(out, "out", (kk, D), _BF16_BITS, dev)
+    _err_word(dev_err, dev)
+    _check(_call(dev, lib().kvc_gather_hidden, _ptr(x), x.stride(0), n, D, _ptr(idx), kk, _ptr(out),
+                 _ptr(dev_err), _stream(stream, dev)), "kvc_gather_hidden")
     return out
 
 
@@ -340,13 +457,17 @@ def kvc_gather_hidden(x: torch.Tensor, idx: torch.Tensor, out: Optional[torch.Te
 def kvc_layer_stats(scores: torch.Tensor, mass_norm: float, n: Optional[int] = None,
                     out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Per row of scores: [entropy, top-1% mass, variance] of scores/mass_norm."""
-    _dev(scores, "scores", torch.float32)
+    dev = scores.device
+    if scores.dim() != 2:
+        raise ValueError(f"scores must be [rows][n], got shape {tuple(scores.shape)}")
     rows = scores.shape[0]
-    n = scores.shape[1] if n is None else n
+    n = scores.shape[1] if n is None else int(n)
+    _rows(scores, "scores", rows, n, torch.float32, dev)
     if out is None:
-        out = torch.empty((rows, 3), dtype=torch.float32, device=scores.device)
-    _check(lib().kvc_layer_stats(_ptr(scores), rows, scores.stride(0), n, float(mass_norm), _ptr(out), None, 0,
-                                 _stream(stream)), "kvc_layer_stats")
+        out = torch.empty((rows, 3), dtype=torch.float32, device=dev)
+    _dense(out, "out", (rows, 3), torch.float32, dev)
+    _check(_call(dev, lib().kvc_layer_stats, _ptr(scores), rows, scores.stride(0), n, float(mass_norm),
+                 _ptr(out), None, 0, _stream(stream, dev)), "kvc_layer_stats")
     return out
 
 
