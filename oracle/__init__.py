@@ -58,6 +58,9 @@ class Oracle:
         lib.oracle_window_scores.argtypes = [_P, _I64, _I64, _P, _I64, _I64, _I64,
                                              _I32, _I32, _I32, _I32, ctypes.c_double, _P]
         lib.oracle_window_scores.restype = _I32
+        lib.oracle_window_scores_lse.argtypes = [_P, _I64, _I64, _P, _I64, _I64, _I64, _I32, _I32, _I32, _I32,
+                                                 ctypes.c_double, _P, _I64, _I64, _P]
+        lib.oracle_window_scores_lse.restype = _I32
         lib.oracle_sum_rows.argtypes = [_P, _I32, _I64, _I64, _P]
         lib.oracle_sum_rows.restype = None
         lib.oracle_avg_pool.argtypes = [_P, _I64, _I32, _P]
@@ -86,6 +89,26 @@ class Oracle:
                                            N, H, Hkv, d, w, float(scale), A.ctypes.data)
         if rc != 0:
             raise ValueError("oracle_window_scores: bad arguments")
+        return A
+
+    def window_scores_lse(self, q: np.ndarray, k: np.ndarray, lse: np.ndarray, H: int, Hkv: int, w: int,
+                          scale: float) -> np.ndarray:
+        """A[g, j] (float64 [Hkv][N]) with each window row's log-sum-exp given:
+        lse [w][H] (any strides), lse[i, h] = ln sum over the keys row i of head
+        h sees of exp(scale * q . k)."""
+        assert q.dtype == np.uint16 and k.dtype == np.uint16
+        assert q.strides[2] == 2 and k.strides[2] == 2
+        N, Hk, d = k.shape
+        assert Hk == Hkv and q.shape == (w, H, d)
+        lse = np.asarray(lse, dtype=np.float64)
+        assert lse.shape == (w, H)
+        A = np.empty((Hkv, N), dtype=np.float64)
+        rc = self.lib.oracle_window_scores_lse(q.ctypes.data, q.strides[0] // 2, q.strides[1] // 2,
+                                               k.ctypes.data, k.strides[0] // 2, k.strides[1] // 2,
+                                               N, H, Hkv, d, w, float(scale), lse.ctypes.data,
+                                               lse.strides[0] // 8, lse.strides[1] // 8, A.ctypes.data)
+        if rc != 0:
+            raise ValueError("oracle_window_scores_lse: bad arguments")
         return A
 
     def sum_rows(self, rows: np.ndarray) -> np.ndarray:

@@ -166,6 +166,59 @@ int oracle_window_scores(const uint16_t* q, int64_t q_si, int64_t q_sh,
   return 0;
 }
 
+/*
+ * The same aggregate with each window row's softmax normaliser given instead
+ * of computed: lse[i*ls_i + h*ls_h] = ln sum_{j <= N-w+i} exp(scale * q[i,h] . k[j,g])
+ * for window row i of query head h (the log-sum-exp a causal prefill
+ * attention produces for that query).  By the definition of the softmax,
+ *   A[g*N + j] = sum over h of group g, i with j <= N-w+i, of
+ *                exp(scale * q[i,h] . k[j,g] - lse[i,h]),
+ * which equals oracle_window_scores when lse is the true log-sum-exp.  FastKV
+ * section 2.A: the TSP layer runs full attention over the prompt, so these
+ * normalisers exist before the token scores are formed.
+ */
+int oracle_window_scores_lse(const uint16_t* q, int64_t q_si, int64_t q_sh,
+                             const uint16_t* k, int64_t k_sn, int64_t k_sh,
+                             int64_t N, int H, int Hkv, int d, int w, double scale,
+                             const double* lse, int64_t ls_i, int64_t ls_h, double* A) {
+  if (!q || !k || !lse || !A || H <= 0 || Hkv <= 0 || H % Hkv || d <= 0 || w < 1 || w > N)
+    return -1;
+  const int G = H / Hkv;
+  const int R = G * w;
+  double* kd = (double*)malloc(sizeof(double) * (size_t)N * d);
+  double* qd = (double*)malloc(sizeof(double) * (size_t)R * d);
+  double* z = (double*)malloc(sizeof(double) * R);
+  int64_t* last = (int64_t*)malloc(sizeof(int64_t) * R);
+  if (!kd || !qd || !z || !last) {
+    free(kd); free(qd); free(z); free(last);
+    return -1;
+  }
+  for (int g = 0; g < Hkv; ++g) {
+    for (int64_t j = 0; j < N; ++j)
+      for (int c = 0; c < d; ++c) kd[j * d + c] = bf16_to_f64(k[j * k_sn + (int64_t)g * k_sh + c]);
+    int r = 0;
+    for (int h = 0; h < H; ++h) {
+      if (kv_head_of(h, H, Hkv) != g) continue;
+      for (int i = 0; i < w; ++i, ++r) {
+        for (int c = 0; c < d; ++c) qd[r * d + c] = bf16_to_f64(q[i * q_si + (int64_t)h * q_sh + c]);
+        last[r] = last_visible(N, w, i);
+        z[r] = lse[(int64_t)i * ls_i + (int64_t)h * ls_h];
+      }
+    }
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < N; ++j) {
+      double a = 0.0;
+      for (int rr = 0; rr < R; ++rr) {
+        if (j > last[rr]) continue;
+        a += exp(logit(qd + rr * d, kd + j * d, d, scale) - z[rr]);
+      }
+      A[(int64_t)g * N + j] = a;
+    }
+  }
+  free(kd); free(qd); free(z); free(last);
+  return 0;
+}
+
 /* out[j] = sum_r rows[r*stride + j], r = 0..nrows-1 (TSP aggregate, C_global). */
 void oracle_sum_rows(const double* rows, int nrows, int64_t stride, int64_t n, double* out) {
   for (int64_t j = 0; j < n; ++j) {

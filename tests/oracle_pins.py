@@ -11,7 +11,8 @@ Sources the pins come from (none of them is the oracle's own code):
   * closed form: with K = 0 every visible logit is 0, so each window row is
     uniform over the keys it may see;
   * a library attention routine: torch's scaled_dot_product_attention in
-    float64 with V = identity returns the attention probabilities;
+    float64 with V = identity returns the attention probabilities (with the
+    rows' normalisers given, scipy's logsumexp supplies them);
   * arbitrary-precision brute force (mpmath) on tiny inputs;
   * the total mass invariant sum_j A[g, j] = w * G;
   * scipy's zero-padded uniform filter for the pooling;
@@ -96,6 +97,79 @@ def pin_sdpa(orc):
         err = np.max(np.abs(A - ref) / np.maximum(ref, 1e-300))
         if err > 1e-10:
             return f"SDPA(V=I) mismatch (N={N}, H={H}, Hkv={Hkv}, w={w}): rel err {err:.3e}"
+    return None
+
+
+def logsumexp_rows(q_bits, k_bits, H, Hkv, w, scale):
+    """lse [w][H]: scipy's logsumexp of each window row's visible logits,
+    the normaliser a causal prefill attention returns for that query."""
+    from scipy.special import logsumexp
+    q, k = _widen(q_bits), _widen(k_bits)
+    N = k.shape[0]
+    G = H // Hkv
+    out = np.empty((w, H))
+    for h in range(H):
+        s = scale * (q[:, h, :] @ k[:, h // G, :].T)   # [w][N]
+        for i in range(w):
+            out[i, h] = logsumexp(s[i, : N - w + i + 1])
+    return out
+
+
+def pin_lse_sdpa(orc):
+    """Given the true row log-sum-exp, the scores are the SDPA probabilities
+    summed over the group's heads and the window rows."""
+    rng = np.random.default_rng(19)
+    for (N, H, Hkv, d, w) in [(48, 6, 2, 64, 5), (70, 8, 2, 128, 12)]:
+        q, k = _rand_qk(rng, N, H, Hkv, d, w, qscale=1.5)
+        scale = 1 / math.sqrt(d)
+        lse = logsumexp_rows(q, k, H, Hkv, w, scale)
+        lse_view = np.ascontiguousarray(lse.T).T          # [w][H] view of [H][w] storage
+        A = orc.window_scores_lse(q, k, lse_view, H, Hkv, w, scale)
+        P = sdpa_probabilities(q, k, H, Hkv, w, scale)
+        ref = P.reshape(Hkv, H // Hkv, w, N).sum(axis=(1, 2))
+        err = np.max(np.abs(A - ref) / np.maximum(ref, 1e-300))
+        if err > 1e-10:
+            return f"given-lse scores != SDPA(V=I) (N={N}, H={H}, Hkv={Hkv}, w={w}): rel err {err:.3e}"
+    return None
+
+
+def pin_lse_zero_keys(orc):
+    """K = 0 with lse[i, h] = ln(#visible keys of row i): the uniform closed form."""
+    for (N, H, Hkv, d, w) in [(40, 4, 2, 64, 6), (19, 3, 1, 64, 19)]:
+        q = _bf16(np.random.default_rng(N).standard_normal((w, H, d)))
+        k = np.zeros((N, Hkv, d), dtype=np.uint16)
+        lse = np.log(N - w + np.arange(w) + 1.0)[:, None].repeat(H, axis=1)
+        A = orc.window_scores_lse(q, k, lse, H, Hkv, w, 1 / math.sqrt(d))
+        ref = closed_form_zero_keys(N, H, Hkv, w)
+        err = np.max(np.abs(A - ref) / ref)
+        if err > 1e-13:
+            return f"given-lse K=0 closed form violated (N={N}, w={w}): rel err {err:.3e}"
+    return None
+
+
+def pin_lse_shift(orc):
+    """exp(s - lse - delta) = exp(-delta) exp(s - lse): shifting one row's
+    normaliser scales exactly that row's contribution."""
+    rng = np.random.default_rng(23)
+    N, H, Hkv, d, w = 50, 4, 2, 64, 5
+    q, k = _rand_qk(rng, N, H, Hkv, d, w)
+    scale = 1 / math.sqrt(d)
+    lse = 3.0 * rng.standard_normal((w, H))
+    A0 = orc.window_scores_lse(q, k, lse, H, Hkv, w, scale)
+    i, h, delta = 2, 3, 1.75
+    lse1 = lse.copy()
+    lse1[i, h] += delta
+    A1 = orc.window_scores_lse(q, k, lse1, H, Hkv, w, scale)
+    one = np.full((w, H), np.inf)       # lse = +inf removes a row
+    one[i, h] = lse[i, h]
+    Arow = orc.window_scores_lse(q, k, one, H, Hkv, w, scale)
+    ref = A0 + (math.exp(-delta) - 1.0) * Arow
+    err = np.max(np.abs(A1 - ref) / A0)
+    if err > 1e-13:
+        return f"row normaliser shift not exact: rel err {err:.3e}"
+    g = h // (H // Hkv)
+    if not (np.all(Arow[1 - g] == 0) and np.all(Arow[g, N - w + i + 1:] == 0) and np.all(Arow[g, : N - w + i + 1] > 0)):
+        return "a single row's contribution reaches keys it may not see or another KV head"
     return None
 
 
@@ -287,5 +361,5 @@ def pin_stats(orc):
     return None
 
 
-ALL_PINS = [pin_zero_keys, pin_sdpa, pin_mpmath, pin_mass, pin_dominant_key, pin_pool,
-            pin_select, pin_gather, pin_stats]
+ALL_PINS = [pin_zero_keys, pin_sdpa, pin_mpmath, pin_mass, pin_dominant_key, pin_lse_sdpa, pin_lse_zero_keys,
+            pin_lse_shift, pin_pool, pin_select, pin_gather, pin_stats]
