@@ -123,6 +123,32 @@ kvc_status kvc_score(const uint16_t* q_win, int64_t q_stride_w, int64_t q_stride
                      void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
 
 /*
+ * kvc_score with the window rows' softmax normalisers supplied by the
+ * caller  [FastKV 2.A: the TSP layer runs full attention over the prompt, so
+ * every window query's normaliser already exists when the token scores are
+ * formed; the softmax definition then gives each probability from its logit
+ * and that normaliser alone].
+ *
+ *  lse  fp32, element (i, h) at lse[i*lse_stride_w + h*lse_stride_h]:
+ *       ln sum_{j <= n - w + i} exp(scale * q[i, h, :] . k[j, g, :]), the
+ *       natural-log log-sum-exp that a causal prefill attention returns for
+ *       the query at position n - w + i (e.g. its [H][seqlen] output viewed
+ *       at columns n - w .. n - 1: lse_stride_w = 1, lse_stride_h = seqlen).
+ *       Finite values; strides >= 0.
+ *     scores[g * n + j] = sum_{h in g} sum_{i : j <= n - w + i}
+ *                         exp(scale * q[i, h, :] . k[j, g, :] - lse[i, h])
+ *  which equals kvc_score's result when lse is the true log-sum-exp.  Only
+ *  the second pass over K runs (one read of K instead of two).  Every other
+ *  argument, the workspace (kvc_score_workspace_size(p, 1, n)) and the
+ *  error behaviour are those of kvc_score.
+ */
+kvc_status kvc_score_lse(const uint16_t* q_win, int64_t q_stride_w, int64_t q_stride_h,
+                         const uint16_t* k, int64_t k_stride_n, int64_t k_stride_h, int64_t n,
+                         const kvc_score_params* p, const float* lse, int64_t lse_stride_w,
+                         int64_t lse_stride_h, float* scores, float* tsp, float* accum, void* ws,
+                         size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/*
  * Ragged batch version of kvc_score.  Sequence b occupies packed tokens
  * [cu_seqlens[b], cu_seqlens[b+1]); its window is its own last w tokens.
  *  q_win       [B][w][H][d] bf16 (q_stride_b, q_stride_w, q_stride_h)

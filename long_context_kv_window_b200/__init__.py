@@ -54,6 +54,8 @@ _SIGS = {
     "kvc_score_varlen": ([_P, _I64, _I64, _I64, _P, _I64, _I64, _P, _I32, _I64, _I64, _P, _P, _P, _P,
                           _P, _SZ, _P, _P], _I32),
     "kvc_score_noalloc": ([_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _I32),
+    "kvc_score_lse": ([_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _I64, _I64, _P, _P, _P, _P, _SZ, _P, _P],
+                      _I32),
     "kvc_select_workspace_size": ([_I32, _I32, _I64, _P], _I32),
     "kvc_select_topk": ([_P, _I32, _I64, _I32, _I64, _I32, _I32, _I64, _P, _I64, _P, _P, _SZ, _P], _I32),
     "kvc_select_topk_varlen": ([_P, _I32, _I64, _I32, _P, _I32, _I64, _I64, _I32, _I32, _I64, _P, _P, _P,
@@ -243,6 +245,37 @@ def kvc_score(q_win: torch.Tensor, k: torch.Tensor, scale: Optional[float] = Non
     _check(_call(dev, lib().kvc_score, _ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k), k.stride(0),
                  k.stride(1), n, ctypes.byref(p), _ptr(scores), _ptr(tsp), _ptr(accum), _ptr(ws),
                  _ws_bytes(ws, dev), _ptr(dev_err), _stream(stream, dev)), "kvc_score")
+    return scores
+
+
+def kvc_score_lse(q_win: torch.Tensor, k: torch.Tensor, lse: torch.Tensor, scale: Optional[float] = None,
+                  scores: Optional[torch.Tensor] = None, tsp: Optional[torch.Tensor] = None,
+                  accum: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                  dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """kvc_score with the window rows' softmax normalisers given: lse fp32
+    [w][H] (any strides), lse[i, h] = ln of the sum of exp(scale * q . k) over
+    the keys window row i of query head h sees -- the log-sum-exp a causal
+    prefill attention returns, e.g. its [H][n] output viewed as
+    ``lse_full[:, n - w:].t()``.  One pass over K instead of two."""
+    _bf16(q_win, "q_win", 3)
+    _bf16(k, "k", 3)
+    dev = k.device
+    _same_device(dev, q_win=q_win)
+    w, H, d = q_win.shape
+    n, Hkv, dk = k.shape
+    if dk != d:
+        raise ValueError("head_dim of q_win and k differ")
+    if lse.dtype != torch.float32 or lse.device != dev:
+        raise TypeError(f"lse must be a float32 tensor on {dev}")
+    if tuple(lse.shape) != (w, H):
+        raise ValueError(f"lse must be [{w}][{H}] (window row, query head), got {tuple(lse.shape)}")
+    p = score_params(H, Hkv, d, w, scale)
+    scores = _score_outputs(dev, Hkv, n, scores, tsp, accum, dev_err)
+    if ws is None:
+        ws = _workspace(score_workspace_size(p, 1, n), dev)
+    _check(_call(dev, lib().kvc_score_lse, _ptr(q_win), q_win.stride(0), q_win.stride(1), _ptr(k), k.stride(0),
+                 k.stride(1), n, ctypes.byref(p), _ptr(lse), lse.stride(0), lse.stride(1), _ptr(scores), _ptr(tsp),
+                 _ptr(accum), _ptr(ws), _ws_bytes(ws, dev), _ptr(dev_err), _stream(stream, dev)), "kvc_score_lse")
     return scores
 
 

@@ -525,6 +525,20 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
   }
 }
 
+// -bias / c as three bf16 parts (words w0 = h1 | h2 << 16, w1 = h3) whose fp32
+// sum is accurate to ~2^-26 relative: each part holds the rounding residual
+// of the previous one.
+__device__ __forceinline__ uint2 split_bias3(double v) {
+  const __nv_bfloat16 h1 = __float2bfloat16_rn((float)v);
+  const double r1 = v - (double)__bfloat162float(h1);
+  const __nv_bfloat16 h2 = __float2bfloat16_rn((float)r1);
+  const double r2 = r1 - (double)__bfloat162float(h2);
+  const __nv_bfloat16 h3 = __float2bfloat16_rn((float)r2);
+  return make_uint2((uint32_t)__bfloat16_as_ushort(h1) | ((uint32_t)__bfloat16_as_ushort(h2) << 16),
+                    (uint32_t)__bfloat16_as_ushort(h3));
+}
+constexpr uint32_t kPadBias = 0xFF7Fu;  // padded row: -3.39e38, so 2^(x * c) = 0
+
 // --------------------------------------------------------------------------
 // between the passes: per (sequence, KV head, row) combine the chunk partials
 // into the row's bias b_r = M + log2(sum_c l_c 2^(m_c - M)), M = max_c m_c,
@@ -553,7 +567,7 @@ __global__ void __launch_bounds__(256) score_combine_kernel(const ScoreArgs a) {
   }
   if (bad) return;
   for (int r = threadIdx.x; r < a.Rn; r += blockDim.x) {
-    uint32_t w0 = 0xFF7Fu, w1 = 0u;  // padded row: -3.39e38, so 2^(x * c) = 0
+    uint2 bias = make_uint2(kPadBias, 0u);
     if (r < a.R) {
       const float* pm = a.part_m + ((size_t)g * a.max_chunks + gid0) * a.Rq + r;
       const double* pl = a.part_l + ((size_t)g * a.max_chunks + gid0) * a.Rq + r;
@@ -582,16 +596,30 @@ __global__ void __launch_bounds__(256) score_combine_kernel(const ScoreArgs a) {
         L = (M == -INFINITY) ? acc : L * (double)exp2f(M - Mn) + acc;
         M = Mn;
       }
-      const double v = -((double)M + log2(L)) / (double)a.c;
-      const __nv_bfloat16 h1 = __float2bfloat16_rn((float)v);
-      const double r1 = v - (double)__bfloat162float(h1);
-      const __nv_bfloat16 h2 = __float2bfloat16_rn((float)r1);
-      const double r2 = r1 - (double)__bfloat162float(h2);
-      const __nv_bfloat16 h3 = __float2bfloat16_rn((float)r2);
-      w0 = (uint32_t)__bfloat16_as_ushort(h1) | ((uint32_t)__bfloat16_as_ushort(h2) << 16);
-      w1 = (uint32_t)__bfloat16_as_ushort(h3);
+      bias = split_bias3(-((double)M + log2(L)) / (double)a.c);
     }
-    a.qsplit[((size_t)b * a.Hkv + g) * a.Rq + r] = make_uint2(w0, w1);
+    a.qsplit[((size_t)b * a.Hkv + g) * a.Rq + r] = bias;
+  }
+}
+
+// With the rows' softmax normalisers given -- lse[i][h] = ln of the sum of
+// exp(scale * q.k) over the keys window row i of query head h sees, the
+// log-sum-exp a causal prefill attention returns for that query -- row
+// r = i*G + h_local has b_r = lse * log2(e) in the log2 domain, and pass 2
+// needs only -b_r / c = -lse / scale: pass 1 and the combine do not run.
+// One sequence; grid = KV heads.
+__global__ void __launch_bounds__(256) score_lse_bias_kernel(const ScoreArgs a, const float* __restrict__ lse,
+                                                             int64_t ls_w, int64_t ls_h) {
+  pdl_wait();  // an earlier kernel of the stream may still read the bias block
+  pdl_trigger();
+  const int g = blockIdx.x;
+  for (int r = threadIdx.x; r < a.Rn; r += blockDim.x) {
+    uint2 bias = make_uint2(kPadBias, 0u);
+    if (r < a.R) {
+      const int i = r / a.G, h = g * a.G + r % a.G;
+      bias = split_bias3(-((double)lse[(int64_t)i * ls_w + (int64_t)h * ls_h] * kLog2e) / (double)a.c);
+    }
+    a.qsplit[(size_t)g * a.Rq + r] = bias;
   }
 }
 
@@ -827,8 +855,15 @@ kvc_status set_smem_attrs(size_t bytes) {
   return KVC_OK;
 }
 
+// The window rows' log-sum-exp when the caller has it (one sequence), else none.
+struct GivenLse {
+  const float* p = nullptr;
+  int64_t sw = 0, sh = 0;  // strides (elements) of window row and query head
+};
+
 template <int D>
-kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, int hp, cudaStream_t st) {
+kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, int hp, const GivenLse& lse,
+                      cudaStream_t st) {
   // deepest TMA ring that fits next to the other blocks in 227 KB of shared memory
   const size_t budget = 227 * 1024;
   int stages[2];
@@ -855,18 +890,24 @@ kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, 
     a.tmem_cols = gm.cols1;
     a.stages = stages[0];
     a.fold = 0;
-    {
-      const Launch l(grid, dim3(64 + 128 * a.nbuf), smem[0], st);
-      if (a.nbuf == 4)
-        KVC_CUDA_TRY(l.run(score_pass1_kernel<D, 4>, kmap, a));
-      else
-        KVC_CUDA_TRY(l.run(score_pass1_kernel<D, 2>, kmap, a));
+    if (lse.p == nullptr) {
+      {
+        const Launch l(grid, dim3(64 + 128 * a.nbuf), smem[0], st);
+        if (a.nbuf == 4)
+          KVC_CUDA_TRY(l.run(score_pass1_kernel<D, 4>, kmap, a));
+        else
+          KVC_CUDA_TRY(l.run(score_pass1_kernel<D, 2>, kmap, a));
+      }
+      {
+        const Launch l(dim3(a.Hkv, a.B), dim3(256), 0, st);
+        KVC_CUDA_TRY(l.run(score_combine_kernel, a));
+      }
+      count_launch(2);
+    } else {
+      const Launch l(dim3(a.Hkv), dim3(256), 0, st);
+      KVC_CUDA_TRY(l.run(score_lse_bias_kernel, a, lse.p, lse.sw, lse.sh));
+      count_launch();
     }
-    {
-      const Launch l(dim3(a.Hkv, a.B), dim3(256), 0, st);
-      KVC_CUDA_TRY(l.run(score_combine_kernel, a));
-    }
-    count_launch();
     a.acc_stride = gm.stride2;
     a.nbuf = gm.nbuf2;
     a.tmem_cols = gm.cols2;
@@ -881,7 +922,7 @@ kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, 
       else
         KVC_CUDA_TRY(l.run(score_pass2_kernel<D, 2>, kmap, a));
     }
-    count_launch(2);
+    count_launch();
   }
   return KVC_OK;
 }
@@ -889,9 +930,10 @@ kvc_status launch_all(const CUtensorMap& kmap, ScoreArgs a, const Geometry& gm, 
 kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_sh, const uint16_t* k,
                       int64_t k_sn, int64_t k_sh, const int32_t* cu, int B, int64_t total,
                       const kvc_score_params* p, float* scores, float* tsp, float* accum, void* ws,
-                      size_t ws_bytes, int32_t* err, cudaStream_t st) {
+                      size_t ws_bytes, int32_t* err, cudaStream_t st, const GivenLse& lse = GivenLse{}) {
   kvc_status s = check_params(p);
   if (s != KVC_OK) return s;
+  KVC_CHECK_ARG(lse.p == nullptr || (cu == nullptr && B == 1), "a given log-sum-exp needs one sequence");
   KVC_CHECK_ARG(q && k && scores, "q_win, k and scores must be non-NULL");
   KVC_CHECK_ARG(aligned(q, 16) && aligned(k, 16), "q_win and k must be 16-byte aligned");
   KVC_CHECK_ARG(q_sw % 8 == 0 && q_sh % 8 == 0 && q_sb % 8 == 0 && q_sw >= 0 && q_sh >= 0 && q_sb >= 0,
@@ -972,7 +1014,7 @@ kvc_status score_impl(const uint16_t* q, int64_t q_sb, int64_t q_sw, int64_t q_s
   a.accum = accum;
   a.total = total;
   a.err = err;
-  s = (d == 128) ? launch_all<128>(kmap, a, gm, hp, st) : launch_all<64>(kmap, a, gm, hp, st);
+  s = (d == 128) ? launch_all<128>(kmap, a, gm, hp, lse, st) : launch_all<64>(kmap, a, gm, hp, lse, st);
   if (s != KVC_OK) return s;
   if (tsp) {
     const int threads = 256;
@@ -1010,6 +1052,25 @@ extern "C" kvc_status kvc_score(const uint16_t* q_win, int64_t q_stride_w, int64
   KVC_CHECK_ARG(n >= p->window && n < (int64_t(1) << 31), "need window <= n < 2^31");
   return score_impl(q_win, 0, q_stride_w, q_stride_h, k, k_stride_n, k_stride_h, nullptr, 1, n, p, scores, tsp,
                     accum, ws, ws_bytes, dev_err, (cudaStream_t)stream);
+}
+
+extern "C" kvc_status kvc_score_lse(const uint16_t* q_win, int64_t q_stride_w, int64_t q_stride_h,
+                                    const uint16_t* k, int64_t k_stride_n, int64_t k_stride_h, int64_t n,
+                                    const kvc_score_params* p, const float* lse, int64_t lse_stride_w,
+                                    int64_t lse_stride_h, float* scores, float* tsp, float* accum, void* ws,
+                                    size_t ws_bytes, int32_t* dev_err, void* stream) {
+  clear_error();
+  kvc_status s = check_params(p);
+  if (s != KVC_OK) return s;
+  KVC_CHECK_ARG(n >= p->window && n < (int64_t(1) << 31), "need window <= n < 2^31");
+  KVC_CHECK_ARG(lse != nullptr, "lse must be non-NULL");
+  KVC_CHECK_ARG(lse_stride_w >= 0 && lse_stride_h >= 0, "lse strides must be >= 0");
+  GivenLse given;
+  given.p = lse;
+  given.sw = lse_stride_w;
+  given.sh = lse_stride_h;
+  return score_impl(q_win, 0, q_stride_w, q_stride_h, k, k_stride_n, k_stride_h, nullptr, 1, n, p, scores, tsp,
+                    accum, ws, ws_bytes, dev_err, (cudaStream_t)stream, given);
 }
 
 extern "C" kvc_status kvc_score_varlen(const uint16_t* q_win, int64_t q_stride_b, int64_t q_stride_w,

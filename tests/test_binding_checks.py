@@ -143,6 +143,21 @@ def test_score_checks_outputs(lib):
     assert lib.calls == ["kvc_score", "kvc_score_noalloc"]
 
 
+def test_score_lse_checks_the_normalisers(lib):
+    w, H, Hkv, d, n = 4, 8, 2, 64, 100
+    q, k = torch.empty((w, H, d), dtype=bf), torch.empty((n, Hkv, d), dtype=bf)
+    full = torch.empty((H, n), dtype=f32)          # a prefill attention's [H][n] log-sum-exp
+    kvc.kvc_score_lse(q, k, full[:, n - w:].t(), ws=_ws())
+    assert lib.calls == ["kvc_score_lse"]
+    for bad in (full[:, n - w:], torch.empty((w, H), dtype=torch.float64), torch.empty((w, H + 1), dtype=f32),
+                torch.empty((w, H), dtype=f32, device="meta")):
+        with pytest.raises((ValueError, TypeError)):
+            kvc.kvc_score_lse(q, k, bad, ws=_ws())
+    with pytest.raises(ValueError):
+        kvc.kvc_score_lse(q, k, full[:, n - w:].t(), scores=torch.empty((Hkv, n - 1), dtype=f32), ws=_ws())
+    assert lib.calls == ["kvc_score_lse"]
+
+
 def test_score_varlen_checks_seqlens_and_outputs(lib):
     B, w, H, Hkv, d, total = 3, 4, 8, 2, 64, 300
     q, k = torch.empty((B, w, H, d), dtype=bf), torch.empty((total, Hkv, d), dtype=bf)

@@ -10,7 +10,7 @@ import torch
 import long_context_kv_window_b200 as kvc
 import oracle
 import workloads
-from tests import parity
+from tests import oracle_pins, parity
 from tests.gpu_helpers import check_layer, dev_bf16, host_bits
 
 pytestmark = pytest.mark.gpu
@@ -437,3 +437,31 @@ def test_shared_accumulator_buffers_repeated_calls_stable():
         assert torch.equal(s, ref)
     torch.cuda.synchronize()
     assert err.item() == 0
+
+
+# --------------------------------------------------------------------------- #
+# one-pass scoring with the window rows' log-sum-exp given
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("base,N,H,Hkv,w", [("C2", 5000, 32, 8, 32), ("C2", 3000, 40, 8, 32), ("C1", 1500, 8, 2, 8)])
+def test_score_with_given_log_sum_exp(base, N, H, Hkv, w):
+    """kvc_score_lse against the oracle given the same fp32 normalisers,
+    passed as a prefill attention lays them out ([H][n], viewed at the window
+    columns), and against the two-pass kvc_score; the head-sum row too."""
+    cfg = workloads.shrink(getattr(workloads, base), N=N, H=H, Hkv=Hkv, w=w, n_sinks=4, n_hitters=8,
+                           seed=6000 + N)
+    lay = workloads.make_layer(cfg, with_x=False)
+    lse = oracle_pins.logsumexp_rows(lay.q, lay.k, H, Hkv, w, cfg.scale)      # float64 [w][H]
+    full = np.zeros((H, N), dtype=np.float32)
+    full[:, N - w:] = lse.T
+    lse_dev = torch.from_numpy(full).cuda()[:, N - w:].t()                   # [w][H], strides (1, N)
+    q, kd = dev_bf16(lay.q), dev_bf16(lay.k)
+    err = _err_word()
+    tsp = torch.empty(N, dtype=torch.float32, device="cuda")
+    got = kvc.kvc_score_lse(q, kd, lse_dev, tsp=tsp, dev_err=err)
+    two = kvc.kvc_score(q, kd, dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref = oracle.get().window_scores_lse(lay.q, lay.k, full[:, N - w:].T.astype(np.float64), H, Hkv, w, cfg.scale)
+    parity.assert_scores_close(got.cpu().numpy(), ref, what="given-lse scores")
+    parity.assert_scores_close(tsp.cpu().numpy(), ref.sum(axis=0), what="given-lse head-sum row")
+    parity.assert_scores_close(got.cpu().numpy(), two.cpu().numpy().astype(np.float64), what="one pass vs two")
