@@ -71,6 +71,8 @@ class Oracle:
         lib.oracle_gather_rows.restype = _I64
         lib.oracle_layer_stats.argtypes = [_P, _I64, ctypes.c_double, _P]
         lib.oracle_layer_stats.restype = _I32
+        lib.oracle_pivot_layer.argtypes = [_P, _I32, _I32, ctypes.c_double, _I32, _I32]
+        lib.oracle_pivot_layer.restype = _I32
         lib.oracle_max_threads.restype = _I32
         lib.oracle_mutant.restype = _I32
         self.lib = lib
@@ -151,6 +153,17 @@ class Oracle:
                                        out.ctypes.data) != 0:
             raise ValueError("oracle_layer_stats: bad arguments")
         return out
+
+    def pivot_layer(self, stats: np.ndarray, tau: float, l_min: int, l_max: int) -> int:
+        """Pivot layer (1-based) from per-layer, per-KV-head statistics
+        stats [L][Hkv][3] float32 (entropy, top-1% mass, variance)."""
+        st = np.ascontiguousarray(stats, dtype=np.float32)
+        assert st.ndim == 3 and st.shape[2] == 3
+        r = int(self.lib.oracle_pivot_layer(st.ctypes.data, st.shape[0], st.shape[1], float(tau), int(l_min),
+                                            int(l_max)))
+        if r < 0:
+            raise ValueError("oracle_pivot_layer: bad arguments")
+        return r
 
     def max_threads(self) -> int:
         return int(self.lib.oracle_max_threads())

@@ -371,3 +371,37 @@ int oracle_layer_stats(const double* A, int64_t N, double mass_norm, double* out
   free(a);
   return 0;
 }
+
+/*
+ * Dynamic pivot detection, online  [StructKV section 2.B: the per-layer
+ * attention entropy, sparsity and variance are watched, and the pivot layer
+ * is where the entropy falls sharply while the sparsity rises].  The page
+ * fixes neither the statistic per layer nor the threshold; reading taken:
+ *   E_l, S_l = mean over the layer's KV-head rows of the entropy and of the
+ *              top-1% mass (the sparsity measure), from the float outputs of
+ *              the layer statistics, summed in float64 in head order;
+ *   the pivot is the first layer l (1-based) with l_min <= l <= l_max and
+ *   l >= 2 such that (E_{l-1} - E_l) >= tau * E_{l-1} and S_l > S_{l-1};
+ *   if none qualifies, l_max.  Variance is monitored but not part of the rule
+ *   (the page's detection sentence names only entropy and sparsity).
+ * stats: [L][Hkv][3] float, per layer and KV head (entropy, top-1% mass,
+ * variance).  Returns the pivot layer, or -1 on bad arguments.
+ */
+int oracle_pivot_layer(const float* stats, int L, int Hkv, double tau, int l_min, int l_max) {
+  if (!stats || L < 1 || Hkv < 1 || !(tau >= 0) || l_min < 1 || l_max < l_min || l_max > L) return -1;
+  double E_prev = 0.0, S_prev = 0.0;
+  for (int l = 1; l <= l_max; ++l) {
+    double E = 0.0, S = 0.0;
+    for (int g = 0; g < Hkv; ++g) {
+      E += (double)stats[((size_t)(l - 1) * Hkv + g) * 3 + 0];
+      S += (double)stats[((size_t)(l - 1) * Hkv + g) * 3 + 1];
+    }
+    E /= (double)Hkv;
+    S /= (double)Hkv;
+    if (l >= 2 && l >= l_min && (E_prev - E) >= tau * E_prev && S > S_prev) return l;
+    E_prev = E;
+    S_prev = S;
+  }
+  return l_max;
+}
+

@@ -361,5 +361,76 @@ def pin_stats(orc):
     return None
 
 
+# --------------------------------------------------------------------------- #
+# dynamic pivot detection
+# --------------------------------------------------------------------------- #
+def _stats(E, S, heads=2):
+    """[L][heads][3] float32 with every head's entropy E[l] and top-1% mass S[l]."""
+    st = np.zeros((len(E), heads, 3), dtype=np.float32)
+    st[:, :, 0] = np.asarray(E, dtype=np.float32)[:, None]
+    st[:, :, 1] = np.asarray(S, dtype=np.float32)[:, None]
+    return st
+
+
+def pin_pivot_hand_cases(orc):
+    """Each clause of the rule on sequences worked out by hand."""
+    flat_s = [0.1] * 6
+    rise_s = [0.1, 0.1, 0.1, 0.2, 0.3, 0.4]
+    cases = [
+        # (E per layer, S per layer, tau, l_min, l_max, expected, what)
+        ([5, 5, 5, 3, 3, 3], rise_s, 0.25, 1, 6, 4, "a 40 % drop with rising sparsity at layer 4"),
+        ([5, 5, 5, 3, 3, 3], flat_s, 0.25, 1, 6, 6, "no sparsity rise: no pivot, l_max"),
+        ([5, 5, 5, 3, 3, 3], rise_s, 0.5, 1, 6, 6, "drop below tau: l_max"),
+        ([4, 4, 4, 3, 2, 2], rise_s, 0.25, 1, 6, 4, "drop of exactly tau * E_prev counts"),
+        ([4, 4, 4, 3.0000002, 2, 2], rise_s, 0.25, 1, 6, 5, "just under tau * E_prev does not"),
+        ([5, 3, 3, 3, 3, 3], [0.1, 0.2, 0.3, 0.4, 0.5, 0.6], 0.25, 3, 6, 6, "a drop before l_min is ignored"),
+        ([5, 5, 5, 5, 5, 3], rise_s, 0.25, 1, 4, 4, "a drop after l_max is ignored"),
+    ]
+    for E, S, tau, lo, hi, want, what in cases:
+        got = orc.pivot_layer(_stats(E, S), tau, lo, hi)
+        if got != want:
+            return f"pivot rule: {what}: got {got}, expected {want}"
+    # the per-layer statistic is the mean over the KV heads
+    st = _stats([4, 4, 4, 4], [0.1, 0.1, 0.2, 0.3])
+    st[2, 0, 0] = 1.0   # one head collapses at layer 3: mean 4 -> 2.5, a 37.5 % drop
+    if orc.pivot_layer(st, 0.3, 1, 4) != 3:
+        return "pivot rule: a head-mean drop above tau did not fire"
+    if orc.pivot_layer(st, 0.4, 1, 4) != 4:
+        return "pivot rule: a head-mean drop below tau fired"
+    st[2, 1, 0] = 7.0   # the other head rises: the mean stays 4, no drop
+    if orc.pivot_layer(st, 0.3, 1, 4) != 4:
+        return "pivot rule: one head's collapse fired without a head-mean drop"
+    return None
+
+
+def _phase_change_scores(rng, N, heads, layer, pivot):
+    """Per-head aggregates of mass 1: flat noise before the pivot layer,
+    a few dominant keys from it on (attention settling on hubs)."""
+    A = rng.random((heads, N)) + 0.5
+    if layer >= pivot:
+        hubs = rng.choice(N, size=8, replace=False)
+        A[:, hubs] += 40.0 * N / 8
+    return A / A.sum(axis=1, keepdims=True)
+
+
+def pin_pivot_synthetic_phase_change(orc):
+    """Statistics of aggregates whose attention concentrates from layer 7 on
+    (computed by the stats routine, itself pinned to closed forms) put the
+    pivot at layer 7; without the change it falls back to l_max."""
+    rng = np.random.default_rng(29)
+    N, heads, L = 4096, 4, 12
+    for pivot, want in ((7, 7), (L + 1, 10)):
+        st = np.zeros((L, heads, 3), dtype=np.float32)
+        for l in range(1, L + 1):
+            A = _phase_change_scores(rng, N, heads, l, pivot)
+            for g in range(heads):
+                st[l - 1, g] = orc.layer_stats(A[g], 1.0)
+        got = orc.pivot_layer(st, 0.1, 2, 10)
+        if got != want:
+            return f"synthetic phase change at layer {pivot}: pivot {got}, expected {want}"
+    return None
+
+
 ALL_PINS = [pin_zero_keys, pin_sdpa, pin_mpmath, pin_mass, pin_dominant_key, pin_lse_sdpa, pin_lse_zero_keys,
-            pin_lse_shift, pin_pool, pin_select, pin_gather, pin_stats]
+            pin_lse_shift, pin_pool, pin_select, pin_gather, pin_stats, pin_pivot_hand_cases,
+            pin_pivot_synthetic_phase_change]
