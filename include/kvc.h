@@ -63,6 +63,7 @@ typedef enum kvc_status {
 #define KVC_DEV_ERR_INDEX 1   /* gather index outside [-1, n) */
 #define KVC_DEV_ERR_SEQLENS 2 /* cu_seqlens not monotone, or a sequence shorter than w */
 #define KVC_DEV_ERR_TIMEOUT 4 /* an internal pipeline wait hit its bound (a bug): outputs invalid */
+#define KVC_DEV_ERR_ORDER 8   /* kvc_pivot_update: a layer folded in out of order */
 
 /* Scoring geometry shared by the score entry points. */
 typedef struct kvc_score_params {
@@ -299,6 +300,39 @@ kvc_status kvc_stats_workspace_size(int32_t rows, int64_t n, size_t* bytes);
  */
 kvc_status kvc_layer_stats(const float* scores, int32_t rows, int64_t row_stride, int64_t n,
                            float mass_norm, float* out, void* ws, size_t ws_bytes, void* stream);
+
+/* Pivot detection ------------------------------------------------------- */
+
+/* Device-resident state of the online pivot rule; zero it before layer 1. */
+typedef struct kvc_pivot_state {
+  double prev_entropy;  /* head-mean entropy of the last layer folded in */
+  double prev_sparsity; /* head-mean top-1% mass of the last layer folded in */
+  int32_t pivot;        /* 0 until decided, then the pivot layer (1-based) */
+  int32_t layers_seen;  /* last layer folded in (0: none) */
+} kvc_pivot_state;
+
+/*
+ * Dynamic pivot detection, online, one layer per call  [StructKV 2.B: the
+ * per-layer attention entropy, sparsity and variance are watched; the pivot
+ * is where the entropy falls sharply while the sparsity rises].  The page
+ * fixes neither the per-layer statistic nor the threshold; the rule is:
+ *     E_l = (1/rows) sum_g stats[3g + 0],  S_l = (1/rows) sum_g stats[3g + 1]
+ * (float64, heads in order), and the pivot is the first layer l with
+ * l_min <= l <= l_max, l >= 2, E_{l-1} - E_l >= tau * E_{l-1} and
+ * S_l > S_{l-1}; if none qualifies, l_max (decided when layer l_max is
+ * folded in).  Variance (stats[3g + 2]) is not part of the rule.
+ *  stats  [rows][3] fp32 device: kvc_layer_stats' output for this layer
+ *  layer  1-based; calls must come in order 1, 2, 3, ... on one state; a call
+ *         whose layer is not state->layers_seen + 1 changes nothing and sets
+ *         KVC_DEV_ERR_ORDER in dev_err
+ *  state  device kvc_pivot_state (zeroed before layer 1); state->pivot holds
+ *         the decision once made, later layers leave it unchanged
+ *  tau >= 0, 1 <= l_min <= l_max
+ * The decision stays on the device (no host synchronisation); read
+ * state->pivot whenever convenient.
+ */
+kvc_status kvc_pivot_update(const float* stats, int32_t rows, int32_t layer, double tau, int32_t l_min,
+                            int32_t l_max, kvc_pivot_state* state, int32_t* dev_err, void* stream);
 
 #ifdef __cplusplus
 }

@@ -26,6 +26,7 @@ KVC_OK = 0
 KVC_DEV_ERR_INDEX = 1
 KVC_DEV_ERR_SEQLENS = 2
 KVC_DEV_ERR_TIMEOUT = 4
+KVC_DEV_ERR_ORDER = 8
 
 
 class KvcError(RuntimeError):
@@ -66,6 +67,7 @@ _SIGS = {
     "kvc_gather_hidden": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P, _P], _I32),
     "kvc_stats_workspace_size": ([_I32, _I64, _P], _I32),
     "kvc_layer_stats": ([_P, _I32, _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P], _I32),
+    "kvc_pivot_update": ([_P, _I32, _I32, ctypes.c_double, _I32, _I32, _P, _P, _P], _I32),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -502,6 +504,35 @@ def kvc_layer_stats(scores: torch.Tensor, mass_norm: float, n: Optional[int] = N
     _check(_call(dev, lib().kvc_layer_stats, _ptr(scores), rows, scores.stride(0), n, float(mass_norm),
                  _ptr(out), None, 0, _stream(stream, dev)), "kvc_layer_stats")
     return out
+
+
+# --------------------------------------------------------------------------- #
+# pivot detection
+# --------------------------------------------------------------------------- #
+def pivot_state(device) -> torch.Tensor:
+    """A zeroed device kvc_pivot_state (24 bytes: two float64, two int32),
+    held as three int64."""
+    return torch.zeros(3, dtype=torch.int64, device=device)
+
+
+def pivot_layer(state: torch.Tensor) -> int:
+    """The decided pivot layer (0 while undecided); reads the device state."""
+    return int(state.view(torch.int32)[4].item())
+
+
+def kvc_pivot_update(stats: torch.Tensor, layer: int, tau: float, l_min: int, l_max: int, state: torch.Tensor,
+                     dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Fold layer `layer`'s statistics (kvc_layer_stats' [rows][3] output) into
+    the online pivot rule held in `state` (see pivot_state); layers in order."""
+    dev = stats.device
+    if stats.dim() != 2 or stats.shape[1] != 3:
+        raise ValueError(f"stats must be [rows][3], got shape {tuple(stats.shape)}")
+    _dense(stats, "stats", (stats.shape[0], 3), torch.float32, dev)
+    _vector(state, "state", 3, torch.int64, dev)
+    _err_word(dev_err, dev)
+    _check(_call(dev, lib().kvc_pivot_update, _ptr(stats), stats.shape[0], int(layer), float(tau), int(l_min),
+                 int(l_max), _ptr(state), _ptr(dev_err), _stream(stream, dev)), "kvc_pivot_update")
+    return state
 
 
 # --------------------------------------------------------------------------- #

@@ -258,3 +258,18 @@ def test_stats_checks(lib):
         with pytest.raises((ValueError, TypeError)):
             kvc.kvc_layer_stats(**args)
     assert lib.calls == ["kvc_layer_stats"]
+
+
+def test_pivot_update_checks(lib):
+    stats = torch.empty((8, 3), dtype=f32)
+    state = torch.zeros(3, dtype=torch.int64)
+    kvc.kvc_pivot_update(stats, 1, 0.1, 2, 10, state)
+    for b in (dict(stats=torch.empty((8, 4), dtype=f32)), dict(stats=torch.empty((3, 8), dtype=f32).t()),
+              dict(state=torch.zeros(2, dtype=torch.int64)), dict(state=torch.zeros(6, dtype=torch.int32)),
+              dict(stats=torch.empty((8, 3), dtype=torch.float64))):
+        args = dict(stats=stats, layer=1, tau=0.1, l_min=2, l_max=10, state=state)
+        args.update(b)
+        with pytest.raises((ValueError, TypeError)):
+            kvc.kvc_pivot_update(**args)
+    assert lib.calls == ["kvc_pivot_update"]
+

@@ -465,3 +465,63 @@ def test_score_with_given_log_sum_exp(base, N, H, Hkv, w):
     parity.assert_scores_close(got.cpu().numpy(), ref, what="given-lse scores")
     parity.assert_scores_close(tsp.cpu().numpy(), ref.sum(axis=0), what="given-lse head-sum row")
     parity.assert_scores_close(got.cpu().numpy(), two.cpu().numpy().astype(np.float64), what="one pass vs two")
+
+
+# --------------------------------------------------------------------------- #
+# dynamic pivot detection
+# --------------------------------------------------------------------------- #
+def _device_pivot(st_np, tau, l_min, l_max):
+    stats = torch.from_numpy(np.ascontiguousarray(st_np, dtype=np.float32)).cuda()
+    state = kvc.pivot_state("cuda")
+    err = _err_word()
+    for layer in range(1, st_np.shape[0] + 1):
+        kvc.kvc_pivot_update(stats[layer - 1], layer, tau, l_min, l_max, state, dev_err=err)
+    torch.cuda.synchronize()
+    return kvc.pivot_layer(state), err.item()
+
+
+def test_pivot_update_matches_oracle():
+    """The device rule, fed one layer at a time, decides exactly the oracle's
+    pivot: random statistic sequences, the hand-worked sequences of the pins,
+    and a phase change whose statistics come from kvc_layer_stats."""
+    orc = oracle.get()
+    rng = np.random.default_rng(31)
+    for trial in range(200):
+        L, heads = int(rng.integers(2, 17)), int(rng.integers(1, 9))
+        E = np.cumsum(-rng.exponential(0.3, size=L)) + 8.0
+        st = np.zeros((L, heads, 3), dtype=np.float32)
+        st[:, :, 0] = E[:, None] + rng.normal(0, 0.2, size=(L, heads))
+        st[:, :, 1] = rng.random((L, heads))
+        st[:, :, 2] = rng.random((L, heads))
+        tau = float(rng.choice([0.0, 0.02, 0.05, 0.1]))
+        l_min = int(rng.integers(1, L + 1))
+        l_max = int(rng.integers(l_min, L + 1))
+        got, err = _device_pivot(st, tau, l_min, l_max)
+        assert err == 0
+        assert got == orc.pivot_layer(st, tau, l_min, l_max), f"trial {trial}"
+    for E, S, tau, lo, hi, want in [([5, 5, 5, 3, 3, 3], [0.1, 0.1, 0.1, 0.2, 0.3, 0.4], 0.25, 1, 6, 4),
+                                    ([4, 4, 4, 3, 2, 2], [0.1, 0.1, 0.1, 0.2, 0.3, 0.4], 0.25, 1, 6, 4),
+                                    ([4, 4, 4, 3.0000002, 2, 2], [0.1, 0.1, 0.1, 0.2, 0.3, 0.4], 0.25, 1, 6, 5)]:
+        st = oracle_pins._stats(E, S)
+        assert _device_pivot(st, tau, lo, hi) == (want, 0)
+    # a phase change at layer 7, statistics on the GPU
+    N, heads, L = 4096, 4, 12
+    st = np.zeros((L, heads, 3), dtype=np.float32)
+    for layer in range(1, L + 1):
+        A = oracle_pins._phase_change_scores(rng, N, heads, layer, 7).astype(np.float32)
+        st[layer - 1] = kvc.kvc_layer_stats(torch.from_numpy(A).cuda(), 1.0).cpu().numpy()
+    assert orc.pivot_layer(st, 0.1, 2, 10) == 7
+    assert _device_pivot(st, 0.1, 2, 10) == (7, 0)
+
+
+def test_pivot_update_out_of_order_is_flagged():
+    stats = torch.rand((4, 3), device="cuda")
+    state = kvc.pivot_state("cuda")
+    err = _err_word()
+    kvc.kvc_pivot_update(stats, 1, 0.1, 1, 8, state, dev_err=err)
+    before = state.clone()
+    kvc.kvc_pivot_update(stats, 3, 0.1, 1, 8, state, dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == kvc.KVC_DEV_ERR_ORDER
+    assert torch.equal(state, before)
+
