@@ -107,3 +107,28 @@ def test_null_pointers_and_bad_sizes_are_rejected(lib):
     assert lib.kvc_score_varlen(dummy, 4096, 512, 64, dummy, 128, 64, dummy, 0, 512, 512, ctypes.byref(p),
                                 dummy, None, None, dummy, 1 << 20, None, None) == 1
     assert lib.kvc_layer_stats(dummy, 2, 512, 512, 0.0, dummy, None, 0, None) == 1
+
+
+def test_given_normaliser_and_pivot_calls_reject_bad_arguments(lib):
+    dummy = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    p = _p()
+    before = kvc.launch_count()
+    # kvc_score_lse: NULL lse, negative lse stride, n < window, workspace too small
+    assert lib.kvc_score_lse(dummy, 512, 64, dummy, 128, 64, 512, ctypes.byref(p), None, 1, 512, dummy, None, None,
+                             dummy, 1 << 20, None, None) == 1
+    assert lib.kvc_score_lse(dummy, 512, 64, dummy, 128, 64, 512, ctypes.byref(p), dummy, -1, 512, dummy, None,
+                             None, dummy, 1 << 20, None, None) == 1
+    assert lib.kvc_score_lse(dummy, 512, 64, dummy, 128, 64, 4, ctypes.byref(p), dummy, 1, 512, dummy, None, None,
+                             dummy, 1 << 20, None, None) == 1
+    assert lib.kvc_score_lse(dummy, 512, 64, dummy, 128, 64, 512, ctypes.byref(p), dummy, 1, 512, dummy, None, None,
+                             dummy, 16, None, None) == 4
+    # kvc_pivot_update: NULL stats, rows 0, layer 0, tau < 0, l_max < l_min, misaligned state
+    state = ctypes.c_void_p(512)
+    assert lib.kvc_pivot_update(None, 8, 1, 0.1, 1, 4, state, None, None) == 1
+    assert lib.kvc_pivot_update(dummy, 0, 1, 0.1, 1, 4, state, None, None) == 1
+    assert lib.kvc_pivot_update(dummy, 8, 0, 0.1, 1, 4, state, None, None) == 1
+    assert lib.kvc_pivot_update(dummy, 8, 1, -0.1, 1, 4, state, None, None) == 1
+    assert lib.kvc_pivot_update(dummy, 8, 1, 0.1, 5, 4, state, None, None) == 1
+    assert lib.kvc_pivot_update(dummy, 8, 1, 0.1, 1, 4, ctypes.c_void_p(516), None, None) == 1
+    assert kvc.last_error() != ""
+    assert kvc.launch_count() == before
