@@ -73,6 +73,8 @@ class Oracle:
         lib.oracle_layer_stats.restype = _I32
         lib.oracle_pivot_layer.argtypes = [_P, _I32, _I32, ctypes.c_double, _I32, _I32]
         lib.oracle_pivot_layer.restype = _I32
+        lib.oracle_decode_attention.argtypes = [_P, _P, _P, _I32, _I32, _I64, _I32, ctypes.c_double, _P]
+        lib.oracle_decode_attention.restype = _I32
         lib.oracle_max_threads.restype = _I32
         lib.oracle_mutant.restype = _I32
         self.lib = lib
@@ -164,6 +166,19 @@ class Oracle:
         if r < 0:
             raise ValueError("oracle_pivot_layer: bad arguments")
         return r
+
+    def decode_attention(self, q: np.ndarray, kc: np.ndarray, vc: np.ndarray, H: int, Hkv: int,
+                         scale: float) -> np.ndarray:
+        """out [H][d] float64: one decode query per head over the compacted
+        cache kc, vc [Hkv][kk][d] (bf16 bits)."""
+        q, kc, vc = (np.ascontiguousarray(a, dtype=np.uint16) for a in (q, kc, vc))
+        Hk, kk, d = kc.shape
+        assert Hk == Hkv and vc.shape == kc.shape and q.shape == (H, d)
+        out = np.empty((H, d), dtype=np.float64)
+        if self.lib.oracle_decode_attention(q.ctypes.data, kc.ctypes.data, vc.ctypes.data, H, Hkv, kk, d,
+                                            float(scale), out.ctypes.data) != 0:
+            raise ValueError("oracle_decode_attention: bad arguments")
+        return out
 
     def max_threads(self) -> int:
         return int(self.lib.oracle_max_threads())

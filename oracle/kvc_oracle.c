@@ -405,3 +405,44 @@ int oracle_pivot_layer(const float* stats, int L, int Hkv, double tau, int l_min
   return l_max;
 }
 
+/*
+ * Decode attention over the compacted cache  [FastKV 2.B: the retained
+ * entries form the KV cache the decoding steps read; FastKV abstract: one
+ * retained set per KV head, shared by its query group].  One new query per
+ * query head, every retained entry visible (positions are already applied to
+ * K before compaction):
+ *   out[h][c] = sum_r softmax_r( scale * q[h] . kc[g][r] ) vc[g][r][c],  g = h / G
+ * q [H][d], kc and vc [Hkv][kk][d], contiguous bf16 bits; out [H][d] float64.
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_decode_attention(const uint16_t* q, const uint16_t* kc, const uint16_t* vc, int H, int Hkv,
+                            int64_t kk, int d, double scale, double* out) {
+  if (!q || !kc || !vc || !out || H <= 0 || Hkv <= 0 || H % Hkv || kk < 1 || d <= 0) return -1;
+  double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+  double* kd = (double*)malloc(sizeof(double) * (size_t)d);
+  double* s = (double*)malloc(sizeof(double) * (size_t)kk);
+  if (!qd || !kd || !s) {
+    free(qd); free(kd); free(s);
+    return -1;
+  }
+  for (int h = 0; h < H; ++h) {
+    const int g = kv_head_of(h, H, Hkv);
+    for (int c = 0; c < d; ++c) qd[c] = bf16_to_f64(q[(int64_t)h * d + c]);
+    double mx = -INFINITY;
+    for (int64_t r = 0; r < kk; ++r) {
+      for (int c = 0; c < d; ++c) kd[c] = bf16_to_f64(kc[((int64_t)g * kk + r) * d + c]);
+      s[r] = logit(qd, kd, d, scale);
+      if (s[r] > mx) mx = s[r];
+    }
+    double z = 0.0;
+    for (int64_t r = 0; r < kk; ++r) z += exp(s[r] - mx);
+    for (int c = 0; c < d; ++c) out[(int64_t)h * d + c] = 0.0;
+    for (int64_t r = 0; r < kk; ++r) {
+      const double p = exp(s[r] - mx) / z;
+      for (int c = 0; c < d; ++c) out[(int64_t)h * d + c] += p * bf16_to_f64(vc[((int64_t)g * kk + r) * d + c]);
+    }
+  }
+  free(qd); free(kd); free(s);
+  return 0;
+}
+

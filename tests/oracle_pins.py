@@ -431,6 +431,48 @@ def pin_pivot_synthetic_phase_change(orc):
     return None
 
 
+# --------------------------------------------------------------------------- #
+# decode attention over the compacted cache
+# --------------------------------------------------------------------------- #
+def pin_decode_sdpa(orc):
+    """Against torch SDPA in float64 (one query per head, every entry visible)."""
+    import torch
+    rng = np.random.default_rng(37)
+    for (H, Hkv, kk, d) in [(8, 2, 50, 64), (6, 3, 7, 128), (4, 4, 1, 64)]:
+        q = _bf16(rng.standard_normal((H, d)) * 1.5)
+        kc = _bf16(rng.standard_normal((Hkv, kk, d)))
+        vc = _bf16(rng.standard_normal((Hkv, kk, d)))
+        scale = 1 / math.sqrt(d)
+        out = orc.decode_attention(q, kc, vc, H, Hkv, scale)
+        G = H // Hkv
+        qt = torch.from_numpy(_widen(q))[:, None, :]                                  # [H][1][d]
+        kt = torch.from_numpy(_widen(kc)).repeat_interleave(G, dim=0)                 # [H][kk][d]
+        vt = torch.from_numpy(_widen(vc)).repeat_interleave(G, dim=0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, scale=scale)[:, 0, :].numpy()
+        err = np.max(np.abs(out - ref)) / max(np.max(np.abs(ref)), 1e-300)
+        if err > 1e-12:
+            return f"decode attention != SDPA (H={H}, Hkv={Hkv}, kk={kk}): err {err:.3e}"
+    return None
+
+
+def pin_decode_closed_forms(orc):
+    """K = 0: each head's output is the mean of its KV head's V rows; one
+    retained entry: exactly that V row."""
+    rng = np.random.default_rng(41)
+    H, Hkv, kk, d = 6, 2, 9, 64
+    q = _bf16(rng.standard_normal((H, d)))
+    vc = _bf16(rng.standard_normal((Hkv, kk, d)))
+    out = orc.decode_attention(q, np.zeros((Hkv, kk, d), dtype=np.uint16), vc, H, Hkv, 0.125)
+    ref = np.repeat(_widen(vc).mean(axis=1), H // Hkv, axis=0)
+    if np.max(np.abs(out - ref)) > 1e-14:
+        return "decode attention with K = 0 is not the mean of V"
+    kc1 = _bf16(rng.standard_normal((Hkv, 1, d)))
+    out1 = orc.decode_attention(q, kc1, vc[:, :1, :], H, Hkv, 0.125)
+    if not np.array_equal(out1, np.repeat(_widen(vc[:, 0, :]), H // Hkv, axis=0)):
+        return "decode attention with one retained entry is not that entry's V row"
+    return None
+
+
 ALL_PINS = [pin_zero_keys, pin_sdpa, pin_mpmath, pin_mass, pin_dominant_key, pin_lse_sdpa, pin_lse_zero_keys,
             pin_lse_shift, pin_pool, pin_select, pin_gather, pin_stats, pin_pivot_hand_cases,
-            pin_pivot_synthetic_phase_change]
+            pin_pivot_synthetic_phase_change, pin_decode_sdpa, pin_decode_closed_forms]
