@@ -75,6 +75,8 @@ class Oracle:
         lib.oracle_pivot_layer.restype = _I32
         lib.oracle_decode_attention.argtypes = [_P, _P, _P, _I32, _I32, _I64, _I32, ctypes.c_double, _P]
         lib.oracle_decode_attention.restype = _I32
+        lib.oracle_rvq_encode.argtypes = [_P, _I64, _I64, _I32, _P, _I32, _I32, _P, _P]
+        lib.oracle_rvq_encode.restype = _I32
         lib.oracle_max_threads.restype = _I32
         lib.oracle_mutant.restype = _I32
         self.lib = lib
@@ -179,6 +181,21 @@ class Oracle:
                                             float(scale), out.ctypes.data) != 0:
             raise ValueError("oracle_decode_attention: bad arguments")
         return out
+
+    def rvq_encode(self, x: np.ndarray, C: np.ndarray):
+        """Residual VQ codes [n][S] int32 and per-stage gaps [n][S] float64 of
+        bf16-bit rows x [n][d] against float32 codebooks C [S][M][d]."""
+        x = np.ascontiguousarray(x, dtype=np.uint16)
+        C = np.ascontiguousarray(C, dtype=np.float32)
+        n, d = x.shape
+        S, M, dc = C.shape
+        assert dc == d
+        codes = np.empty((n, S), dtype=np.int32)
+        gap = np.empty((n, S), dtype=np.float64)
+        if self.lib.oracle_rvq_encode(x.ctypes.data, d, n, d, C.ctypes.data, S, M, codes.ctypes.data,
+                                      gap.ctypes.data) != 0:
+            raise ValueError("oracle_rvq_encode: bad arguments")
+        return codes, gap
 
     def max_threads(self) -> int:
         return int(self.lib.oracle_max_threads())

@@ -446,3 +446,59 @@ int oracle_decode_attention(const uint16_t* q, const uint16_t* kc, const uint16_
   return 0;
 }
 
+/*
+ * Residual vector quantisation of retained K or V rows  [VQKV (gist.science
+ * 2603.16435) section 2: each cached vector is mapped to nearest codewords
+ * stage by stage, the first codebook taking the main approximation and every
+ * later one the residual the earlier stages left].  The codebooks are inputs
+ * (random ones in the tests: trained ones need data).  Reading taken: whole
+ * head rows (d values), squared Euclidean distance, ties to the lowest index:
+ *   r_1 = x,  c_s = argmin_m ||r_s - C_s[m]||^2,  r_{s+1} = r_s - C_s[c_s].
+ * x [n][d] bf16 bits, row stride x_stride elements; C [S][M][d] float32;
+ * codes [n][S] int32 out; gap [n][S] float64 out or NULL: the second-best
+ * minus the best squared distance at each stage (+inf when M == 1).
+ * Returns 0, or -1 on bad arguments.
+ */
+int oracle_rvq_encode(const uint16_t* x, int64_t x_stride, int64_t n, int d, const float* C, int S, int M,
+                      int32_t* codes, double* gap) {
+  if (!x || !C || !codes || n < 0 || d <= 0 || S < 1 || M < 1 || x_stride < d) return -1;
+#pragma omp parallel
+  {
+    double* r = (double*)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(static)
+    for (int64_t t = 0; t < n; ++t) {
+      for (int c = 0; c < d; ++c) r[c] = bf16_to_f64(x[t * x_stride + c]);
+      for (int st = 0; st < S; ++st) {
+        const float* Cs = C + (size_t)st * M * d;
+        double best = INFINITY, second = INFINITY;
+        int arg = 0;
+        for (int m = 0; m < M; ++m) {
+          double dist = 0.0;
+          for (int c = 0; c < d; ++c) {
+            const double e = r[c] - (double)Cs[(size_t)m * d + c];
+            dist += e * e;
+          }
+#if ORACLE_MUTANT == 8
+          if (dist <= best) { /* mutant: ties to the highest index */
+#else
+          if (dist < best) {
+#endif
+            second = best;
+            best = dist;
+            arg = m;
+          } else if (dist < second) {
+            second = dist;
+          }
+        }
+        codes[t * S + st] = arg;
+        if (gap) gap[t * S + st] = second - best;
+#if ORACLE_MUTANT != 7
+        for (int c = 0; c < d; ++c) r[c] -= (double)Cs[(size_t)arg * d + c];
+#endif /* mutant 7: every stage encodes the row itself, not the residual */
+      }
+    }
+    free(r);
+  }
+  return 0;
+}
+

@@ -5,7 +5,8 @@ describing the violation.  The same functions run against the real oracle
 (every one must hold) and against deliberately broken builds of it (each
 broken build must violate at least one), which shows that a plausible
 mistake -- a dropped mask, a dropped scale, a wrong head->group map, a wrong
-pooling divisor, a reversed tie-break, a lost window token -- cannot hide.
+pooling divisor, a reversed tie-break, a lost window token, a residual not
+passed on, a codeword tie to the wrong index -- cannot hide.
 
 Sources the pins come from (none of them is the oracle's own code):
   * closed form: with K = 0 every visible logit is 0, so each window row is
@@ -473,6 +474,74 @@ def pin_decode_closed_forms(orc):
     return None
 
 
+# --------------------------------------------------------------------------- #
+# residual vector quantisation of retained K/V rows
+# --------------------------------------------------------------------------- #
+def _nearest(r, Cs):
+    """scipy's squared-Euclidean distances: (argmin, best, second best) per row."""
+    from scipy.spatial.distance import cdist
+    D = cdist(r, Cs.astype(np.float64), metric="sqeuclidean")
+    order = np.argsort(D, axis=1, kind="stable")
+    rows = np.arange(len(r))
+    return order[:, 0], D[rows, order[:, 0]], D[rows, order[:, 1]]
+
+
+def pin_rvq_nearest_and_residual(orc):
+    """Stage 1 is scipy's nearest codeword; stage 2 is scipy's nearest
+    codeword of the residual the test forms itself; the gaps are scipy's."""
+    rng = np.random.default_rng(43)
+    n, d, M = 300, 32, 64
+    x = _bf16(rng.standard_normal((n, d)))
+    C = rng.standard_normal((2, M, d)).astype(np.float32)
+    codes, gap = orc.rvq_encode(x, C)
+    r = _widen(x)
+    for st in range(2):
+        arg, best, second = _nearest(r, C[st])
+        if not np.array_equal(codes[:, st], arg):
+            return f"stage {st + 1} codes differ from scipy's nearest codeword"
+        if np.max(np.abs(gap[:, st] - (second - best))) > 1e-9:
+            return f"stage {st + 1} gaps differ from scipy's"
+        r = r - C[st][arg].astype(np.float64)
+    return None
+
+
+def pin_rvq_planted_codes(orc):
+    """Codebooks at scales 1, 1/8, 1/64 with entries +-scale: a row built as
+    the sum of one codeword per stage (exact in bf16) gives those codes back
+    and reconstructs exactly."""
+    rng = np.random.default_rng(47)
+    n, d, M, S = 200, 16, 32, 3
+    C = np.stack([rng.choice([-1.0, 1.0], size=(M, d)) * 8.0 ** -s for s in range(S)]).astype(np.float32)
+    planted = rng.integers(0, M, size=(n, S))
+    xf = sum(C[s][planted[:, s]].astype(np.float64) for s in range(S))
+    x = _bf16(xf)
+    if not np.array_equal(_widen(x), xf):
+        return "planted rows are not exact in bf16 (test construction)"
+    codes, gap = orc.rvq_encode(x, C)
+    if not np.array_equal(codes, planted):
+        return "planted codes not recovered"
+    rec = sum(C[s][codes[:, s]].astype(np.float64) for s in range(S))
+    if not np.array_equal(rec, xf) or np.any(gap <= 0):
+        return "planted rows do not reconstruct exactly"
+    return None
+
+
+def pin_rvq_tie_to_lowest_index(orc):
+    """Equal codewords: the lower index wins; the gap is zero."""
+    rng = np.random.default_rng(53)
+    d, M = 16, 10
+    C = rng.standard_normal((1, M, d)).astype(np.float32)
+    C[0, 7] = C[0, 3]
+    x = _bf16(C[0, 3].astype(np.float64)[None, :])
+    C[0, 3] = _widen(x)[0]
+    C[0, 7] = C[0, 3]
+    codes, gap = orc.rvq_encode(x, C)
+    if codes[0, 0] != 3 or gap[0, 0] != 0.0:
+        return f"tie between codewords 3 and 7 gave code {codes[0, 0]}, gap {gap[0, 0]}"
+    return None
+
+
 ALL_PINS = [pin_zero_keys, pin_sdpa, pin_mpmath, pin_mass, pin_dominant_key, pin_lse_sdpa, pin_lse_zero_keys,
             pin_lse_shift, pin_pool, pin_select, pin_gather, pin_stats, pin_pivot_hand_cases,
-            pin_pivot_synthetic_phase_change, pin_decode_sdpa, pin_decode_closed_forms]
+            pin_pivot_synthetic_phase_change, pin_decode_sdpa, pin_decode_closed_forms,
+            pin_rvq_nearest_and_residual, pin_rvq_planted_codes, pin_rvq_tie_to_lowest_index]
