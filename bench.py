@@ -151,32 +151,44 @@ def measured_peaks():
 # --------------------------------------------------------------------------- #
 # CPU oracle (baseline / reference arm)
 # --------------------------------------------------------------------------- #
-def oracle_head_step(orc, lay, cfg, g: int) -> None:
-    """One KV head of the layer on the oracle: its window scores over all N
-    keys, its pooled top-k and K/V gather, and 1/Hkv of the hidden gather."""
-    G = cfg.G
-    q = lay.q[:, g * G:(g + 1) * G, :]
-    k = lay.k[:, g:g + 1, :]
-    A = orc.window_scores(q, k, G, 1, cfg.w, cfg.scale)
-    S = orc.rank_scores(A[0], cfg.N, cfg.w, cfg.pool)
-    idx = orc.select_topk(S, cfg.N, cfg.w, cfg.k_kv)
-    orc.gather_rows(lay.k[:, g, :], idx, nsrc=cfg.N)
-    orc.gather_rows(lay.v[:, g, :], idx, nsrc=cfg.N)
-    it = orc.select_topk(S, cfg.N, cfg.w, cfg.k_tsp)
-    part = it[g::cfg.Hkv]
-    orc.gather_rows(lay.x, part)
+class OracleLayerSteps:
+    """The float64 oracle over one layer, one KV head per step: that head's
+    window scores over all N keys, its pooled top-k and K/V gather; the
+    head's scores also go into the all-head (TSP) sum, and the step that adds
+    the last head ranks that sum (pooled top-k) and gathers the hidden
+    states.  Hkv consecutive steps are one whole layer of the method."""
+
+    def __init__(self, orc, lay, cfg):
+        self.orc, self.lay, self.cfg = orc, lay, cfg
+        self.T = np.zeros(cfg.N)
+        self.g = 0
+
+    def step(self) -> None:
+        orc, lay, cfg, g = self.orc, self.lay, self.cfg, self.g
+        G = cfg.G
+        A = orc.window_scores(lay.q[:, g * G:(g + 1) * G, :], lay.k[:, g:g + 1, :], G, 1, cfg.w, cfg.scale)[0]
+        S = orc.rank_scores(A, cfg.N, cfg.w, cfg.pool)
+        idx = orc.select_topk(S, cfg.N, cfg.w, cfg.k_kv)
+        orc.gather_rows(lay.k[:, g, :], idx, nsrc=cfg.N)
+        orc.gather_rows(lay.v[:, g, :], idx, nsrc=cfg.N)
+        self.T += A
+        if g == cfg.Hkv - 1:
+            pt = orc.rank_scores(self.T, cfg.N, cfg.w, cfg.pool)
+            orc.gather_rows(lay.x, orc.select_topk(pt, cfg.N, cfg.w, cfg.k_tsp))
+            self.T[:] = 0.0
+        self.g = (g + 1) % cfg.Hkv
 
 
-def cpu_baseline(orc, lay, cfg, heads: int = 8) -> dict:
+def cpu_baseline(orc, lay, cfg) -> dict:
+    """One whole layer on the oracle (Hkv head steps)."""
+    steps = OracleLayerSteps(orc, lay, cfg)
     t0 = time.perf_counter()
-    for g in range(heads):
-        oracle_head_step(orc, lay, cfg, g)
+    for _ in range(cfg.Hkv):
+        steps.step()
     dt = time.perf_counter() - t0
-    per_layer = dt * cfg.Hkv / heads
-    return {"value": cfg.N / per_layer, "unit": "tokens/s", "cores": orc.max_threads(), "kind": "oracle",
-            "sample": f"{heads} of {cfg.Hkv} KV heads of one N={cfg.N} layer (scores over all keys, pooled "
-                      f"top-k, K/V gather, 1/{cfg.Hkv} of the hidden gather each), scaled to a full layer; "
-                      f"{dt:.1f} s wall"}
+    return {"value": cfg.N / dt, "unit": "tokens/s", "cores": orc.max_threads(), "kind": "oracle",
+            "sample": f"one whole N={cfg.N} layer: {cfg.Hkv} KV heads (scores over all keys, pooled top-k, K/V "
+                      f"gather), the all-head sum, its pooled top-k and the hidden gather; {dt:.1f} s wall"}
 
 
 def run_reference(args, cfg, rank: int) -> None:
@@ -187,17 +199,19 @@ def run_reference(args, cfg, rank: int) -> None:
 
     orc = oracle.get()
     lay = workloads.make_layer(cfg)
-    for s in range(args.warmup):
-        oracle_head_step(orc, lay, cfg, s % cfg.Hkv)
+    steps = OracleLayerSteps(orc, lay, cfg)
+    for _ in range(args.warmup):
+        steps.step()
     t0 = time.perf_counter()
-    for s in range(args.steps):
-        oracle_head_step(orc, lay, cfg, s % cfg.Hkv)
-    dt = (time.perf_counter() - t0) / args.steps  # seconds per head-step
+    for _ in range(args.steps):
+        steps.step()
+    dt = (time.perf_counter() - t0) / args.steps  # seconds per step (one KV head)
     value = cfg.N / (dt * cfg.Hkv)
-    sample = (f"each step: one KV head of the N={cfg.N} layer (scores over all keys, pooled top-k, K/V gather, "
-              f"1/{cfg.Hkv} of the hidden gather); a layer = {cfg.Hkv} steps")
+    sample = (f"each step: one KV head of the N={cfg.N} layer (scores over all keys, pooled top-k, K/V gather) "
+              f"added into the all-head sum; every {cfg.Hkv}th step also ranks that sum (pooled top-k) and "
+              f"gathers the hidden states; a layer = {cfg.Hkv} steps")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3 * cfg.Hkv,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": workload_config(cfg),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": orc.max_threads(), "kind": "oracle",
@@ -210,23 +224,31 @@ def run_reference(args, cfg, rank: int) -> None:
 # the other configurations (per-layer time; the headline is the 128K layer)
 # --------------------------------------------------------------------------- #
 def other_bytes(cfg, total: int) -> int:
-    """Algorithmic HBM bytes of one layer of cfg (K once, Q_win, scores written
-    and read once, the K/V gather's rows in and out; the head-sum row when a
-    TSP budget is given)."""
+    """Algorithmic HBM bytes of one step of cfg.  A single sequence or a
+    ragged batch: K once, Q_win, the scores written and read once, the K(/V)
+    gather's rows in and out.  The 16-layer accumulation: per layer K once,
+    Q_win, the scores written and read once (statistics), C_global read and
+    written; then C_global read by the two selections and the K gather's rows
+    in and out."""
     B = cfg.batch
-    b = total * cfg.Hkv * cfg.d * 2 + B * cfg.w * cfg.H * cfg.d * 2 + 2 * cfg.Hkv * total * 4
     kv_rows = cfg.Hkv * B * min(cfg.k_kv, cfg.N)
-    b += (2 if cfg.with_v else 1) * 2 * kv_rows * cfg.d * 2
-    if cfg.k_tsp:
-        b += 2 * total * 4
-    return b
+    gather = (2 if cfg.with_v else 1) * 2 * kv_rows * cfg.d * 2
+    per_layer = total * cfg.Hkv * cfg.d * 2 + B * cfg.w * cfg.H * cfg.d * 2 + 2 * cfg.Hkv * total * 4
+    if cfg.layers > 1:
+        return cfg.layers * (per_layer + 2 * cfg.Hkv * total * 4) + 2 * cfg.Hkv * total * 4 + gather
+    return per_layer + gather
 
 
 def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
-    """Per-layer time of configuration cfg on one GPU: score (with the head-sum
-    row and C_global accumulation where cfg has them) -> per-KV-head top-k ->
-    K(/V) gather, plus the TSP top-k and the layer statistics for the
-    16-layer configuration; ragged batches through the varlen calls."""
+    """Time per layer of configuration cfg on one GPU.
+
+    A single sequence: score -> per-KV-head top-k -> K(/V) gather; a ragged
+    batch: the same through the varlen calls.  The 16-layer accumulation
+    (StructKV): one step is the whole job -- per layer the scores are added
+    into C_global and the layer statistics feed the pivot rule; after the
+    last layer C_global is ranked twice (the propagation set over the sum of
+    the KV-head rows, and the K set of every KV head) and the retained K rows
+    of that layer are gathered."""
     layers = ([workloads.make_layer(cfg, layer=l) for l in range(1, cfg.layers + 1)] if cfg.layers > 1
               else [workloads.make_layer(cfg)])
     lay0 = layers[0]
@@ -239,8 +261,8 @@ def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
     cu = torch.from_numpy(lay0.cu_seqlens).to(dev)
     kk = min(cfg.k_kv, cfg.N)
     scores = torch.empty((cfg.Hkv, total), dtype=torch.float32, device=dev)
-    tsp = torch.empty((1, total), dtype=torch.float32, device=dev) if cfg.k_tsp else None
-    accum = torch.zeros((cfg.Hkv, total), dtype=torch.float32, device=dev) if cfg.layers > 1 else None
+    multi = cfg.layers > 1
+    accum = torch.zeros((cfg.Hkv, total), dtype=torch.float32, device=dev) if multi else None
     err = torch.zeros(1, dtype=torch.int32, device=dev)
     p = kvc.score_params(cfg.H, cfg.Hkv, cfg.d, cfg.w)
     ws_s = torch.empty(kvc.score_workspace_size(p, B, total), dtype=torch.uint8, device=dev)
@@ -254,29 +276,37 @@ def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
         idx = torch.empty((cfg.Hkv, kk), dtype=torch.int32, device=dev)
         k_c = torch.empty((cfg.Hkv, kk, cfg.d), dtype=torch.bfloat16, device=dev)
     v_c = torch.empty_like(k_c) if cfg.with_v else None
-    idx_t = torch.empty((1, min(cfg.k_tsp, cfg.N)), dtype=torch.int32, device=dev) if cfg.k_tsp else None
-    stats = torch.empty((cfg.Hkv, 3), dtype=torch.float32, device=dev) if cfg.layers > 1 else None
+    idx_t = torch.empty((1, min(cfg.k_tsp, cfg.N)), dtype=torch.int32, device=dev) if multi else None
+    stats = torch.empty((cfg.Hkv, 3), dtype=torch.float32, device=dev) if multi else None
+    pivot = kvc.pivot_state(dev) if multi else None
 
-    def step(l: int, st):
-        q, k, v = qs[l], ks[l], vs[l]
+    def step(st):
         if B > 1:
-            kvc.kvc_score_varlen(q, k, cu, max_len, scores=scores, tsp=tsp, accum=accum, ws=ws_s, dev_err=err,
-                                 stream=st)
+            q, k, v = qs[0], ks[0], vs[0]
+            kvc.kvc_score_varlen(q, k, cu, max_len, scores=scores, ws=ws_s, dev_err=err, stream=st)
             kvc.kvc_select_topk_varlen(scores, cu, max_len, cfg.w, cfg.pool, cfg.k_kv, idx=idx, counts=counts,
                                        ws=ws_k, dev_err=err, stream=st)
             kvc.kvc_gather_kv_varlen(k, v, cu, idx, k_out=k_c, v_out=v_c, dev_err=err, stream=st)
             return
-        kvc.kvc_score(q, k, scores=scores, tsp=tsp, accum=accum, ws=ws_s, dev_err=err, stream=st)
-        if cfg.k_tsp:
-            kvc.kvc_select_topk(tsp, cfg.w, cfg.pool, cfg.k_tsp, idx=idx_t, ws=ws_t, stream=st)
-        kvc.kvc_select_topk(scores, cfg.w, cfg.pool, cfg.k_kv, idx=idx, ws=ws_k, stream=st)
-        kvc.kvc_gather_kv(k, v, idx, k_out=k_c, v_out=v_c, dev_err=err, stream=st)
-        if stats is not None:
+        if not multi:
+            kvc.kvc_score(qs[0], ks[0], scores=scores, ws=ws_s, dev_err=err, stream=st)
+            kvc.kvc_select_topk(scores, cfg.w, cfg.pool, cfg.k_kv, idx=idx, ws=ws_k, stream=st)
+            kvc.kvc_gather_kv(ks[0], vs[0], idx, k_out=k_c, v_out=v_c, dev_err=err, stream=st)
+            return
+        with torch.cuda.stream(st):
+            accum.zero_()
+            pivot.zero_()
+        for l in range(cfg.layers):
+            kvc.kvc_score(qs[l], ks[l], scores=scores, accum=accum, ws=ws_s, dev_err=err, stream=st)
             kvc.kvc_layer_stats(scores, float(cfg.w * cfg.G), out=stats, stream=st)
+            kvc.kvc_pivot_update(stats, l + 1, 0.05, 2, cfg.layers, pivot, dev_err=err, stream=st)
+        kvc.kvc_select_topk(accum, cfg.w, cfg.pool, cfg.k_tsp, row_group=cfg.Hkv, idx=idx_t, ws=ws_t, stream=st)
+        kvc.kvc_select_topk(accum, cfg.w, cfg.pool, cfg.k_kv, idx=idx, ws=ws_k, stream=st)
+        kvc.kvc_gather_kv(ks[-1], None, idx, k_out=k_c, dev_err=err, stream=st)
 
     st = torch.cuda.current_stream(dev)
     for i in range(args.warmup):
-        step(i % cfg.layers, st)
+        step(st)
     torch.cuda.synchronize(dev)
     if err.item() != 0:
         raise RuntimeError(f"device error word {err.item()}")
@@ -288,7 +318,7 @@ def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
         with torch.cuda.graph(graph):
             cap = torch.cuda.current_stream(dev)
             for i in range(nsteps):
-                step(i % cfg.layers, cap)
+                step(cap)
         torch.cuda.synchronize(dev)
     launches = kvc.launch_count() - launches0
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -300,7 +330,7 @@ def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
             graph.replay()
         else:
             for i in range(nsteps):
-                step(i % cfg.layers, st)
+                step(st)
         t1.record(st)
         torch.cuda.synchronize(dev)
     if graph is None:
@@ -311,14 +341,15 @@ def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
     alg = other_bytes(cfg, total)
     peak, peak_kind = measured_peaks()
     gbs = alg / (ms * 1e-3) / 1e9
-    line = {"metric": "context tokens scored+compressed/s per layer", "value": total / (ms * 1e-3),
+    line = {"metric": "context tokens scored+compressed/s per layer", "value": cfg.layers * total / (ms * 1e-3),
             "unit": "tokens/s", "n_gpus": 1, "steps": nsteps, "warmup": args.warmup, "ms_per_step": ms,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": {"workload": cfg.name, "tokens_per_layer": total, "batch": B, "layers_cycled": cfg.layers,
+            "ms_per_layer": ms / cfg.layers, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": cfg.name, "tokens_per_layer": total, "batch": B, "layers_per_step": cfg.layers,
                        "N": cfg.N, "H": cfg.H, "Hkv": cfg.Hkv, "d": cfg.d, "w": cfg.w, "pool": cfg.pool,
-                       "k_kv": cfg.k_kv, "k_tsp": cfg.k_tsp, "with_v": cfg.with_v},
-            "hbm": {"alg_bytes_per_layer": alg, "achieved_gbs": round(gbs, 1), "peak": peak,
+                       "k_kv": cfg.k_kv, "k_tsp": cfg.k_tsp, "with_v": cfg.with_v,
+                       "selection_source": "C_global after the last layer" if cfg.layers > 1 else "the layer's scores"},
+            "hbm": {"alg_bytes_per_step": alg, "achieved_gbs": round(gbs, 1), "peak": peak,
                     "peak_kind": peak_kind, "frac": round(gbs / peak, 4)},
             "gpu_launches": launches, "graph": graph is not None, "clocks": sampler.summary()}
     print(json.dumps(line), flush=True)
@@ -330,7 +361,8 @@ def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
 def main() -> None:
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 1000; 24 for --impl reference, three layers of head steps)")
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="kvc", choices=["kvc", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -344,6 +376,8 @@ def main() -> None:
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     args.e2e_steps = max(args.e2e_steps, 1)
+    if args.steps is None:
+        args.steps = 24 if args.impl == "reference" else 1000
 
     import workloads
 
@@ -474,21 +508,55 @@ def main() -> None:
     if plan.dev_err.item() != 0:
         raise RuntimeError(f"device error word {plan.dev_err.item()} after the timed region")
 
+    # ---- the one-read variant: normalisers given (kvc_score_lse) ---------------
+    # The window rows' log-sum-exp, as a causal prefill attention of the layer
+    # would return it, formed here once with torch (input preparation only,
+    # outside the timed region): lse[i, h] over keys <= N - w + i.
+    with torch.no_grad():
+        qf = q.float()
+        lse = torch.empty((cfg.w, cfg.H), dtype=torch.float32, device=dev)
+        for g in range(cfg.Hkv):
+            kg = k[:, g, :].float()
+            for hl in range(cfg.G):
+                h = g * cfg.G + hl
+                logit = (qf[:, h, :] @ kg.t()) * cfg.scale  # [w][N]
+                pos = torch.arange(cfg.N, device=dev)
+                lim = cfg.N - cfg.w + torch.arange(cfg.w, device=dev)
+                logit.masked_fill_(pos[None, :] > lim[:, None], float("-inf"))
+                lse[:, h] = torch.logsumexp(logit, dim=1)
+        del qf, logit
+    lse_scores = torch.empty_like(plan.scores)
+    for _ in range(3):
+        kvc.kvc_score_lse(q, k, lse, scores=lse_scores, ws=plan.ws_score, dev_err=plan.dev_err, stream=st)
+    torch.cuda.synchronize(dev)
+    l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_lse = 20
+    l0.record(st)
+    for _ in range(n_lse):
+        kvc.kvc_score_lse(q, k, lse, scores=lse_scores, ws=plan.ws_score, dev_err=plan.dev_err, stream=st)
+    l1.record(st)
+    torch.cuda.synchronize(dev)
+    ms_lse = l0.elapsed_time(l1) / n_lse
+    rel_lse = float(((lse_scores - plan.scores).abs() / plan.scores.abs().clamp_min(1e-30)).max())
+    del lse_scores
+
     # ---- end to end through the public API with host buffers ------------------
     hq, hk, hv, hx = (workloads.torch_bf16(a).pin_memory() for a in (lay.q, lay.k, lay.v, lay.x))
-    h_idx_kv = torch.empty(plan.idx_kv.shape, dtype=torch.int32).pin_memory()
-    h_idx_tsp = torch.empty(plan.idx_tsp.shape, dtype=torch.int32).pin_memory()
+    outs = [plan.idx_kv, plan.idx_tsp, plan.k_c, plan.v_c, plan.x_c]
+    h_outs = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
     h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hx))
-    d2h = h_idx_kv.numel() * 4 + h_idx_tsp.numel() * 4
+    d2h = sum(t.numel() * t.element_size() for t in h_outs)
 
     def e2e_step():
+        """Inputs in from pinned host memory, the layer, and every result of
+        the step back: both index sets, the compacted K/V and hidden states."""
         q.copy_(hq, non_blocking=True)
         k.copy_(hk, non_blocking=True)
         v.copy_(hv, non_blocking=True)
         x.copy_(hx, non_blocking=True)
         plan.run(q, k, v, x)
-        h_idx_kv.copy_(plan.idx_kv, non_blocking=True)
-        h_idx_tsp.copy_(plan.idx_tsp, non_blocking=True)
+        for h, t in zip(h_outs, outs):
+            h.copy_(t, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize(dev)
@@ -526,6 +594,11 @@ def main() -> None:
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
                          "traffic": load_traffic(dom)},
             "calls": breakdown,
+            "score_lse": {"ms": round(ms_lse, 5), "alg_bytes": alg["score"],
+                          "gbs": round(alg["score"] / (ms_lse * 1e-3) / 1e9, 1),
+                          "max_rel_diff_vs_two_pass": rel_lse,
+                          "note": "kvc_score_lse: the window rows' normalisers given (one read of K), "
+                                  "timed alone; not part of the headline step"},
             "ms_per_step_with_call_events": ms_step_events,
             "e2e": {"value": world * cfg.N / (ms_e2e * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": ms_e2e},

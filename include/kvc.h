@@ -61,7 +61,7 @@ typedef enum kvc_status {
 
 /* Device-side error bits (OR-ed into *dev_err when dev_err != NULL). */
 #define KVC_DEV_ERR_INDEX 1   /* gather index outside [-1, n) */
-#define KVC_DEV_ERR_SEQLENS 2 /* cu_seqlens not monotone, or a sequence shorter than w */
+#define KVC_DEV_ERR_SEQLENS 2 /* cu_seqlens malformed (not monotone, past the total) or a sequence shorter than w */
 #define KVC_DEV_ERR_TIMEOUT 4 /* an internal pipeline wait hit its bound (a bug): outputs invalid */
 #define KVC_DEV_ERR_ORDER 8   /* kvc_pivot_update: a layer folded in out of order */
 
@@ -186,7 +186,9 @@ kvc_status kvc_score_varlen(const uint16_t* q_win, int64_t q_stride_b, int64_t q
  *    launches nothing (8 KV heads x 128 window rows fit up to ~330K tokens).
  *  - First call on a device: it looks up (once per device, with that device
  *    current) the device address of the array.  Make the first call on each
- *    device before any stream capture.
+ *    device before any stream capture.  A device reset (cudaDeviceReset)
+ *    ends the context the address belongs to; the next call then looks it
+ *    up again, so after a reset, too, make one call before any capture.
  *  - Sharing: every call on a device uses the same array, which keeps the
  *    previous call's contents (nothing in it needs to start at zero: each
  *    call writes every entry it later reads).  Calls that may overlap on the

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <mutex>
 #include <string>
 
 #include "kvc.h"
@@ -24,6 +25,34 @@ inline void count_launch(int64_t n = 1) { g_launches.fetch_add(n, std::memory_or
 
 // Number of SMs of the current device (cached per device).
 int num_sms();
+
+// Unique id (cuCtxGetId) of the CUDA context current on the calling thread,
+// 0 if there is none yet or the driver cannot tell.  A device reset ends the
+// context and the next runtime call creates one with a new id, so state the
+// library sets up once per device (function attributes, the address of a
+// static device array) is keyed on it.
+uint64_t current_context_id();
+
+// Runs setup() unless it already succeeded on the current device in the
+// current context (one cache per kind of set-up).
+struct ContextCache {
+  std::mutex mu;
+  uint64_t ids[64] = {};
+};
+template <class F>
+kvc_status once_per_context(ContextCache& c, F&& setup) {
+  int dev = 0;
+  const cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(c.mu);
+  const bool slot = dev >= 0 && dev < 64;
+  const uint64_t id = current_context_id();
+  if (slot && id != 0 && c.ids[dev] == id) return KVC_OK;
+  const kvc_status s = setup();
+  if (s != KVC_OK) return s;
+  if (slot) c.ids[dev] = current_context_id();
+  return KVC_OK;
+}
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 

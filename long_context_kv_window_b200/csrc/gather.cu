@@ -29,7 +29,15 @@ gather_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int64
   const int bg = blockIdx.y;
   const int g = bg % Hkv;
   const int b = bg / Hkv;
-  const SeqSpan span = seq_span(cu, b, n);
+  SeqSpan span = seq_span(cu, b, n);
+  // a malformed cu_seqlens entry (negative start or length, or a sequence
+  // past the packed total) gathers nothing: its rows are zero and the
+  // sequence error bit is set instead of reading outside K / V
+  const bool bad_span = cu != nullptr && (span.start < 0 || span.len < 0 || span.start + span.len > n);
+  if (bad_span) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) set_dev_err(err, KVC_DEV_ERR_SEQLENS);
+    span.len = 0;
+  }
   const int32_t* irow = idx + (cu ? (int64_t)bg * kk : (int64_t)g * idx_row_stride);
   const int64_t items = kk * VPR;
   const int64_t out_base = (int64_t)bg * kk * VPR;
@@ -51,7 +59,7 @@ gather_kv_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int64
           const int64_t src = (span.start + j) * sn + (int64_t)g * sh + vec;
           kr[u] = __ldg(k + src);
           if (v) vr[u] = __ldg(v + src);
-        } else if (j != -1 && vec == 0) {
+        } else if (j != -1 && vec == 0 && !bad_span) {
           set_dev_err(err, KVC_DEV_ERR_INDEX);
         }
       }

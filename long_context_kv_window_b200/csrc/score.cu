@@ -840,19 +840,15 @@ size_t score_ws_bytes(const kvc_score_params* p, int B, int64_t total) {
 template <int D>
 kvc_status set_smem_attrs(size_t bytes) {
   if (bytes > 227 * 1024) return fail(KVC_ERR_UNSUPPORTED, "score kernel shared memory above 227 KB");
-  static std::mutex mu;
-  static uint64_t done = 0;  // bit per device ordinal (< 64)
-  int dev = 0;
-  KVC_CUDA_TRY(cudaGetDevice(&dev));
-  std::lock_guard<std::mutex> lk(mu);
-  if (dev < 64 && (done >> dev) & 1) return KVC_OK;
-  const void* fns[] = {(const void*)score_pass1_kernel<D, 2>, (const void*)score_pass1_kernel<D, 4>,
-                       (const void*)score_pass2_kernel<D, 2>, (const void*)score_pass2_kernel<D, 3>,
-                       (const void*)score_pass2_kernel<D, 4>};
-  for (const void* f : fns)
-    KVC_CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
-  if (dev < 64) done |= (uint64_t)1 << dev;
-  return KVC_OK;
+  static ContextCache cache;
+  return once_per_context(cache, [] {
+    const void* fns[] = {(const void*)score_pass1_kernel<D, 2>, (const void*)score_pass1_kernel<D, 4>,
+                         (const void*)score_pass2_kernel<D, 2>, (const void*)score_pass2_kernel<D, 3>,
+                         (const void*)score_pass2_kernel<D, 4>};
+    for (const void* f : fns)
+      KVC_CUDA_TRY(cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024));
+    return KVC_OK;
+  });
 }
 
 // The window rows' log-sum-exp when the caller has it (one sequence), else none.
@@ -1107,22 +1103,27 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[KVC_NOALLOC_SCR
 
 // Device address of g_noalloc_scratch on the current device.  Host code may
 // not use the symbol itself (it names a host-side shadow, not device
-// memory), so the address is looked up once per device with that device
-// current and cached.
+// memory), so the address is looked up with that device current and cached
+// per device, keyed on the CUDA context: after a device reset the module is
+// loaded again in a new context, the array may sit elsewhere, and the next
+// call looks the address up afresh.
 kvc_status noalloc_scratch_ptr(void** out) {
   static std::mutex mu;
-  static void* cache[64] = {};
+  static void* ptr[64] = {};
+  static uint64_t ctx[64] = {};
   int dev = 0;
   KVC_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return fail(KVC_ERR_UNSUPPORTED, "device ordinal >= 64");
   std::lock_guard<std::mutex> lk(mu);
-  if (cache[dev] == nullptr) {
+  const uint64_t id = current_context_id();
+  if (ptr[dev] == nullptr || id == 0 || ctx[dev] != id) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
-    cache[dev] = p;
+    ptr[dev] = p;
+    ctx[dev] = current_context_id();  // the lookup made the context current if it was not
   }
-  *out = cache[dev];
+  *out = ptr[dev];
   return KVC_OK;
 }
 

@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
   if (varlen) {
     start = a.cu[b];
     len = (int64_t)a.cu[b + 1] - start;
-    bad = (start < 0 || len < a.w);
+    bad = (start < 0 || len < a.w || start + len > a.n);  // a.n: packed total of the batch
     // a sequence longer than the max_seqlen the launch was sized for
     if (!bad && a.smem_vals && sel_segment(len - a.w, CS) > a.seg_cap) bad = true;
   }
@@ -982,18 +982,13 @@ bool sel_fits_smem(int64_t seg, int half) {
 // Launch: kCS-CTA clusters, one per (sequence, output row).
 kvc_status launch_select(SelArgs a, int out_rows, int batch, cudaStream_t st) {
   a.v_off = a.smem_vals ? (int)sel_stage_words(a.seg_cap, a.pool / 2) : 0;
-  static std::mutex mu;
-  static uint64_t done = 0;
-  int dev = 0;
-  KVC_CUDA_TRY(cudaGetDevice(&dev));
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    if (dev >= 64 || !((done >> dev) & 1)) {
-      KVC_CUDA_TRY(cudaFuncSetAttribute(select_kernel<kCS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        (int)kSelDynMax));
-      if (dev < 64) done |= (uint64_t)1 << dev;
-    }
-  }
+  static ContextCache cache;
+  kvc_status s = once_per_context(cache, [] {
+    KVC_CUDA_TRY(cudaFuncSetAttribute(select_kernel<kCS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kSelDynMax));
+    return KVC_OK;
+  });
+  if (s != KVC_OK) return s;
   Launch l(dim3(kCS, out_rows, batch), dim3(kThreads), kSelDynMax, st);
   l.cluster_x(kCS);
   KVC_CUDA_TRY(l.run(select_kernel<kCS>, a));

@@ -43,10 +43,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Upper bound of any single wait inside a kernel.  A healthy pipeline waits
-// microseconds; reaching the bound means a bug, and the kernel then records
-// an error and unwinds instead of spinning forever.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+// Upper bound of any single pipeline wait inside a kernel.  A healthy
+// pipeline waits microseconds; reaching the bound means a bug, and the kernel
+// then records an error and unwinds instead of spinning forever.  A test
+// build sets KVC_WAIT_LIMIT_NS to a few nanoseconds so that the unwinding
+// path runs; the waits of the unwinding itself (mbar_drain: copies and MMAs
+// already in flight must land before shared memory or TMEM is released)
+// always keep the full bound.
+#ifndef KVC_WAIT_LIMIT_NS
+#define KVC_WAIT_LIMIT_NS 2000000000ull
+#endif
+constexpr uint64_t kWaitLimitNs = KVC_WAIT_LIMIT_NS;
+constexpr uint64_t kDrainLimitNs = 2000000000ull;  // 2 s
 constexpr uint32_t kWaitLimitIters = 1u << 28;
 
 // Wait for phase `parity` of `bar`.  Returns false (and raises *abort) when
@@ -69,7 +77,7 @@ __device__ __forceinline__ bool mbar_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 0; it < kWaitLimitIters; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63) == 0 && global_timer_ns() - t0 > kWaitLimitNs) break;
+    if ((it & 63) == 0 && global_timer_ns() - t0 > kDrainLimitNs) break;
   }
   return false;
 }

@@ -84,29 +84,39 @@ def test_c4_full_ragged_batch():
 
 def test_c5_full_sixteen_layers():
     """Sixteen layers of N = 65536 with 40 query / 8 KV heads (160 window rows
-    per KV head), no pooling: C_global after all layers, and the last
-    layer's scores, K/V selection and statistics, for one KV head (the
-    oracle's cost grows with the heads it computes)."""
+    per KV head), no pooling, all eight KV heads.  C_global (the sum of the
+    per-layer scores, accumulated by the scoring call) is compared after the
+    last layer, and both of that layer's selections rank C_global: the
+    propagation set of 15 % of the tokens over the sum of the eight rows
+    (9830 kept) and the 4096-per-KV-head K set.  The last layer's own scores
+    and statistics are compared too."""
     cfg = workloads.C5
-    N, G, w, g = cfg.N, cfg.G, cfg.w, 3
+    N, G, w, Hkv = cfg.N, cfg.G, cfg.w, cfg.Hkv
     orc = oracle.get()
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
-    accum = torch.zeros((cfg.Hkv, N), dtype=torch.float32, device="cuda")
-    tsp = torch.empty((1, N), dtype=torch.float32, device="cuda")
-    ref_c = np.zeros(N)
+    accum = torch.zeros((Hkv, N), dtype=torch.float32, device="cuda")
+    ref_c = np.zeros((Hkv, N))
     A = None
     for layer in range(1, cfg.layers + 1):
         lay = workloads.make_layer(cfg, layer=layer)
-        scores = kvc.kvc_score(dev_bf16(lay.q), dev_bf16(lay.k), tsp=tsp, accum=accum, dev_err=err)
-        A = orc.window_scores(lay.q[:, g * G:(g + 1) * G, :], lay.k[:, g:g + 1, :], G, 1, w, cfg.scale)[0]
+        scores = kvc.kvc_score(dev_bf16(lay.q), dev_bf16(lay.k), accum=accum, dev_err=err)
+        A = orc.window_scores(lay.q, lay.k, cfg.H, Hkv, w, cfg.scale)
         ref_c += A
-    idx = kvc.kvc_select_topk(scores, w, cfg.pool, cfg.k_kv)
+    idx_prop = kvc.kvc_select_topk(accum, w, cfg.pool, cfg.k_tsp, row_group=Hkv)
+    idx_kv = kvc.kvc_select_topk(accum, w, cfg.pool, cfg.k_kv)
     stats = kvc.kvc_layer_stats(scores, float(w * G))
     torch.cuda.synchronize()
     assert err.item() == 0
-    parity.assert_scores_close(accum[g].cpu().numpy(), ref_c, what="c5 C_global")
-    parity.assert_scores_close(scores[g].cpu().numpy(), A, what="c5 last-layer scores")
-    S = orc.rank_scores(A, N, w, cfg.pool)
-    parity.assert_selection_matches(idx[g].cpu().numpy(), orc.select_topk(S, N, w, cfg.k_kv), S, N, w, cfg.k_kv,
-                                    what="c5 last-layer selection")
-    parity.assert_scores_close(stats[g].cpu().numpy(), orc.layer_stats(A, w * G), what="c5 last-layer stats")
+    parity.assert_scores_close(accum.cpu().numpy(), ref_c, what="c5 C_global")
+    parity.assert_scores_close(scores.cpu().numpy(), A, what="c5 last-layer scores")
+    T = orc.sum_rows(ref_c)
+    S_prop = orc.rank_scores(T, N, w, cfg.pool)
+    parity.assert_selection_matches(idx_prop[0].cpu().numpy(), orc.select_topk(S_prop, N, w, cfg.k_tsp), S_prop,
+                                    N, w, cfg.k_tsp, what="c5 propagation set (C_global, all heads)")
+    ik = idx_kv.cpu().numpy()
+    st = stats.cpu().numpy()
+    for g in range(Hkv):
+        S = orc.rank_scores(ref_c[g], N, w, cfg.pool)
+        parity.assert_selection_matches(ik[g], orc.select_topk(S, N, w, cfg.k_kv), S, N, w, cfg.k_kv,
+                                        what=f"c5 K set of head {g} (C_global)")
+        parity.assert_scores_close(st[g], orc.layer_stats(A[g], w * G), what=f"c5 last-layer stats head {g}")

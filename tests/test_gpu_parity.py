@@ -327,6 +327,45 @@ def test_varlen_bad_seqlens_flagged():
     assert counts[1].item() == 0 and torch.all(idx[1] == -1)
 
 
+def test_varlen_seqlens_past_the_total_flagged():
+    """A cu_seqlens whose last sequence ends past the packed total: the
+    selection and the K/V gather report KVC_DEV_ERR_SEQLENS and pad that
+    sequence (-1 indices, zero rows) instead of reading past the buffers.  The
+    buffers carry slack past the total, so that even an unguarded read would
+    stay inside them."""
+    rng = np.random.default_rng(12)
+    lens = np.array([300, 400])
+    total, slack = int(lens.sum()), 256
+    scores = torch.from_numpy(rng.random((2, total + slack)).astype(np.float32)).cuda()[:, :total]
+    cu_np = np.array([0, 300, total + 100], dtype=np.int32)  # sequence 1 runs 100 tokens past the total
+    cu = torch.from_numpy(cu_np).cuda()
+    err = _err_word()
+    idx, counts = kvc.kvc_select_topk_varlen(scores, cu, 800, 16, 3, 64, dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() & kvc.KVC_DEV_ERR_SEQLENS
+    assert counts.cpu().tolist() == [64, 0]
+    assert torch.all(idx[1] == -1)
+    orc = oracle.get()
+    S0 = scores[:, :300].cpu().numpy().astype(np.float64)
+    for r in range(2):
+        Sp = orc.rank_scores(S0[r], 300, 16, 3)
+        parity.assert_selection_matches(idx[0, r].cpu().numpy(), orc.select_topk(Sp, 300, 16, 64), Sp, 300, 16,
+                                        64)
+
+    kbig = torch.from_numpy(rng.standard_normal((total + slack, 2, 64)).astype(np.float32)).to(torch.bfloat16)
+    k = kbig.cuda()[:total]
+    gidx = torch.from_numpy(rng.integers(0, 300, size=(2, 2, 16)).astype(np.int32)).cuda()
+    err = _err_word()
+    ko, _ = kvc.kvc_gather_kv_varlen(k, None, cu, gidx, dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == kvc.KVC_DEV_ERR_SEQLENS  # the sequence bit only: no index is out of its range
+    KO, K = host_bits(ko), host_bits(k)
+    G = gidx.cpu().numpy()
+    for g in range(2):
+        assert np.array_equal(KO[0, g], K[G[0, g], g, :])
+    assert not KO[1].any()
+
+
 # --------------------------------------------------------------------------- #
 # statistics
 # --------------------------------------------------------------------------- #
