@@ -264,9 +264,18 @@ __device__ __forceinline__ void issue_mmas(const ScoreArgs& a, Barriers* bars, u
                                            uint8_t* kst, uint8_t* ones, uint8_t* qb, int ntiles) {
   constexpr int kChunks = D / 64;
   const uint32_t idesc = kRowsOnM ? tc::idesc_bf16_f32(128, kTile) : tc::idesc_bf16_f32(128, a.Rn);
-  const uint32_t qbase = tc::smem_u32(qs), kbase = tc::smem_u32(kst);
+  // Shared-memory descriptors are formed once: an MMA K-step or a stage only
+  // moves the start-address field (bits [0,14): address >> 4; shared memory
+  // is below 256 KB, so adding offset >> 4 never carries out of the field).
+  // The issuing thread shares its sub-partition with busy epilogue warps, so
+  // its instruction count per tile is kept small.
+  const uint64_t q_desc0 = tc::desc_k_sw128(tc::smem_u32(qs));
+  const uint64_t k_desc0 = tc::desc_k_sw128(tc::smem_u32(kst));
   const uint64_t ones_desc = tc::desc_k_sw32(tc::smem_u32(ones));
   const uint64_t qb_desc = tc::desc_k_sw32(tc::smem_u32(qb));
+  const uint32_t q_chunk = (uint32_t)a.Rq * 8u;                          // (Rq * 128 B) >> 4
+  constexpr uint32_t kChunk = (uint32_t)(kTile * 128) >> 4;                 // one 64-column block of a K tile
+  constexpr uint32_t kStage = (uint32_t)Smem<D>::kStageBytes >> 4;
   int issued = 0;
   const bool go = kRowsOnM || tc::mbar_wait(&bars->bias_ready, 0, &bars->abort);
   for (int t = 0; go && t < ntiles; ++t) {
@@ -275,20 +284,21 @@ __device__ __forceinline__ void issue_mmas(const ScoreArgs& a, Barriers* bars, u
     if (!tc::mbar_wait(&bars->full[s], (t / a.stages) & 1, &bars->abort)) break;
     if (ub > 0 && !tc::mbar_wait(&bars->tempty[buf], (ub - 1) & 1, &bars->abort)) break;
     tc::tc_fence_after();
-    const uint32_t kst_s = kbase + (uint32_t)(s * Smem<D>::kStageBytes);
+    const uint64_t kd = k_desc0 + (uint64_t)((uint32_t)s * kStage);
     const int nblk = kRowsOnM ? a.nb1 : 1;
     for (int mb = 0; mb < nblk; ++mb) {
       const uint32_t d = tmem + (uint32_t)(buf * a.acc_stride + mb * kTile);
+      const uint64_t qd = q_desc0 + (uint64_t)((uint32_t)mb * kChunk);  // row block mb of Q (pass 1)
 #pragma unroll
       for (int c = 0; c < kChunks; ++c)
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-          const uint32_t qa = qbase + (uint32_t)(c * a.Rq * 128 + mb * kTile * 128 + ks * 32);
-          const uint32_t ka = kst_s + (uint32_t)(c * kTile * 128 + ks * 32);
+          const uint64_t qo = qd + (uint64_t)((uint32_t)c * q_chunk + (uint32_t)(ks * 2));
+          const uint64_t ko = kd + (uint64_t)((uint32_t)c * kChunk + (uint32_t)(ks * 2));
           if (kRowsOnM)
-            tc::mma_bf16(d, tc::desc_k_sw128(qa), tc::desc_k_sw128(ka), idesc, (c | ks) != 0);
+            tc::mma_bf16(d, qo, ko, idesc, (c | ks) != 0);
           else
-            tc::mma_bf16(d, tc::desc_k_sw128(ka), tc::desc_k_sw128(qa), idesc, (c | ks) != 0);
+            tc::mma_bf16(d, ko, qo, idesc, (c | ks) != 0);
         }
       // pass 2: + (h1 + h2 + h3) = -bias/c on every (key, row)
       if (!kRowsOnM) tc::mma_bf16(d, ones_desc, qb_desc, idesc, 1u);
@@ -351,6 +361,10 @@ __device__ __forceinline__ void walk_columns(uint32_t base, int ncols, Proc&& pr
   uint32_t xa[kCols], xb[kCols];
   const int ng = (ncols + kCols - 1) / kCols;
   __syncwarp();
+  if (ng <= 0) {  // nothing to read (a warp whose rows are all padding): release at once
+    release();
+    return;
+  }
   tmem_ld_cols(base, xa, min(kCols, ncols));
   for (int gi = 0; gi < ng; gi += 2) {
     KVC_TMEM_WAIT_LD32(xa);
@@ -372,14 +386,33 @@ __device__ __forceinline__ void walk_columns(uint32_t base, int ncols, Proc&& pr
   }
 }
 
-// sum_e 2^(x[e]*c + off) over kCols values, 8 independent accumulators
+// Two consecutive accumulator values as a packed pair.
+__device__ __forceinline__ float2 pair(const uint32_t (&x)[kCols], int e) {
+  return make_float2(__uint_as_float(x[e]), __uint_as_float(x[e + 1]));
+}
+
+// acc += 2^(x[e]*c + off) over kCols values: per pair of columns one packed
+// fma for the arguments, two ex2 and one packed add (four packed
+// accumulators, i.e. eight independent sums).
+__device__ __forceinline__ void acc_ex2(const uint32_t (&x)[kCols], float2 c2, float2 off2, float2 (&acc)[4]) {
+#pragma unroll
+  for (int e = 0; e < kCols; e += 2) {
+    const float2 t = tc::fma2(pair(x, e), c2, off2);
+    acc[(e >> 1) & 3] = tc::add2(acc[(e >> 1) & 3], make_float2(tc::ex2_approx(t.x), tc::ex2_approx(t.y)));
+  }
+}
+__device__ __forceinline__ float sum4(const float2 (&acc)[4]) {
+  const float2 u = tc::add2(tc::add2(acc[0], acc[1]), tc::add2(acc[2], acc[3]));
+  return u.x + u.y;
+}
+
+// sum_e 2^(x[e]*c + off) over kCols values
 __device__ __forceinline__ float sum_ex2(const uint32_t (&x)[kCols], float c, float off) {
-  float s8[8];
+  float2 acc[4];
 #pragma unroll
-  for (int u = 0; u < 8; ++u) s8[u] = 0.f;
-#pragma unroll
-  for (int e = 0; e < kCols; ++e) s8[e & 7] += tc::ex2_approx(fmaf(__uint_as_float(x[e]), c, off));
-  return ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+  for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
+  acc_ex2(x, make_float2(c, c), make_float2(off, off), acc);
+  return sum4(acc);
 }
 
 __device__ __forceinline__ float max_cols(const uint32_t (&x)[kCols]) {
@@ -460,16 +493,28 @@ score_pass1_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
     float m_run[2] = {-INFINITY, -INFINITY};
     double l_run[2] = {0.0, 0.0};
     const int64_t first_window_key = wk.len - a.w;  // earliest window row sees keys <= this
+    // row blocks in which this warp owns window rows: a warp whose 32 rows of a
+    // block are all padding skips that block's columns
+    const int blocks_w = std::min(a.nb1, std::max(0, (a.R - 32 * q + kTile - 1) / kTile));
     for (int t = grp; t < ntiles; t += NB) {
       const int buf = t % a.nbuf;
       if (!wait_filled(a, bars, t)) break;
       tc::tc_fence_after();
       const int64_t j0 = k0 + (int64_t)t * kTile;  // first key of the tile (sequence-local)
       const bool masked = (j0 + kTile - 1 > first_window_key);
+      // every lane of a walked block is a window row and no key is masked
+      const bool fast = !masked && (a.R % 32) == 0;
       const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * a.acc_stride);
       walk_columns<true>(
-          base, a.nb1 * kTile,
+          base, blocks_w * kTile,
           [&](int gi, uint32_t(&x)[kCols]) {
+            if (fast) {  // warp-uniform: the common case
+              if (gi < kPerBlock)
+                pass1_group(x, a.c, m_run[0], l_run[0]);
+              else
+                pass1_group(x, a.c, m_run[1], l_run[1]);
+              return;
+            }
             const int mb = gi / kPerBlock;
             const int r = mb * kTile + rl;
             if (r >= a.R) return;
@@ -713,10 +758,16 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
       const int64_t lim = j - first_window_key;
       const int rmin = lim <= 0 ? 0 : (int)std::min<int64_t>(lim * a.G, a.Rn);
       const uint32_t base = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * a.acc_stride);
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      float2 acc[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = make_float2(0.f, 0.f);
       walk_columns<false>(
           base, a.Rn,
           [&](int gi, uint32_t(&x)[kCols]) {
+            if (!masked && (a.Rn % kCols) == 0) {  // warp-uniform: the common case
+              acc_ex2(x, make_float2(a.c, a.c), make_float2(0.f, 0.f), acc);
+              return;
+            }
             const int col0 = gi * kCols;
             const int ncol = min(kCols, a.Rn - col0);
             // columns past ncol (not loaded) and, on tiles reaching into the
@@ -733,8 +784,7 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
               for (int e = 0; e < kCols; ++e)
                 if (col0 + e < rmin) x[e] = __float_as_uint(-INFINITY);
             }
-#pragma unroll
-            for (int e = 0; e < kCols; ++e) s4[e & 3] += tc::ex2_approx(__uint_as_float(x[e]) * a.c);
+            acc_ex2(x, make_float2(a.c, a.c), make_float2(0.f, 0.f), acc);
           },
           [&]() {
             tc::tc_fence_before();
@@ -742,7 +792,7 @@ score_pass2_kernel(const __grid_constant__ CUtensorMap kmap, const ScoreArgs a) 
             if (lane == 0) tc::mbar_arrive(&bars->tempty[buf]);
           });
       if (j < k1) {
-        const float v = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        const float v = sum4(acc);
         const int64_t o = (int64_t)g * a.total + wk.start + j;
         a.scores[o] = v;
         if (a.accum) a.accum[o] += v;

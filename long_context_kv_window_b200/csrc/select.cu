@@ -38,6 +38,8 @@ namespace {
 constexpr int kThreads = 1024;
 constexpr int kWarps = kThreads / 32;
 constexpr int kCS = 8;          // CTAs per ranking row (portable cluster size)
+constexpr int kCSWide = 16;     // CTAs for a lone long row (non-portable cluster size)
+constexpr int64_t kWideMinKeys = 32768;  // shortest row that gets the wide cluster
 constexpr int kMaxHalf = 32;    // pool_kernel <= 65
 constexpr int kBins = 2048;     // radix bins of the first two passes
 constexpr int kWinBins = 1024;  // bins of the windowed histogram
@@ -196,8 +198,8 @@ struct SelShared {
   uint32_t sample[kSampleTotal];   // this CTA's sampled keys
   uint32_t sall[kSampleTotal];     // the cluster's samples (rank order), then ...
   uint32_t ssort[kSampleTotal];    // ... sorted, largest first
-  uint32_t soff[kCS + 1];      // sample slots per rank
-  uint32_t cand_off[kCS + 1];  // candidate slots per rank, total last
+  uint32_t soff[kCSWide + 1];      // sample slots per rank
+  uint32_t cand_off[kCSWide + 1];  // candidate slots per rank, total last
   uint32_t cand_n;                 // candidate slots this CTA has taken
   uint32_t above;                  // this CTA's keys in bins above the threshold bin
   uint32_t T, need_eq;             // threshold resolved from the candidate list
@@ -979,19 +981,53 @@ bool sel_fits_smem(int64_t seg, int half) {
   return (sel_v_words(seg) + sel_stage_words(seg, half)) * sizeof(float) <= kSelDynMax;
 }
 
-// Launch: kCS-CTA clusters, one per (sequence, output row).
-kvc_status launch_select(SelArgs a, int out_rows, int batch, cudaStream_t st) {
-  a.v_off = a.smem_vals ? (int)sel_stage_words(a.seg_cap, a.pool / 2) : 0;
+// Whether this device can place a 16-CTA selection cluster (looked up once per
+// context; the kernel attributes are set on the way).
+bool wide_clusters_available() {
   static ContextCache cache;
-  kvc_status s = once_per_context(cache, [] {
+  static bool ok[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const kvc_status s = once_per_context(cache, [dev] {
+    ok[dev] = false;
     KVC_CUDA_TRY(cudaFuncSetAttribute(select_kernel<kCS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kSelDynMax));
+    KVC_CUDA_TRY(cudaFuncSetAttribute(select_kernel<kCSWide>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kSelDynMax));
+    if (cudaFuncSetAttribute(select_kernel<kCSWide>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return KVC_OK;
+    }
+    Launch l(dim3(kCSWide, 1, 1), dim3(kThreads), kSelDynMax, nullptr);
+    l.cluster_x(kCSWide);
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, select_kernel<kCSWide>, &l.cfg) == cudaSuccess)
+      ok[dev] = clusters > 0;
+    else
+      cudaGetLastError();
     return KVC_OK;
   });
-  if (s != KVC_OK) return s;
-  Launch l(dim3(kCS, out_rows, batch), dim3(kThreads), kSelDynMax, st);
-  l.cluster_x(kCS);
-  KVC_CUDA_TRY(l.run(select_kernel<kCS>, a));
+  return s == KVC_OK && ok[dev];
+}
+
+// CTAs per ranking row: a lone long row (the all-head TSP row of a long
+// sequence) is spread over a 16-CTA cluster when the device can place one --
+// half the keys per CTA, and it runs alone -- every other launch uses 8.
+int select_cluster_size(int rows_total, int64_t L) {
+  return (rows_total == 1 && L >= kWideMinKeys && wide_clusters_available()) ? kCSWide : kCS;
+}
+
+// Launch: cs-CTA clusters, one per (sequence, output row).
+kvc_status launch_select(SelArgs a, int out_rows, int batch, int cs, cudaStream_t st) {
+  a.v_off = a.smem_vals ? (int)sel_stage_words(a.seg_cap, a.pool / 2) : 0;
+  wide_clusters_available();  // sets the kernel attributes once per context
+  Launch l(dim3(cs, out_rows, batch), dim3(kThreads), kSelDynMax, st);
+  l.cluster_x(cs);
+  if (cs == kCSWide)
+    KVC_CUDA_TRY(l.run(select_kernel<kCSWide>, a));
+  else
+    KVC_CUDA_TRY(l.run(select_kernel<kCS>, a));
   count_launch();
   return KVC_OK;
 }
@@ -1050,7 +1086,8 @@ extern "C" kvc_status kvc_select_topk(const float* scores, int32_t rows, int64_t
   a.counts = nullptr;
   a.out_rows = out_rows;
   a.err = nullptr;
-  const int64_t seg = sel_segment(n - window, kCS);
+  const int cs = select_cluster_size(out_rows, n - window);
+  const int64_t seg = sel_segment(n - window, cs);
   a.smem_vals = sel_fits_smem(seg, pool_kernel / 2);
   a.seg_cap = seg;
   if (pooled) {
@@ -1068,7 +1105,7 @@ extern "C" kvc_status kvc_select_topk(const float* scores, int32_t rows, int64_t
     a.vals_stride = n;
     a.vals_packed = true;
   }
-  return launch_select(a, out_rows, 1, (cudaStream_t)stream);
+  return launch_select(a, out_rows, 1, cs, (cudaStream_t)stream);
 }
 
 extern "C" kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, int64_t row_stride,
@@ -1111,7 +1148,7 @@ extern "C" kvc_status kvc_select_topk_varlen(const float* scores, int32_t rows, 
   a.smem_vals = sel_fits_smem(seg_max, pool_kernel / 2);
   a.seg_cap = seg_max;
   if (!a.smem_vals) a.vals_g = static_cast<float*>(ws);
-  return launch_select(a, out_rows, batch, (cudaStream_t)stream);
+  return launch_select(a, out_rows, batch, kCS, (cudaStream_t)stream);
 }
 
 extern "C" kvc_status kvc_stats_workspace_size(int32_t rows, int64_t n, size_t* bytes) {

@@ -126,6 +126,45 @@ def test_select_window_miss_falls_back_to_plain_radix():
         assert np.array_equal(idx[r], ref), f"row {r}"
 
 
+@pytest.mark.parametrize("case", ["levels50", "levels3", "levels1", "lognormal_pool7", "window_miss",
+                                  "uniform_pool7_n65536"])
+def test_select_single_long_row_wide_cluster(case):
+    """A lone ranking row of 32K positions or more (the all-head TSP row) is
+    spread over a 16-CTA cluster where the device can place one.  It must
+    rank like the oracle and exactly like the 8-CTA launch of the same row
+    (two identical rows in one call take the 8-CTA path)."""
+    rng = np.random.default_rng(abs(hash(case)) % 2**32)
+    n, w, k, pool = 131072, 32, 26214, 1
+    if case.startswith("levels"):
+        S = rng.integers(0, int(case[6:]), size=n).astype(np.float32) * 0.25
+    elif case == "lognormal_pool7":
+        S, pool = np.exp(3.0 * rng.standard_normal(n)).astype(np.float32), 7
+    elif case == "window_miss":
+        # the evenly spaced positions each CTA samples hold large values
+        L, cs = n - w, 16
+        seg = ((L + cs - 1) // cs + 3) & ~3
+        S = rng.random(n).astype(np.float32)
+        for c in range(cs):
+            s0 = min(c * seg, L)
+            nseg = min(seg, L - s0)
+            nsc = min(128 // cs, nseg)
+            S[s0 + ((2 * np.arange(nsc) + 1) * nseg) // (2 * nsc)] = 100.0 + rng.random(nsc).astype(np.float32)
+    else:
+        n, k, pool = 65536, 9830, 7
+        S = rng.random(n).astype(np.float32)
+    one = torch.from_numpy(S).view(1, n).cuda()
+    idx1 = kvc.kvc_select_topk(one, w, pool, k).cpu().numpy()[0]
+    idx8 = kvc.kvc_select_topk(one.expand(2, n).contiguous(), w, pool, k).cpu().numpy()
+    assert np.array_equal(idx1, idx8[0]) and np.array_equal(idx1, idx8[1]), "16-CTA and 8-CTA launches differ"
+    orc = oracle.get()
+    Sp = orc.rank_scores(S.astype(np.float64), n, w, pool)
+    ref = orc.select_topk(Sp, n, w, k)
+    if pool == 1:
+        assert np.array_equal(idx1, ref)
+    else:
+        parity.assert_selection_matches(idx1, ref, Sp, n, w, k)
+
+
 @pytest.mark.parametrize("n,pool", [(420000, 7), (420000, 1)])
 def test_select_long_row_global_memory_mode(n, pool):
     """Rows too long for the per-CTA shared-memory segments: pooled values
