@@ -140,6 +140,16 @@ def load_traffic(kernel: str):
         return None
 
 
+def tensor_peak_tf32():
+    """Dense tf32 tensor peak: the measured bf16 GEMM peak times the nominal
+    tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s)."""
+    try:
+        mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return round(float(mp["bf16_tflops"]) * 1.1 / 2.25, 1), "measured bf16 x nominal tf32/bf16"
+    except Exception:
+        return round(1590.0 * 1.1 / 2.25, 1), "fallback bf16 x nominal tf32/bf16"
+
+
 def measured_peaks():
     try:
         mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -356,6 +366,61 @@ def run_other(args, cfg, torch, kvc, workloads, dev) -> None:
 
 
 # --------------------------------------------------------------------------- #
+# one layer split by KV head over the ranks
+# --------------------------------------------------------------------------- #
+def run_split(args, cfg, world, rank, local, torch, dist, kvc, shard, workloads) -> None:
+    """The 128K layer split by KV head over `world` ranks (strong scaling):
+    every rank scores, selects and gathers the K/V of its KV heads; the
+    partial all-head rows are summed with an NCCL all-reduce; every rank then
+    ranks the summed row and gathers its column slice of the hidden states.
+    Steps are launched one by one (no graph); the time is the max over ranks."""
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    lay = workloads.make_layer(cfg)  # the same layer on every rank; each reads its slices
+    q, k, v, x = (workloads.torch_bf16(a, dev) for a in (lay.q, lay.k, lay.v, lay.x))
+    part = shard.HeadSplitLayer(rank, world, cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden,
+                                dev, pool_kernel=cfg.pool)
+    reduce_sum = (lambda t: dist.all_reduce(t, op=dist.ReduceOp.SUM)) if world > 1 else None
+    st = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        part.run(q, k, v, x, reduce_sum=reduce_sum)
+    torch.cuda.synchronize(dev)
+    if part.dev_err.item() != 0:
+        raise RuntimeError(f"device error word {part.dev_err.item()}")
+    launches0 = kvc.launch_count()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    with sampler:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        t0.record(st)
+        for _ in range(args.steps):
+            part.run(q, k, v, x, reduce_sum=reduce_sum)
+        t1.record(st)
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+    launches = kvc.launch_count() - launches0
+    ms = shard.max_over_ranks(t0.elapsed_time(t1), dist, dev) / args.steps
+    if rank == 0:
+        conf = workload_config(cfg)
+        conf["parallelism"] = f"one layer split by KV head over {world} rank(s), the TSP row all-reduced"
+        line = {"metric": METRIC, "value": cfg.N / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": conf,
+                "hbm_gbs": round(layer_bytes(cfg) / (ms * 1e-3) / 1e9, 1), "gpu_launches": launches,
+                "graph": False, "clocks": sampler.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# --------------------------------------------------------------------------- #
 # CUDA arm
 # --------------------------------------------------------------------------- #
 def main() -> None:
@@ -371,6 +436,9 @@ def main() -> None:
                     help="launch the timed steps one by one instead of replaying a CUDA graph")
     ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5"],
                     help="c3 (the 128K layer) is the headline; the others print their per-layer time")
+    ap.add_argument("--split", default="replicas", choices=["replicas", "heads"],
+                    help="N > 1: replicas (each rank its own layer, weak scaling; default) or heads (one layer "
+                         "split by KV head over the ranks, the TSP row all-reduced; strong scaling)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="same layer structure at another N (small cases for profiling)")
     args = ap.parse_args()
@@ -406,6 +474,10 @@ def main() -> None:
 
     import long_context_kv_window_b200 as kvc
     from long_context_kv_window_b200 import shard
+
+    if args.split == "heads":
+        run_split(args, cfg, world, rank, local, torch, dist, kvc, shard, workloads)
+        return
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -540,6 +612,58 @@ def main() -> None:
     rel_lse = float(((lse_scores - plan.scores).abs() / plan.scores.abs().clamp_min(1e-30)).max())
     del lse_scores
 
+    # ---- decode over the compacted cache (the consumer of the K/V retention) ----
+    # One decode query per head over the retained entries.  The cache (K_c +
+    # V_c, 53.7 MB) fits in L2, so the timed calls cycle through four copies
+    # (215 MB) and read from HBM.
+    gq = torch.Generator(device=dev)
+    gq.manual_seed(17)
+    q_dec = torch.randn(cfg.H, cfg.d, device=dev, generator=gq).to(torch.bfloat16)
+    caches = [(plan.k_c, plan.v_c)] + [(plan.k_c.clone(), plan.v_c.clone()) for _ in range(3)]
+    dec_out = torch.empty((cfg.H, cfg.d), dtype=torch.float32, device=dev)
+    ws_dec = torch.empty(kvc.decode_workspace_size(cfg.H, cfg.Hkv, cfg.d, cfg.k_kv), dtype=torch.uint8, device=dev)
+    for i in range(4):
+        kvc.kvc_decode_attention(q_dec, *caches[i], out=dec_out, ws=ws_dec, dev_err=plan.dev_err, stream=st)
+    torch.cuda.synchronize(dev)
+    n_dec = 40
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0.record(st)
+    for i in range(n_dec):
+        kvc.kvc_decode_attention(q_dec, *caches[i % 4], out=dec_out, ws=ws_dec, dev_err=plan.dev_err, stream=st)
+    d1.record(st)
+    torch.cuda.synchronize(dev)
+    ms_dec = d0.elapsed_time(d1) / n_dec
+    dec_bytes = 2 * cfg.Hkv * cfg.k_kv * cfg.d * 2 + cfg.H * cfg.d * (2 + 4)
+    del caches
+
+    # ---- residual VQ encode of the compacted cache (K and V rows) ------------
+    # Four stages of 256 codewords (random stand-ins for trained codebooks);
+    # the scores are a tf32 tensor-core contraction: 2 * rows * M * d FLOP per
+    # stage.
+    rvq_S, rvq_M = 4, 256
+    cbk = torch.from_numpy(workloads.make_codebooks(rvq_S, rvq_M, cfg.d, seed=9)).to(dev)
+    cbv = torch.from_numpy(workloads.make_codebooks(rvq_S, rvq_M, cfg.d, seed=10)).to(dev)
+    rows_k, rows_v = plan.k_c.view(-1, cfg.d), plan.v_c.view(-1, cfg.d)
+    codes_k = torch.empty((rows_k.shape[0], rvq_S), dtype=torch.int32, device=dev)
+    codes_v = torch.empty_like(codes_k)
+
+    def rvq_both():
+        kvc.kvc_rvq_encode(rows_k, cbk, codes=codes_k, dev_err=plan.dev_err, stream=st)
+        kvc.kvc_rvq_encode(rows_v, cbv, codes=codes_v, dev_err=plan.dev_err, stream=st)
+    rvq_both()
+    torch.cuda.synchronize(dev)
+    n_rvq = 5
+    r0, r1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    r0.record(st)
+    for _ in range(n_rvq):
+        rvq_both()
+    r1.record(st)
+    torch.cuda.synchronize(dev)
+    ms_rvq = r0.elapsed_time(r1) / n_rvq
+    rvq_rows = rows_k.shape[0] + rows_v.shape[0]
+    rvq_flop = 2 * rvq_rows * rvq_M * cfg.d * rvq_S
+    tf32_peak, tf32_kind = tensor_peak_tf32()
+
     # ---- end to end through the public API with host buffers ------------------
     hq, hk, hv, hx = (workloads.torch_bf16(a).pin_memory() for a in (lay.q, lay.k, lay.v, lay.x))
     outs = [plan.idx_kv, plan.idx_tsp, plan.k_c, plan.v_c, plan.x_c]
@@ -594,6 +718,19 @@ def main() -> None:
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": round(ach / peak, 4),
                          "traffic": load_traffic(dom)},
             "calls": breakdown,
+            "rvq_encode": {"ms": round(ms_rvq, 5), "rows": rvq_rows, "stages": rvq_S, "codebook": rvq_M,
+                           "rows_per_s": round(rvq_rows / (ms_rvq * 1e-3), 1),
+                           "tflops": round(rvq_flop / (ms_rvq * 1e-3) / 1e12, 2), "tflops_peak_tf32": tf32_peak,
+                           "peak_kind": tf32_kind,
+                           "frac": round(rvq_flop / (ms_rvq * 1e-3) / 1e12 / tf32_peak, 4),
+                           "note": "kvc_rvq_encode of the compacted K and V rows (tf32 scores, exact fp32 "
+                                   "decision); not part of the headline step"},
+            "decode": {"ms": round(ms_dec, 5), "alg_bytes": dec_bytes,
+                       "gbs": round(dec_bytes / (ms_dec * 1e-3) / 1e9, 1),
+                       "frac": round(dec_bytes / (ms_dec * 1e-3) / 1e9 / peak, 4),
+                       "note": "kvc_decode_attention: one decode query per head over the compacted cache "
+                               f"({cfg.Hkv} x {cfg.k_kv} entries, K and V), cache copies cycled past L2; "
+                               "not part of the headline step"},
             "score_lse": {"ms": round(ms_lse, 5), "alg_bytes": alg["score"],
                           "gbs": round(alg["score"] / (ms_lse * 1e-3) / 1e9, 1),
                           "max_rel_diff_vs_two_pass": rel_lse,

@@ -287,6 +287,61 @@ kvc_status kvc_gather_hidden(const uint16_t* x, int64_t stride_n, int64_t n, int
                              const int32_t* idx, int64_t kk, uint16_t* out, int32_t* dev_err,
                              void* stream);
 
+/* Decode over the compacted cache ---------------------------------------- */
+
+/* Workspace bytes for kvc_decode_attention (host only). */
+kvc_status kvc_decode_workspace_size(int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, int64_t kk,
+                                     size_t* bytes);
+
+/*
+ * Attention of one decode query per query head over the compacted cache
+ * [FastKV 2.B: the retained entries of every KV head are the cache the later
+ * decoding steps read; FastKV 1: decoding is bound by reading that cache].
+ * For query head h of KV head g = h / G (G = num_heads / num_kv_heads) and
+ * the kk retained entries of g:
+ *     s_j = scale * q[h, :] . k_c[g, j, :]
+ *     out[h, :] = sum_j exp(s_j - max s) v_c[g, j, :] / sum_j exp(s_j - max s)
+ * every retained entry visible (the decode query follows all of them).
+ *  q        [H][d] bf16, row h at q + h * q_stride_h (q_stride_h >= d)
+ *  k_c, v_c [Hkv][kk][d] bf16, contiguous (as kvc_gather_kv writes them),
+ *           16-byte aligned; kk >= 1, kk * Hkv < 2^31
+ *  out      [H][d] fp32, contiguous
+ *  ws       kvc_decode_workspace_size(H, Hkv, d, kk) bytes, 256-B aligned
+ *  dev_err  device int32 or NULL (KVC_DEV_ERR_TIMEOUT only)
+ * head_dim in {64, 128}; at most 16 query heads per KV head.  fp32
+ * arithmetic from the bf16 values; deterministic.
+ */
+kvc_status kvc_decode_attention(const uint16_t* q, int64_t q_stride_h, const uint16_t* k_c, const uint16_t* v_c,
+                                int64_t kk, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                                float* out, void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/* Residual vector quantisation of retained rows --------------------------- */
+
+/*
+ * Residual VQ codes of retained K or V rows  [VQKV (gist.science 2603.16435)
+ * 2: each cached vector becomes indices into codebooks; the first codebook
+ * encodes the vector, each later one the residual the earlier ones leave].
+ * For row t and stages s = 0 .. S-1 with codebooks C[s] ([M][d] each):
+ *     r_0 = x[t]
+ *     codes[t][s] = argmin_m ||r_s - C[s][m]||^2   (equal distances: lowest m)
+ *     r_{s+1}     = r_s - C[s][codes[t][s]]
+ *  x          [n][d] bf16, row t at x + t * x_stride (x_stride >= d); e.g. a
+ *             compacted cache [Hkv][kk][d] as n = Hkv * kk rows
+ *  codebooks  [S][M][d] fp32, contiguous, 16-byte aligned
+ *  codes      [n][S] int32 out
+ *  residual   [n][d] fp32 out or NULL: r_S, the row minus its reconstruction
+ *  dev_err    device int32 or NULL (KVC_DEV_ERR_TIMEOUT only)
+ * head_dim in {64, 128}; 16 <= M <= 256 with M % 16 == 0; 1 <= S <= 16.
+ * The scores r . C[s][m] are a tf32 tensor-core contraction; every codeword
+ * whose score lies within the bound of that rounding from the best one is
+ * re-scored as an fp32 distance, so a code departs from the exact argmin only
+ * where fp32 rounding of two nearly equal distances decides it.  The
+ * residual is carried in fp32.
+ */
+kvc_status kvc_rvq_encode(const uint16_t* x, int64_t x_stride, int64_t n, int32_t head_dim, const float* codebooks,
+                          int32_t stages, int32_t codebook_size, int32_t* codes, float* residual, int32_t* dev_err,
+                          void* stream);
+
 /* Statistics ------------------------------------------------------------- */
 
 /* Workspace bytes for kvc_layer_stats over `rows` rows. */

@@ -68,6 +68,10 @@ _SIGS = {
     "kvc_stats_workspace_size": ([_I32, _I64, _P], _I32),
     "kvc_layer_stats": ([_P, _I32, _I64, _I64, ctypes.c_float, _P, _P, _SZ, _P], _I32),
     "kvc_pivot_update": ([_P, _I32, _I32, ctypes.c_double, _I32, _I32, _P, _P, _P], _I32),
+    "kvc_rvq_encode": ([_P, _I64, _I64, _I32, _P, _I32, _I32, _P, _P, _P, _P], _I32),
+    "kvc_decode_workspace_size": ([_I32, _I32, _I32, _I64, _P], _I32),
+    "kvc_decode_attention": ([_P, _I64, _P, _P, _I64, _I32, _I32, _I32, ctypes.c_float, _P, _P, _SZ, _P, _P],
+                             _I32),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -484,6 +488,72 @@ def kvc_gather_hidden(x: torch.Tensor, idx: torch.Tensor, out: Optional[torch.Te
     _check(_call(dev, lib().kvc_gather_hidden, _ptr(x), x.stride(0), n, D, _ptr(idx), kk, _ptr(out),
                  _ptr(dev_err), _stream(stream, dev)), "kvc_gather_hidden")
     return out
+
+
+# --------------------------------------------------------------------------- #
+# decode over the compacted cache
+# --------------------------------------------------------------------------- #
+def decode_workspace_size(H: int, Hkv: int, d: int, kk: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(lib().kvc_decode_workspace_size(H, Hkv, d, kk, ctypes.byref(out)), "kvc_decode_workspace_size")
+    return int(out.value)
+
+
+def kvc_decode_attention(q: torch.Tensor, k_c: torch.Tensor, v_c: torch.Tensor, scale: Optional[float] = None,
+                         out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                         dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """One decode query per head, q [H][d], over the compacted cache
+    k_c, v_c [Hkv][kk][d] (every retained entry visible); returns fp32 [H][d]."""
+    _bf16(q, "q", 2)
+    _bf16(k_c, "k_c", 3)
+    _bf16(v_c, "v_c", 3)
+    dev = k_c.device
+    _same_device(dev, q=q, v_c=v_c)
+    H, d = q.shape
+    Hkv, kk, dk = k_c.shape
+    if dk != d or tuple(v_c.shape) != (Hkv, kk, d):
+        raise ValueError("q [H][d], k_c and v_c [Hkv][kk][d] must agree")
+    if not (k_c.is_contiguous() and v_c.is_contiguous()):
+        raise ValueError("k_c and v_c must be contiguous")
+    if out is None:
+        out = torch.empty((H, d), dtype=torch.float32, device=dev)
+    _dense(out, "out", (H, d), torch.float32, dev)
+    _err_word(dev_err, dev)
+    if ws is None:
+        ws = _workspace(decode_workspace_size(H, Hkv, d, kk), dev)
+    sc = float(1.0 / math.sqrt(d) if scale is None else scale)
+    _check(_call(dev, lib().kvc_decode_attention, _ptr(q), q.stride(0), _ptr(k_c), _ptr(v_c), kk, H, Hkv, d, sc,
+                 _ptr(out), _ptr(ws), _ws_bytes(ws, dev), _ptr(dev_err), _stream(stream, dev)),
+           "kvc_decode_attention")
+    return out
+
+
+# --------------------------------------------------------------------------- #
+# residual vector quantisation
+# --------------------------------------------------------------------------- #
+def kvc_rvq_encode(x: torch.Tensor, codebooks: torch.Tensor, codes: Optional[torch.Tensor] = None,
+                   residual: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                   stream=None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Residual VQ of rows x [n][d] (bf16) against fp32 codebooks [S][M][d]:
+    returns (codes int32 [n][S], residual fp32 [n][d] if one was passed)."""
+    _bf16(x, "x", 2)
+    dev = x.device
+    _same_device(dev, codebooks=codebooks)
+    n, d = x.shape
+    if codebooks.dtype != torch.float32 or codebooks.dim() != 3 or codebooks.shape[2] != d:
+        raise ValueError(f"codebooks must be float32 [S][M][{d}]")
+    if not codebooks.is_contiguous():
+        raise ValueError("codebooks must be contiguous")
+    S, M = codebooks.shape[0], codebooks.shape[1]
+    if codes is None:
+        codes = torch.empty((n, S), dtype=torch.int32, device=dev)
+    _dense(codes, "codes", (n, S), torch.int32, dev)
+    if residual is not None:
+        _dense(residual, "residual", (n, d), torch.float32, dev)
+    _err_word(dev_err, dev)
+    _check(_call(dev, lib().kvc_rvq_encode, _ptr(x), x.stride(0), n, d, _ptr(codebooks), S, M, _ptr(codes),
+                 _ptr(residual), _ptr(dev_err), _stream(stream, dev)), "kvc_rvq_encode")
+    return codes, residual
 
 
 # --------------------------------------------------------------------------- #

@@ -12,6 +12,18 @@ the same number of positions.  The GPU set must in any case be ascending,
 unique, of the right size and contain the window.
 
 Gathers: bit-exact.
+
+Residual VQ codes: where the oracle's best and second-best distances of a
+stage differ by more than 1e-4 of the best (float64 against the kernel's fp32
+residual and distances), the codes must be identical; at a closer call the
+kernel's codeword must be within that band of the best along the same
+residual, and the row is not followed further (the residuals part ways).
+
+Decode attention over the compacted cache: per query head,
+max |gpu - oracle| <= 1e-3 * max |oracle| over the head's output row (the
+outputs are signed sums that can cancel, so the row's largest magnitude sets
+the scale; fp32 arithmetic keeps the error about 1e-6 of the weighted sum of
+|v|, i.e. well inside this bound).
 """
 from __future__ import annotations
 
@@ -80,3 +92,44 @@ def assert_selection_matches(gpu_idx, orc_idx, orc_S, n: int, w: int, k: int, wh
     assert np.array_equal(g[~band], o[~band]), f"{what}: sets differ outside the near-tie band"
     assert g[band].sum() == o[band].sum(), f"{what}: different counts inside the near-tie band"
     return "band"
+
+
+def assert_decode_close(gpu, ref, rtol: float = SCORE_RTOL, what: str = "decode"):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    worst = 0.0
+    for h in range(ref.shape[0]):
+        scale = np.max(np.abs(ref[h]))
+        err = np.max(np.abs(gpu[h] - ref[h])) / scale if scale > 0 else np.max(np.abs(gpu[h]))
+        worst = max(worst, err)
+        assert err <= rtol, f"{what}: head {h} error {err:.3e} of the row's largest magnitude > {rtol:.0e}"
+    return worst
+
+
+RVQ_BAND = 1e-4
+
+
+def check_rvq_codes(gpu_codes, orc_codes, orc_gap, x_bits, C, what: str = "rvq"):
+    """Returns the number of rows decided inside the near-tie band."""
+    gpu_codes = np.asarray(gpu_codes)
+    orc_codes = np.asarray(orc_codes)
+    n, S = orc_codes.shape
+    near = 0
+    x = x_bits.astype(np.uint32) << 16
+    xf = x.view(np.float32).astype(np.float64)
+    for t in range(n):
+        for s in range(S):
+            if gpu_codes[t, s] == orc_codes[t, s]:
+                continue
+            # the residual the oracle ranked at this stage (earlier codes agree)
+            r = xf[t] - sum(C[u][orc_codes[t, u]].astype(np.float64) for u in range(s))
+            dist = np.sum((r[None, :] - C[s].astype(np.float64)) ** 2, axis=1)
+            best = dist.min()
+            assert orc_gap[t, s] <= RVQ_BAND * max(best, 1e-12), (
+                f"{what}: row {t} stage {s}: code {gpu_codes[t, s]} != {orc_codes[t, s]} with a gap of "
+                f"{orc_gap[t, s]:.3e} (best {best:.6e})")
+            assert dist[gpu_codes[t, s]] - best <= RVQ_BAND * max(best, 1e-12), (
+                f"{what}: row {t} stage {s}: code {gpu_codes[t, s]} is not a near-argmin")
+            near += 1
+            break
+    return near

@@ -132,3 +132,37 @@ def test_given_normaliser_and_pivot_calls_reject_bad_arguments(lib):
     assert lib.kvc_pivot_update(dummy, 8, 1, 0.1, 1, 4, ctypes.c_void_p(516), None, None) == 1
     assert kvc.last_error() != ""
     assert kvc.launch_count() == before
+
+
+def test_decode_attention_rejects_bad_arguments(lib):
+    dummy = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    before = kvc.launch_count()
+    n = ctypes.c_size_t()
+    assert lib.kvc_decode_workspace_size(32, 8, 128, 13107, ctypes.byref(n)) == 0 and n.value > 0
+    assert lib.kvc_decode_workspace_size(32, 8, 96, 13107, ctypes.byref(n)) == 2      # head_dim 96
+    assert lib.kvc_decode_workspace_size(32, 8, 128, 0, ctypes.byref(n)) == 1         # no entries
+    assert lib.kvc_decode_workspace_size(34, 2, 128, 100, ctypes.byref(n)) == 2       # 17 heads per KV head
+    assert lib.kvc_decode_workspace_size(30, 8, 128, 100, ctypes.byref(n)) == 1       # H not a multiple of Hkv
+    ws = 1 << 20
+    # NULL out, misaligned k_c, q stride below head_dim, zero scale, workspace too small
+    assert lib.kvc_decode_attention(dummy, 128, dummy, dummy, 100, 32, 8, 128, 0.1, None, dummy, ws, None, None) == 1
+    assert lib.kvc_decode_attention(dummy, 128, ctypes.c_void_p(264), dummy, 100, 32, 8, 128, 0.1, dummy, dummy, ws,
+                                    None, None) == 1
+    assert lib.kvc_decode_attention(dummy, 64, dummy, dummy, 100, 32, 8, 128, 0.1, dummy, dummy, ws, None, None) == 1
+    assert lib.kvc_decode_attention(dummy, 128, dummy, dummy, 100, 32, 8, 128, 0.0, dummy, dummy, ws, None, None) == 1
+    assert lib.kvc_decode_attention(dummy, 128, dummy, dummy, 100, 32, 8, 128, 0.1, dummy, dummy, 16, None, None) == 4
+    assert kvc.launch_count() == before
+
+
+def test_rvq_encode_rejects_bad_arguments(lib):
+    dummy = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    before = kvc.launch_count()
+    assert lib.kvc_rvq_encode(dummy, 128, 10, 96, dummy, 4, 256, dummy, None, None, None) == 2   # head_dim 96
+    assert lib.kvc_rvq_encode(dummy, 128, 10, 128, dummy, 4, 300, dummy, None, None, None) == 2  # M > 256
+    assert lib.kvc_rvq_encode(dummy, 128, 10, 128, dummy, 4, 40, dummy, None, None, None) == 2   # M % 16
+    assert lib.kvc_rvq_encode(dummy, 128, 10, 128, dummy, 0, 256, dummy, None, None, None) == 1  # no stage
+    assert lib.kvc_rvq_encode(dummy, 64, 10, 128, dummy, 4, 256, dummy, None, None, None) == 1   # stride < d
+    assert lib.kvc_rvq_encode(dummy, 128, 10, 128, ctypes.c_void_p(260), 4, 256, dummy, None, None, None) == 1
+    assert lib.kvc_rvq_encode(dummy, 128, 10, 128, dummy, 4, 256, None, None, None, None) == 1   # NULL codes
+    assert lib.kvc_rvq_encode(dummy, 128, 0, 128, dummy, 4, 256, dummy, None, None, None) == 0   # nothing to do
+    assert kvc.launch_count() == before

@@ -406,6 +406,157 @@ def test_varlen_seqlens_past_the_total_flagged():
 
 
 # --------------------------------------------------------------------------- #
+# one layer split by KV head (the ranks emulated one after another)
+# --------------------------------------------------------------------------- #
+def test_kv_head_split_reproduces_the_layer():
+    """Two ranks of a KV-head split run one after another on this GPU (no
+    rank waits for another): each scores its four KV heads through strided
+    views of the layer's tensors; their partial all-head rows are added (the
+    all-reduce of a multi-GPU run); each then ranks the summed row and
+    gathers its half of the hidden columns and its heads' K/V.  Against the
+    oracle: TSP and K/V sets under the band rule, gathers bit-exact."""
+    from long_context_kv_window_b200 import shard
+    cfg = workloads.shrink(workloads.C3, N=20000, k_kv=2000, k_tsp=4000, hidden=1024, n_hitters=64, seed=88)
+    lay = workloads.make_layer(cfg)
+    q, k, v, x = (dev_bf16(a) for a in (lay.q, lay.k, lay.v, lay.x))
+    parts = [shard.HeadSplitLayer(r, 2, cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden, "cuda",
+                                  pool_kernel=cfg.pool) for r in range(2)]
+    rows = [p.score_local(q, k) for p in parts]
+    total = rows[0] + rows[1]
+    for p in parts:
+        p.tsp.copy_(total)
+        p.finish(k, v, x)
+    torch.cuda.synchronize()
+    res = oracle.layer(lay.q, lay.k, cfg.H, cfg.Hkv, cfg.w, cfg.scale, cfg.pool, cfg.k_kv, cfg.k_tsp)
+    it = parts[0].idx_tsp[0].cpu().numpy()
+    assert np.array_equal(it, parts[1].idx_tsp[0].cpu().numpy())
+    parity.assert_selection_matches(it, res.idx_tsp, res.pooled_tsp, cfg.N, cfg.w, cfg.k_tsp, what="split TSP set")
+    xc = np.concatenate([host_bits(p.x_c) for p in parts], axis=1)
+    assert np.array_equal(xc, lay.x[it])
+    for p in parts:
+        assert p.dev_err.item() == 0
+        parity.assert_scores_close(p.scores.cpu().numpy(), res.A[p.g0:p.g1], what=f"rank {p.rank} scores")
+        idx = p.idx_kv.cpu().numpy()
+        kc, vc = host_bits(p.k_c), host_bits(p.v_c)
+        for gl, g in enumerate(range(p.g0, p.g1)):
+            parity.assert_selection_matches(idx[gl], res.idx_kv[g], res.pooled[g], cfg.N, cfg.w, cfg.k_kv,
+                                            what=f"split K/V set of head {g}")
+            assert np.array_equal(kc[gl], lay.k[idx[gl], g, :]) and np.array_equal(vc[gl], lay.v[idx[gl], g, :])
+
+
+# --------------------------------------------------------------------------- #
+# decode attention over the compacted cache
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("H,Hkv,d,kk", [(32, 8, 128, 13107), (32, 8, 128, 1), (32, 8, 128, 63), (8, 8, 64, 64),
+                                        (40, 8, 128, 4096), (16, 1, 128, 2000), (8, 2, 64, 65), (6, 3, 128, 777)])
+def test_decode_attention_matches_oracle(H, Hkv, d, kk):
+    """One decode query per head over [Hkv][kk][d] retained entries: the
+    128K layer's 13107 entries per head, single and ragged tiles, G = 1, 5
+    and 16 query heads per KV head, head_dim 64; a few planted entries carry
+    most of the attention."""
+    rng = np.random.default_rng(H * 1000 + kk + d)
+    q = workloads.f32_to_bf16_bits(rng.standard_normal((H, d)).astype(np.float32))
+    kc = workloads.f32_to_bf16_bits(rng.standard_normal((Hkv, kk, d)).astype(np.float32))
+    vc = workloads.f32_to_bf16_bits(rng.standard_normal((Hkv, kk, d)).astype(np.float32))
+    if kk > 8:  # planted heavy entries: K aligned with the group's queries
+        G = H // Hkv
+        qf = workloads.bf16_bits_to_f32(q).reshape(Hkv, G, d).mean(axis=1)
+        for g in range(Hkv):
+            pos = rng.choice(kk, size=3, replace=False)
+            u = qf[g] / np.linalg.norm(qf[g])
+            kc[g, pos] = workloads.f32_to_bf16_bits((3.0 * np.sqrt(d) * u)[None, :].repeat(3, 0).astype(np.float32))
+    err = _err_word()
+    out = kvc.kvc_decode_attention(dev_bf16(q), dev_bf16(kc), dev_bf16(vc), dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref = oracle.get().decode_attention(q, kc, vc, H, Hkv, 1 / math.sqrt(d))
+    parity.assert_decode_close(out.cpu().numpy(), ref, what=f"decode H={H} Hkv={Hkv} d={d} kk={kk}")
+
+
+def test_decode_over_the_layers_compacted_cache():
+    """The cache a 32K layer's K/V retention leaves (scores -> per-KV-head
+    top-k -> K/V gather) decoded with a fresh query per head, against the
+    oracle's decode of the same cache."""
+    cfg = workloads.shrink(workloads.C2, N=32768, seed=202)
+    lay = workloads.make_layer(cfg)
+    q, k, v = dev_bf16(lay.q), dev_bf16(lay.k), dev_bf16(lay.v)
+    scores = kvc.kvc_score(q, k)
+    idx = kvc.kvc_select_topk(scores, cfg.w, cfg.pool, cfg.k_kv)
+    kc, vc = kvc.kvc_gather_kv(k, v, idx)
+    rng = np.random.default_rng(5)
+    qd = workloads.f32_to_bf16_bits(rng.standard_normal((cfg.H, cfg.d)).astype(np.float32))
+    out = kvc.kvc_decode_attention(dev_bf16(qd), kc, vc)
+    torch.cuda.synchronize()
+    ref = oracle.get().decode_attention(qd, host_bits(kc), host_bits(vc), cfg.H, cfg.Hkv, cfg.scale)
+    parity.assert_decode_close(out.cpu().numpy(), ref, what="decode over the compacted 32K layer")
+
+
+# --------------------------------------------------------------------------- #
+# residual vector quantisation
+# --------------------------------------------------------------------------- #
+@pytest.mark.parametrize("n,d,S,M", [(1000, 128, 4, 256), (129, 128, 2, 256), (300, 64, 3, 64), (77, 128, 1, 16),
+                                     (5000, 128, 8, 128)])
+def test_rvq_encode_matches_oracle(n, d, S, M):
+    """Random rows against random codebooks (stage s at scale 2^-s): codes
+    identical to the oracle outside the near-tie band, and the returned
+    residual is the row minus its reconstruction."""
+    rng = np.random.default_rng(n + d + S + M)
+    x = workloads.f32_to_bf16_bits(rng.standard_normal((n, d)).astype(np.float32))
+    C = workloads.make_codebooks(S, M, d, seed=n + M)
+    xd, Cd = dev_bf16(x), torch.from_numpy(C).cuda()
+    residual = torch.empty((n, d), dtype=torch.float32, device="cuda")
+    err = _err_word()
+    codes, _ = kvc.kvc_rvq_encode(xd, Cd, residual=residual, dev_err=err)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    ref_codes, gap = oracle.get().rvq_encode(x, C)
+    gc = codes.cpu().numpy()
+    near = parity.check_rvq_codes(gc, ref_codes, gap, x, C, what=f"rvq n={n} d={d} S={S} M={M}")
+    assert near <= max(2, n // 100), f"{near} rows decided inside the near-tie band"
+    xf = workloads.bf16_bits_to_f32(x).astype(np.float64)
+    rec = sum(C[s][gc[:, s]].astype(np.float64) for s in range(S))
+    np.testing.assert_allclose(residual.cpu().numpy(), xf - rec, rtol=0, atol=1e-5)
+
+
+def test_rvq_encode_planted_codes_and_ties():
+    """Rows built as one codeword per stage (codebooks of entries +-8^-s,
+    exact in bf16) come back with exactly those codes and a zero residual;
+    a duplicated codeword resolves to the lower index."""
+    rng = np.random.default_rng(71)
+    n, d, M, S = 700, 128, 64, 3
+    C = np.stack([rng.choice([-1.0, 1.0], size=(M, d)) * 8.0 ** -s for s in range(S)]).astype(np.float32)
+    C[0, 40] = C[0, 9]  # codeword 40 duplicates codeword 9
+    planted = rng.integers(0, M, size=(n, S))
+    planted[:, 0] = np.where(planted[:, 0] == 40, 9, planted[:, 0])
+    xf = sum(C[s][planted[:, s]].astype(np.float64) for s in range(S))
+    x = workloads.f32_to_bf16_bits(xf.astype(np.float32))
+    assert np.array_equal(workloads.bf16_bits_to_f32(x).astype(np.float64), xf)
+    residual = torch.empty((n, d), dtype=torch.float32, device="cuda")
+    codes, _ = kvc.kvc_rvq_encode(dev_bf16(x), torch.from_numpy(C).cuda(), residual=residual)
+    torch.cuda.synchronize()
+    assert np.array_equal(codes.cpu().numpy(), planted)
+    assert not residual.cpu().numpy().any()
+
+
+def test_rvq_encode_the_layers_compacted_cache():
+    """The compacted K cache of a 32K layer ([8][2048][128] as 16384 rows),
+    four stages of 256 codewords, against the oracle."""
+    cfg = workloads.shrink(workloads.C2, N=32768, seed=303)
+    lay = workloads.make_layer(cfg)
+    q, k = dev_bf16(lay.q), dev_bf16(lay.k)
+    idx = kvc.kvc_select_topk(kvc.kvc_score(q, k), cfg.w, cfg.pool, cfg.k_kv)
+    kc, _ = kvc.kvc_gather_kv(k, None, idx)
+    rows = kc.view(-1, cfg.d)
+    C = workloads.make_codebooks(4, 256, cfg.d, seed=9)
+    codes, _ = kvc.kvc_rvq_encode(rows, torch.from_numpy(C).cuda())
+    torch.cuda.synchronize()
+    xb = host_bits(rows)
+    ref_codes, gap = oracle.get().rvq_encode(xb, C)
+    near = parity.check_rvq_codes(codes.cpu().numpy(), ref_codes, gap, xb, C, what="rvq of the compacted cache")
+    assert near <= rows.shape[0] // 100
+
+
+# --------------------------------------------------------------------------- #
 # statistics
 # --------------------------------------------------------------------------- #
 def test_layer_stats_against_oracle():

@@ -1,5 +1,7 @@
 """Multi-rank host logic on CPU (gloo, world size 2): sequence sharding of a
-ragged batch and the max-over-ranks timing used by bench.py."""
+ragged batch, the max-over-ranks timing used by bench.py, and one layer
+split by KV head (partition, all-reduced TSP row, column slices of the hidden
+states) on the float64 oracle's scores."""
 import os
 import socket
 
@@ -71,3 +73,75 @@ def test_two_ranks_agree_on_the_shards_and_the_max_time():
         assert got == expect
         assert mx == 1.5
     assert sorted(i for p in expect for i in p) == list(range(len(lens)))
+
+
+def test_head_and_column_ranges_partition_everything():
+    for Hkv in (1, 2, 8):
+        for world in range(1, Hkv + 1):
+            r = shard.head_ranges(Hkv, world)
+            assert r[0][0] == 0 and r[-1][1] == Hkv
+            assert all(a[1] == b[0] for a, b in zip(r, r[1:]))
+            assert max(b - a for a, b in r) - min(b - a for a, b in r) <= 1
+    for world in (1, 2, 3, 8):
+        c = shard.column_ranges(4096, world)
+        assert c[0][0] == 0 and c[-1][1] == 4096 and all(a % 8 == 0 for a, _ in c)
+        assert all(a[1] == b[0] for a, b in zip(c, c[1:]))
+
+
+def _split_worker(rank, world, port, q):
+    """One rank of a KV-head split of a small layer, on the oracle: its heads'
+    scores, its partial all-head row, the row summed over ranks (gloo), the
+    TSP set and its column slice of the hidden gather, its heads' K sets."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import oracle
+        import workloads
+        cfg = workloads.shrink(workloads.C3, N=4096, k_kv=410, k_tsp=819, hidden=512, n_hitters=16, seed=77)
+        lay = workloads.make_layer(cfg)
+        orc = oracle.get()
+        g0, g1 = shard.head_ranges(cfg.Hkv, world)[rank]
+        c0, c1 = shard.column_ranges(cfg.hidden, world)[rank]
+        A = orc.window_scores(lay.q[:, g0 * cfg.G:g1 * cfg.G, :], lay.k[:, g0:g1, :], (g1 - g0) * cfg.G, g1 - g0,
+                              cfg.w, cfg.scale)
+        T = torch.from_numpy(orc.sum_rows(A))
+        dist.all_reduce(T, op=dist.ReduceOp.SUM)
+        pt = orc.rank_scores(T.numpy(), cfg.N, cfg.w, cfg.pool)
+        idx_tsp = orc.select_topk(pt, cfg.N, cfg.w, cfg.k_tsp)
+        x_c, _ = orc.gather_rows(lay.x[:, c0:c1], idx_tsp)
+        idx_kv, _ = orc.select_rows(A, cfg.N, cfg.w, cfg.pool, cfg.k_kv)
+        q.put((rank, (g0, g1), (c0, c1), idx_tsp, pt, x_c, idx_kv))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_split_one_layer_by_kv_head():
+    """The KV-head split reproduces the single-rank layer: the summed row
+    ranks to the single-rank TSP set (near-tie band: the float64 sum runs in
+    another order), each rank's K sets are the single-rank sets of its heads,
+    and the column slices of the hidden gather concatenate to the full one."""
+    import oracle
+    import workloads
+    from tests import parity
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_split_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=300) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    cfg = workloads.shrink(workloads.C3, N=4096, k_kv=410, k_tsp=819, hidden=512, n_hitters=16, seed=77)
+    lay = workloads.make_layer(cfg)
+    full = oracle.layer(lay.q, lay.k, cfg.H, cfg.Hkv, cfg.w, cfg.scale, cfg.pool, cfg.k_kv, cfg.k_tsp)
+    assert [r[1] for r in res] == [(0, 4), (4, 8)] and [r[2] for r in res] == [(0, 256), (256, 512)]
+    for rank, (g0, g1), _, idx_tsp, pt, _, idx_kv in res:
+        parity.assert_selection_matches(idx_tsp, full.idx_tsp, full.pooled_tsp, cfg.N, cfg.w, cfg.k_tsp,
+                                        what=f"TSP set on rank {rank}")
+        np.testing.assert_allclose(pt, full.pooled_tsp, rtol=1e-12)
+        assert np.array_equal(idx_kv, full.idx_kv[g0:g1])
+    assert np.array_equal(res[0][3], res[1][3]), "the ranks must select the same TSP set"
+    x_full, _ = oracle.get().gather_rows(lay.x, res[0][3])
+    assert np.array_equal(np.concatenate([res[0][5], res[1][5]], axis=1), x_full)

@@ -283,3 +283,12 @@ def make_layer(cfg: LayerConfig, with_x: Optional[bool] = None, seed: Optional[i
         sinks.append(s)
         hitters.append(hpos)
     return Layer(cfg, q, k, v, x, cu.astype(np.int32), sinks, hitters)
+
+
+def make_codebooks(stages: int, size: int, d: int, seed: int) -> np.ndarray:
+    """Random residual-VQ codebooks float32 [stages][size][d]: stage s draws
+    N(0, 1) * 2^-s (each later stage refines a smaller residual).  Stand-ins
+    for trained codebooks, which need training data."""
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed)))
+    scale = (2.0 ** -np.arange(stages, dtype=np.float64))[:, None, None]
+    return (g.standard_normal((stages, size, d)) * scale).astype(np.float32)
