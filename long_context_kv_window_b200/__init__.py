@@ -623,7 +623,7 @@ class LayerPlan:
     """Pre-allocated buffers for repeated calls of ``compress_layer`` on one shape."""
 
     def __init__(self, n: int, H: int, Hkv: int, d: int, w: int, k_kv: int, k_tsp: Optional[int],
-                 hidden: Optional[int], with_v: bool, device, pool_kernel: int = 1):
+                 hidden: Optional[int], with_v: bool, device, pool_kernel: int = 1, tsp_row: bool = False):
         self.n, self.H, self.Hkv, self.d, self.w = n, H, Hkv, d, w
         self.k_kv, self.k_tsp, self.hidden, self.pool = k_kv, k_tsp, hidden, pool_kernel
         f32, i32, bf = torch.float32, torch.int32, torch.bfloat16
@@ -636,8 +636,10 @@ class LayerPlan:
         self.v_c = torch.empty_like(self.k_c) if with_v else None
         self.dev_err = torch.zeros(1, dtype=i32, device=device)
         self.tsp = None
+        self.tsp_row = tsp_row
         if k_tsp is not None:
-            self.tsp = torch.empty((1, n), dtype=f32, device=device)  # all-head score sums
+            if tsp_row:  # the scoring call also writes the all-head sum row, which the TSP selection ranks
+                self.tsp = torch.empty((1, n), dtype=f32, device=device)
             self.ws_sel_tsp = _workspace(select_workspace_size(1, 1, n), device)
             self.idx_tsp = torch.empty((1, min(k_tsp, n)), dtype=i32, device=device)
             self.x_c = (torch.empty((min(k_tsp, n), hidden), dtype=bf, device=device)
@@ -650,8 +652,10 @@ class LayerPlan:
         """Score -> per-KV-head top-k -> K/V gather; with a TSP budget also the
         all-head top-k -> hidden-state gather.
 
-        The scoring call also writes the all-head sum of the scores (one row),
-        which the TSP selection ranks.  The two selection -> gather chains only
+        The TSP selection ranks the sum of the KV-head score rows, formed as it
+        stages them (heads in order, the same fp32 sum as the scoring call's
+        optional head-sum row, which it writes to out.tsp when the plan was
+        made with tsp_row=True).  The two selection -> gather chains only
         share the scores, so the K/V chain runs on a side stream concurrently
         with the TSP chain (enqueued first: it leads to the longer gather);
         both join the calling stream before returning.  Nothing is
@@ -665,8 +669,12 @@ class LayerPlan:
             self._kv_chain(k, v, main)
             return out
         self._ev_scores.record(main)
-        kvc_select_topk(self.tsp, self.w, self.pool, self.k_tsp, idx=self.idx_tsp, ws=self.ws_sel_tsp,
-                        stream=main)
+        if self.tsp_row:
+            kvc_select_topk(self.tsp, self.w, self.pool, self.k_tsp, idx=self.idx_tsp, ws=self.ws_sel_tsp,
+                            stream=main)
+        else:
+            kvc_select_topk(self.scores, self.w, self.pool, self.k_tsp, row_group=self.Hkv, idx=self.idx_tsp,
+                            ws=self.ws_sel_tsp, stream=main)
         self.side.wait_event(self._ev_scores)
         self._kv_chain(k, v, self.side)
         out.idx_tsp = self.idx_tsp

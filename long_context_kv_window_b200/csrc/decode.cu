@@ -14,7 +14,13 @@
 // Kc[g] / Vc[g] in 64-entry tiles through TMA (128-byte swizzle, so that one
 // lane per entry reads its row without bank conflicts), keeps an online
 // softmax per query head, and writes a partial (max, sum, output row); a
-// second kernel merges the partials of each head.
+// second kernel, launched early (programmatic dependent launch) and waiting
+// on the first, merges the partials of each head.
+//
+// A dedicated producer warp keeps the TMA ring full: it refills a stage as
+// soon as the eight compute warps have released it, so loads of later tiles
+// are in flight while the compute warps work on earlier ones (a refill
+// issued by a compute warp would wait for the slowest warp of every tile).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -27,7 +33,8 @@ namespace kvc {
 namespace {
 
 constexpr int kT = 64;             // retained entries per tile
-constexpr int kDecThreads = 256;
+constexpr int kDecThreads = 256;              // compute warps
+constexpr int kDecBlock = kDecThreads + 32;   // + the producer warp
 constexpr int kDecStages = 3;
 constexpr int kDecMaxG = 16;       // query heads per KV head
 constexpr int kDecCtaTarget = 296; // CTAs per launch: two per SM on 148 SMs
@@ -54,8 +61,8 @@ struct DecSmem {
   static constexpr int kMatBytes = kBoxes * kT * 128;        // one K or V tile
   static constexpr int kStageBytes = 2 * kMatBytes;          // K tile, then V tile
   static constexpr size_t kFloats = (size_t)kDecMaxG * (D + 16) + (size_t)kDecMaxG * kT + 3 * kDecMaxG;
-  static_assert((size_t)kDecStages * kStageBytes >= (size_t)(kDecThreads / (D / 2)) * kDecMaxG * D * 4,
-                "the partial reduction reuses the stages");
+  static_assert((size_t)kDecStages * kStageBytes >= (size_t)(kDecThreads / 32) * kDecMaxG * (D + 2) * 4,
+                "the merge of the warps reuses the stages");
   static constexpr size_t kBytes = 1024 + (size_t)kDecStages * kStageBytes + kFloats * 4 + 128;
 };
 
@@ -70,52 +77,60 @@ __device__ __forceinline__ int sw128(int j, int k16) { return j * 128 + ((k16 ^ 
 
 // KG: query heads per KV head the kernel is built for (a.G <= KG; heads
 // past a.G are zero padding whose outputs are dropped).
+//
+// Every warp owns 8 entries of each 64-entry tile from start to end: their
+// logits (four lanes per entry, a quarter of the dimensions each), an online
+// softmax per head over the warp's own entries, and the warp's output rows
+// (four or two dimensions per lane).  No block-wide barrier runs per tile: a
+// warp releases the stage through an mbarrier (one arrival per warp) and
+// thread 0 refills it once all eight have.  The eight warps' (max, sum,
+// output) are merged once at the end.
+// Two CTAs per SM up to four heads per group; wider groups keep their
+// per-head state in registers at one CTA per SM instead of spilling it.
 template <int D, int KG>
-__global__ void __launch_bounds__(kDecThreads, 2)
+__global__ void __launch_bounds__(kDecBlock, KG <= 4 ? 2 : 1)
 decode_partial_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                       const DecArgs a) {
   using L = DecSmem<D>;
+  constexpr int kWarps = kDecThreads / 32;       // 8
+  constexpr int kPerWarp = kT / kWarps;          // entries per warp and tile (8)
+  constexpr int kQuarter = D / 4;                // dimensions per logit lane
+  constexpr int kQRow = D + 16;                  // floats per head of q (four padded quarters)
+  constexpr int kQChunks = kQuarter / 8;         // 16-byte chunks per logit lane
+  constexpr int kDL = D / 32;                    // output dimensions per lane (4 or 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* stages = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float* qs = reinterpret_cast<float*>(stages + (size_t)kDecStages * L::kStageBytes);  // [KG][D + 16]
-  float* P = qs + kDecMaxG * (D + 16);                                                  // [kT][KG]: logits, then p
-  float* m_run = P + kDecMaxG * kT;
-  float* l_run = m_run + kDecMaxG;
-  float* alpha = l_run + kDecMaxG;
-  uint64_t* full = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(alpha + kDecMaxG) + 15) & ~uintptr_t(15));
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(full + kDecStages);
+  float* pw = qs + kDecMaxG * (D + 16);                    // [warp][kPerWarp][KG]: this tile's p
+  uint64_t* full = reinterpret_cast<uint64_t*>(
+      (reinterpret_cast<uintptr_t>(pw + kDecMaxG * kT) + 15) & ~uintptr_t(15));
+  uint64_t* empty = full + kDecStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + kDecStages);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = blockIdx.y, chunk = blockIdx.x;
   const int G = a.G;
-  constexpr int kQuarter = D / 4;            // dimensions per logit thread
-  constexpr int kQRow = D + 16;              // floats per head of q (four padded quarters)
   const int64_t e0 = (int64_t)chunk * a.chunk;
   const int64_t e1 = std::min<int64_t>(a.kk, e0 + a.chunk);
   const int ntiles = (int)((e1 - e0 + kT - 1) / kT);
   const int64_t row0 = (int64_t)g * a.kk + e0;  // first row of the chunk in the [Hkv*kk][D] view
 
   if (tid == 0) {
-    for (int s = 0; s < kDecStages; ++s) tc::mbar_init(&full[s], 1);
+    for (int s = 0; s < kDecStages; ++s) {
+      tc::mbar_init(&full[s], 1);
+      tc::mbar_init(&empty[s], kWarps);
+    }
     *abort_flag = 0;
     tc::fence_mbar_init();
+  }
+  if (tid == kDecThreads) {
     tc::prefetch_tmap(&kmap);
     tc::prefetch_tmap(&vmap);
   }
-  if (tid < kDecMaxG) {
-    m_run[tid] = -INFINITY;
-    l_run[tid] = 0.f;
-  }
-  pdl_wait();  // Kc / Vc / q may come from the previous kernel of the stream
-  // q as fp32, each head's D values in four quarters of D/4, every quarter
-  // padded by 4 floats: the four threads of an entry read their quarters at
-  // different shared-memory banks
-  for (int i = tid; i < KG * D; i += kDecThreads) {
-    const int h = i / D, e = i % D;
-    qs[h * kQRow + (e / kQuarter) * (kQuarter + 4) + e % kQuarter] =
-        h < G ? __uint_as_float((uint32_t)a.q[(int64_t)(g * G + h) * a.q_sh + e] << 16) : 0.f;
-  }
   __syncthreads();
+  pdl_wait();  // Kc / Vc / q may come from the previous kernel of the stream
+  // the merge kernel may launch now: it waits for this grid's completion
+  pdl_trigger();
 
   auto issue = [&](int t) {
     const int s = t % kDecStages;
@@ -128,45 +143,62 @@ decode_partial_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
       tc::tma_load_2d(dst + L::kMatBytes + cb * kT * 128, &vmap, &full[s], cb * 64, y);
     }
   };
-  int issued = 0;  // thread 0
-  if (tid == 0)
-    for (; issued < min(ntiles, kDecStages); ++issued) issue(issued);
-
-  // Logits: four threads per entry, each a quarter of the D dimensions for
-  // every head of the group (one read and unpack of each K element).
-  constexpr int kQChunks = kQuarter / 8;     // 16-byte chunks per thread
-  const int lj = tid >> 2, lq = tid & 3;     // entry, quarter
-  // Output: one thread per pair of dimensions and group of entries; it adds
-  // every head's p * v for its entries (one read of each V element).
-  constexpr int kPairs = D / 2;
-  constexpr int kGroups = kDecThreads / kPairs;  // 4 (D = 128) or 8 (D = 64)
-  constexpr int kPerGroup = kT / kGroups;
-  const int dp = tid % kPairs, og = tid / kPairs;
-  const int oe = 2 * dp, ocb = oe / 64, oe64 = oe % 64;
-  float2 o[KG];
+  const int je = lane >> 2, lq = lane & 3;  // logits: entry of the warp, quarter
+  constexpr int kDP = kDL / 2;              // output dimension pairs per lane
+  constexpr int kKG4 = (KG + 3) / 4;        // float4 groups of a p row
+  float m_w[KG], l_w[KG];                   // this warp's running max and sum per head
+  float2 o[KG][kDP];                        // this warp's output dims of this lane, per head
 #pragma unroll
-  for (int h = 0; h < KG; ++h) o[h] = make_float2(0.f, 0.f);
-
-  int t = 0;
-  for (; t < ntiles; ++t) {
-    const int s = t % kDecStages;
-    const bool ok = tc::mbar_wait(&full[s], (t / kDecStages) & 1, abort_flag);
-    if (__syncthreads_or(!ok)) break;  // every thread leaves together
-    const uint8_t* kt = stages + (size_t)s * L::kStageBytes;
-    const uint8_t* vt = kt + L::kMatBytes;
-    const int nvalid = (int)std::min<int64_t>(kT, e1 - (e0 + (int64_t)t * kT));
-
-    // ---- logits (log2 domain), entry-major P[j][h]
-    {
-      float2 acc[KG];
+  for (int h = 0; h < KG; ++h) {
+    m_w[h] = -INFINITY;
+    l_w[h] = 0.f;
 #pragma unroll
-      for (int h = 0; h < KG; ++h) acc[h] = make_float2(0.f, 0.f);
-      if (lj < nvalid) {
+    for (int u = 0; u < kDP; ++u) o[h][u] = make_float2(0.f, 0.f);
+  }
+  float* pme = pw + warp * kPerWarp * (4 * kKG4);  // this warp's p block, rows padded to float4
+  const int oe = kDL * lane, ocb = oe / 64, oe64 = oe % 64;
+
+  int issued = 0;  // producer lane
+  if (warp == kDecThreads / 32) {
+    // ---- producer: the first stages at once, then each stage again as soon
+    // as all compute warps have released it
+    if (lane == 0) {
+      for (; issued < ntiles; ++issued) {
+        const int s = issued % kDecStages;
+        if (issued >= kDecStages && !tc::mbar_wait(&empty[s], ((issued / kDecStages) - 1) & 1, abort_flag)) break;
+        issue(issued);
+      }
+    }
+  } else {
+    // q as fp32, each head's D values in four quarters of D/4, every quarter
+    // padded by 4 floats: the four lanes of an entry read their quarters at
+    // different shared-memory banks (the stage loads are already in flight)
+    for (int i = tid; i < KG * D; i += kDecThreads) {
+      const int h = i / D, e = i % D;
+      qs[h * kQRow + (e / kQuarter) * (kQuarter + 4) + e % kQuarter] =
+          h < G ? __uint_as_float((uint32_t)a.q[(int64_t)(g * G + h) * a.q_sh + e] << 16) : 0.f;
+    }
+    tc::named_bar_sync(1, kDecThreads);
+    for (int t = 0; t < ntiles; ++t) {
+      const int s = t % kDecStages;
+      if (!tc::mbar_wait(&full[s], (t / kDecStages) & 1, abort_flag)) break;
+      const uint8_t* kt = stages + (size_t)s * L::kStageBytes;
+      const uint8_t* vt = kt + L::kMatBytes;
+      const int nvalid = (int)std::min<int64_t>(kT, e1 - (e0 + (int64_t)t * kT));
+      const int jw = warp * kPerWarp;                       // the warp's first entry of the tile
+      const int nw = max(0, min(kPerWarp, nvalid - jw));    // of which valid
+      const int j = jw + je;
+
+      // ---- logits of the warp's entries (log2 domain)
+      float sc[KG];
+      {
+        float2 acc[KG];
+#pragma unroll
+        for (int h = 0; h < KG; ++h) acc[h] = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c = 0; c < kQChunks; ++c) {
-          const int col = lq * kQuarter + c * 8;  // first dimension of this chunk
-          const int cb = col / 64, k16 = (col % 64) / 8;
-          const uint4 kw = *reinterpret_cast<const uint4*>(kt + cb * kT * 128 + sw128(lj, k16));
+          const int col = lq * kQuarter + c * 8;
+          const uint4 kw = *reinterpret_cast<const uint4*>(kt + (col / 64) * kT * 128 + sw128(j, (col % 64) / 8));
           const float2 k0 = bf16x2_to_f2(kw.x), k1 = bf16x2_to_f2(kw.y), k2 = bf16x2_to_f2(kw.z),
                        k3 = bf16x2_to_f2(kw.w);
 #pragma unroll
@@ -180,117 +212,169 @@ decode_partial_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             acc[h] = tc::fma2(k3, make_float2(q1.z, q1.w), u);
           }
         }
+#pragma unroll
+        for (int h = 0; h < KG; ++h) {
+          float v = acc[h].x + acc[h].y;
+          v += __shfl_xor_sync(0xffffffffu, v, 1);
+          v += __shfl_xor_sync(0xffffffffu, v, 2);
+          sc[h] = je < nw ? v * a.c : -INFINITY;
+        }
       }
+      // ---- online softmax per head over the warp's entries
 #pragma unroll
       for (int h = 0; h < KG; ++h) {
-        float v = acc[h].x + acc[h].y;
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        if (lq == 0) P[lj * KG + h] = lj < nvalid ? v * a.c : -INFINITY;
+        float mx = sc[h];
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+        const float m_new = fmaxf(m_w[h], mx);
+        const float al = m_w[h] == -INFINITY ? 0.f : tc::ex2_approx(m_w[h] - m_new);
+        const float p = m_new == -INFINITY ? 0.f : tc::ex2_approx(sc[h] - m_new);
+        float ps = p;
+        ps += __shfl_xor_sync(0xffffffffu, ps, 4);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 8);
+        ps += __shfl_xor_sync(0xffffffffu, ps, 16);
+        l_w[h] = l_w[h] * al + ps;
+        m_w[h] = m_new;
+#pragma unroll
+        for (int u = 0; u < kDP; ++u) o[h][u] = make_float2(o[h][u].x * al, o[h][u].y * al);
+        if (lq == 0) pme[je * (4 * kKG4) + h] = p;
       }
+      __syncwarp();
+      // ---- the warp's output dims: o_h += sum over its entries of p_jh v_j
+      const uint8_t* vrow = vt + ocb * kT * 128 + (oe64 & 7) * 2;
+#pragma unroll 2
+      for (int q = 0; q < nw; ++q) {
+        const int jj = jw + q;
+        float2 v[kDP];
+        if constexpr (kDP == 2) {
+          const uint2 w = *reinterpret_cast<const uint2*>(vrow + sw128(jj, oe64 >> 3));
+          v[0] = bf16x2_to_f2(w.x);
+          v[1] = bf16x2_to_f2(w.y);
+        } else {
+          v[0] = bf16x2_to_f2(*reinterpret_cast<const uint32_t*>(vrow + sw128(jj, oe64 >> 3)));
+        }
+        float pv[4 * kKG4];
+#pragma unroll
+        for (int b = 0; b < kKG4; ++b) {
+          const float4 p4 = *reinterpret_cast<const float4*>(pme + q * (4 * kKG4) + 4 * b);
+          pv[4 * b] = p4.x;
+          pv[4 * b + 1] = p4.y;
+          pv[4 * b + 2] = p4.z;
+          pv[4 * b + 3] = p4.w;
+        }
+#pragma unroll
+        for (int h = 0; h < KG; ++h)
+#pragma unroll
+          for (int u = 0; u < kDP; ++u) o[h][u] = tc::fma2(v[u], make_float2(pv[h], pv[h]), o[h][u]);
+      }
+      __syncwarp();  // every lane is done with the stage and p block
+      if (lane == 0) tc::mbar_arrive(&empty[s]);
     }
-    __syncthreads();
-
-    // ---- online softmax per head: one warp per head
-    for (int h = warp; h < G; h += kDecThreads / 32) {
-      const float x0 = P[lane * KG + h], x1 = P[(lane + 32) * KG + h];
-      float mx = fmaxf(x0, x1);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      const float m_old = m_run[h];
-      const float m_new = fmaxf(m_old, mx);
-      float p0 = 0.f, p1 = 0.f;
-      if (m_new != -INFINITY) {
-        p0 = tc::ex2_approx(x0 - m_new);
-        p1 = tc::ex2_approx(x1 - m_new);
-      }
-      P[lane * KG + h] = p0;
-      P[(lane + 32) * KG + h] = p1;
-      float sum = p0 + p1;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      if (lane == 0) {
-        const float al = (m_old == -INFINITY) ? 0.f : tc::ex2_approx(m_old - m_new);
-        l_run[h] = l_run[h] * al + sum;
-        m_run[h] = m_new;
-        alpha[h] = al;
-      }
-    }
-    __syncthreads();
-
-    // ---- output rows: o_h <- alpha_h * o_h + sum_j p_hj v_j (this thread's
-    // two dimensions, its group of entries; masked entries have p = 0, and
-    // their V rows are real data or TMA zero fill)
-    {
-#pragma unroll
-      for (int h = 0; h < KG; ++h) {
-        const float al = h < G ? alpha[h] : 0.f;
-        o[h] = make_float2(o[h].x * al, o[h].y * al);
-      }
-      const uint8_t* vcol = vt + ocb * kT * 128 + (oe64 & 7) * 2;
-      const int k16 = oe64 >> 3;
-      const int jb = og * kPerGroup, je = min(nvalid, jb + kPerGroup);
-      for (int j = jb; j < je; ++j) {
-        const float2 v = bf16x2_to_f2(*reinterpret_cast<const uint32_t*>(vcol + sw128(j, k16)));
-        const float* pj = P + j * KG;
-#pragma unroll
-        for (int h = 0; h < KG; ++h) o[h] = tc::fma2(v, make_float2(pj[h], pj[h]), o[h]);
-      }
-    }
-    __syncthreads();  // stage s and P are free
-    if (tid == 0 && issued < ntiles) issue(issued++);
-  }
-
+  }  // compute warps
+  __syncthreads();
   if (*abort_flag) {
-    if (tid == 0) {
-      // let every copy already issued land before shared memory is released
-      for (int u = t; u < issued; ++u) tc::mbar_drain(&full[u % kDecStages], (u / kDecStages) & 1);
+    if (tid == kDecThreads) {
+      // let the latest copy of every stage land before shared memory is released
+      for (int u = max(0, issued - kDecStages); u < issued; ++u)
+        tc::mbar_drain(&full[u % kDecStages], (u / kDecStages) & 1);
       set_dev_err(a.err, KVC_DEV_ERR_TIMEOUT);
     }
     return;
   }
-  // ---- this chunk's partial: sum the entry groups of every (head, pair)
-  // through shared memory (the stages are free now), then write
-  float* red = reinterpret_cast<float*>(stages);  // [kGroups][G][D]
+  // ---- merge the eight compute warps (the stages are free now)
+  float* wm = reinterpret_cast<float*>(stages);      // [warp][KG] max
+  float* wl = wm + kWarps * KG;                      // [warp][KG] sum
+  float* wo = wl + kWarps * KG;                      // [warp][KG][D] output rows
+  if (warp < kWarps) {
+    if (lane == 0)
 #pragma unroll
-  for (int h = 0; h < KG; ++h)
-    if (h < G) *reinterpret_cast<float2*>(red + ((size_t)og * G + h) * D + oe) = o[h];
-  __syncthreads();
-  for (int i = tid; i < G * D; i += kDecThreads) {
-    float sum = 0.f;
-    for (int q = 0; q < kGroups; ++q) sum += red[(size_t)q * G * D + i];
-    const int h = i / D, e = i % D;
-    a.part_o[((size_t)(g * G + h) * a.nchunks + chunk) * D + e] = sum;
+      for (int h = 0; h < KG; ++h) {
+        wm[warp * KG + h] = m_w[h];
+        wl[warp * KG + h] = l_w[h];
+      }
+#pragma unroll
+    for (int h = 0; h < KG; ++h)
+#pragma unroll
+      for (int u = 0; u < kDP; ++u) *reinterpret_cast<float2*>(wo + ((size_t)warp * KG + h) * D + oe + 2 * u) = o[h][u];
   }
-  if (tid < G) {
-    a.part_m[(size_t)(g * G + tid) * a.nchunks + chunk] = m_run[tid];
-    a.part_l[(size_t)(g * G + tid) * a.nchunks + chunk] = l_run[tid];
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kDecBlock) {
+    const int h = i / D, e = i % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[w * KG + h]);
+    float O = 0.f, Lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = wm[w * KG + h];
+      const float sc = mw == -INFINITY ? 0.f : tc::ex2_approx(mw - M);
+      O += sc * wo[((size_t)w * KG + h) * D + e];
+      Lsum += sc * wl[w * KG + h];
+    }
+    a.part_o[((size_t)(g * G + h) * a.nchunks + chunk) * D + e] = O;
+    if (e == 0) {
+      a.part_m[(size_t)(g * G + h) * a.nchunks + chunk] = M;
+      a.part_l[(size_t)(g * G + h) * a.nchunks + chunk] = Lsum;
+    }
   }
 }
 
 // Merge the chunk partials of head h: out = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+// The chunk weights are formed once (shared memory), then every thread sums
+// its dimension over the chunks with the loads of eight chunks in flight.
+constexpr int kMaxChunks = 1024;
 template <int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(const DecArgs a) {
+  __shared__ float wsh[kMaxChunks];
+  __shared__ float red[D / 32];
+  __shared__ float msh;
   pdl_wait();
-  const int h = blockIdx.x, e = threadIdx.x;
-  const float* pm = a.part_m + (size_t)h * a.nchunks;
-  const float* pl = a.part_l + (size_t)h * a.nchunks;
-  float M = -INFINITY;
-  for (int c = 0; c < a.nchunks; ++c) M = fmaxf(M, pm[c]);
-  float L = 0.f, O = 0.f;
-  for (int c = 0; c < a.nchunks; ++c) {
-    if (pm[c] == -INFINITY) continue;
-    const float w = tc::ex2_approx(pm[c] - M);
-    L += w * pl[c];
-    O += w * a.part_o[((size_t)h * a.nchunks + c) * D + e];
+  const int h = blockIdx.x, e = threadIdx.x, lane = e & 31, warp = e >> 5;
+  const int nch = a.nchunks;
+  const float* pm = a.part_m + (size_t)h * nch;
+  const float* pl = a.part_l + (size_t)h * nch;
+  float mx = -INFINITY;
+  for (int c = e; c < nch; c += D) mx = fmaxf(mx, pm[c]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  if (e == 0) {
+    float m = red[0];
+    for (int w = 1; w < D / 32; ++w) m = fmaxf(m, red[w]);
+    msh = m;
   }
-  a.out[(size_t)h * D + e] = O / L;
+  __syncthreads();
+  const float M = msh;
+  float lsum = 0.f;
+  for (int c = e; c < nch; c += D) {
+    const float w = pm[c] == -INFINITY ? 0.f : tc::ex2_approx(pm[c] - M);
+    wsh[c] = w;
+    lsum += w * pl[c];
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+  __syncthreads();  // wsh complete; red reused below
+  if (lane == 0) red[warp] = lsum;
+  __syncthreads();
+  float L = 0.f;
+  for (int w = 0; w < D / 32; ++w) L += red[w];
+  const float* po = a.part_o + (size_t)h * nch * D + e;
+  float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  int c = 0;
+  for (; c + 8 <= nch; c += 8) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) o[u] += wsh[c + u] * po[(size_t)(c + u) * D];
+  }
+  for (; c < nch; ++c) o[0] += wsh[c] * po[(size_t)c * D];
+  a.out[(size_t)h * D + e] = (((o[0] + o[1]) + (o[2] + o[3])) + ((o[4] + o[5]) + (o[6] + o[7]))) / L;
 }
 
 // Chunks per KV head: about two CTAs per SM in all, never more than one per tile.
 int decode_chunks(int64_t kk, int Hkv) {
   const int64_t tiles = (kk + kT - 1) / kT;
-  const int64_t want = std::max<int64_t>(1, kDecCtaTarget / Hkv);
+  const int64_t want = std::min<int64_t>(kMaxChunks, std::max<int64_t>(1, kDecCtaTarget / Hkv));
   const int64_t per = (tiles + std::min(tiles, want) - 1) / std::min(tiles, want);  // tiles per chunk
   return (int)((tiles + per - 1) / per);
 }
@@ -418,7 +502,7 @@ extern "C" kvc_status kvc_decode_attention(const uint16_t* q, int64_t q_stride_h
   const cudaStream_t st = (cudaStream_t)stream;
   {
     const size_t smem = d == 128 ? DecSmem<128>::kBytes : DecSmem<64>::kBytes;
-    const Launch l(dim3((unsigned)a.nchunks, (unsigned)Hkv), dim3(kDecThreads), smem, st);
+    const Launch l(dim3((unsigned)a.nchunks, (unsigned)Hkv), dim3(kDecBlock), smem, st);
     s = d == 128 ? launch_decode<128>(l, kg, maps, a) : launch_decode<64>(l, kg, maps, a);
     if (s != KVC_OK) return s;
   }

@@ -26,6 +26,10 @@ def test_c3_full_layer_through_layer_plan():
     plan = kvc.LayerPlan(cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden, True, "cuda",
                          pool_kernel=cfg.pool)
     out = plan.run(q, k, v, x)
+    # the same layer with the scoring call writing the head-sum row, which the TSP selection then ranks
+    plan_row = kvc.LayerPlan(cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden, True, "cuda",
+                             pool_kernel=cfg.pool, tsp_row=True)
+    out_row = plan_row.run(q, k, v, x)
     torch.cuda.synchronize()
     assert plan.dev_err.item() == 0
     res = oracle.layer(lay.q, lay.k, cfg.H, cfg.Hkv, cfg.w, cfg.scale, cfg.pool, cfg.k_kv, cfg.k_tsp)
@@ -35,8 +39,9 @@ def test_c3_full_layer_through_layer_plan():
     for g in range(cfg.Hkv):
         parity.assert_selection_matches(idx[g], res.idx_kv[g], res.pooled[g], cfg.N, cfg.w, cfg.k_kv,
                                         what=f"c3 head {g}")
-    parity.assert_scores_close(out.tsp[0].cpu().numpy(), res.T, what="c3 head-sum row")
+    parity.assert_scores_close(out_row.tsp[0].cpu().numpy(), res.T, what="c3 head-sum row")
     it = out.idx_tsp[0].cpu().numpy()
+    assert np.array_equal(it, out_row.idx_tsp[0].cpu().numpy()), "TSP set: summed on the fly vs the head-sum row"
     parity.assert_selection_matches(it, res.idx_tsp, res.pooled_tsp, cfg.N, cfg.w, cfg.k_tsp, what="c3 TSP set")
 
     kc, vc = host_bits(out.k_c), host_bits(out.v_c)

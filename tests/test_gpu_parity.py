@@ -607,25 +607,33 @@ def test_varlen_select_rejects_sequences_longer_than_max_seqlen():
 
 
 def test_layer_plan_matches_the_single_calls():
-    """LayerPlan ranks the TSP set on the head-sum row that scoring writes;
-    that row sums the heads in the same order and precision as the grouped
-    selection, so both index sets are identical.  The K/V chain runs on a
-    side stream; its results equal the direct calls."""
+    """LayerPlan ranks the TSP set either by summing the KV-head score rows
+    inside the selection or on the head-sum row that scoring writes
+    (tsp_row=True); both sum the heads in the same order and precision, so
+    the index sets are identical.  The K/V chain runs on a side stream; its
+    results equal the direct calls."""
     cfg = workloads.shrink(workloads.C3, N=20000, k_kv=2000, k_tsp=4000, hidden=512)
     lay = workloads.make_layer(cfg)
     q, kd, vd, xd = dev_bf16(lay.q), dev_bf16(lay.k), dev_bf16(lay.v), dev_bf16(lay.x)
     plan = kvc.LayerPlan(cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden, True, "cuda",
                          pool_kernel=cfg.pool)
     out = plan.run(q, kd, vd, xd)
+    plan_row = kvc.LayerPlan(cfg.N, cfg.H, cfg.Hkv, cfg.d, cfg.w, cfg.k_kv, cfg.k_tsp, cfg.hidden, True, "cuda",
+                             pool_kernel=cfg.pool, tsp_row=True)
+    out_row = plan_row.run(q, kd, vd, xd)
     torch.cuda.synchronize()
+    assert out.tsp is None
     scores = kvc.kvc_score(q, kd)
     assert torch.equal(out.scores, scores)
+    assert torch.equal(out_row.scores, scores)
     ref_tsp = scores[0].clone()
     for g in range(1, cfg.Hkv):
         ref_tsp += scores[g]
-    assert torch.equal(out.tsp[0], ref_tsp)
+    assert torch.equal(out_row.tsp[0], ref_tsp)
     it = kvc.kvc_select_topk(scores, cfg.w, cfg.pool, cfg.k_tsp, row_group=cfg.Hkv)
     assert torch.equal(out.idx_tsp, it)
+    assert torch.equal(out_row.idx_tsp, it)
+    assert torch.equal(out_row.x_c, out.x_c)
     ik = kvc.kvc_select_topk(scores, cfg.w, cfg.pool, cfg.k_kv)
     assert torch.equal(out.idx_kv, ik)
     ko, vo = kvc.kvc_gather_kv(kd, vd, ik)
