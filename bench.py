@@ -621,7 +621,7 @@ def main() -> None:
     q_dec = torch.randn(cfg.H, cfg.d, device=dev, generator=gq).to(torch.bfloat16)
     caches = [(plan.k_c, plan.v_c)] + [(plan.k_c.clone(), plan.v_c.clone()) for _ in range(3)]
     dec_out = torch.empty((cfg.H, cfg.d), dtype=torch.float32, device=dev)
-    ws_dec = torch.empty(kvc.decode_workspace_size(cfg.H, cfg.Hkv, cfg.d, cfg.k_kv), dtype=torch.uint8, device=dev)
+    ws_dec = torch.zeros(kvc.decode_workspace_size(cfg.H, cfg.Hkv, cfg.d, cfg.k_kv), dtype=torch.uint8, device=dev)
     for i in range(4):
         kvc.kvc_decode_attention(q_dec, *caches[i], out=dec_out, ws=ws_dec, dev_err=plan.dev_err, stream=st)
     torch.cuda.synchronize(dev)

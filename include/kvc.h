@@ -305,11 +305,18 @@ kvc_status kvc_decode_workspace_size(int32_t num_heads, int32_t num_kv_heads, in
  *  q        [H][d] bf16, row h at q + h * q_stride_h (q_stride_h >= d)
  *  k_c, v_c [Hkv][kk][d] bf16, contiguous (as kvc_gather_kv writes them),
  *           16-byte aligned; kk >= 1, kk * Hkv < 2^31
- *  out      [H][d] fp32, contiguous
- *  ws       kvc_decode_workspace_size(H, Hkv, d, kk) bytes, 256-B aligned
+ *  out      [H][d] fp32, contiguous, 16-byte aligned
+ *  ws       kvc_decode_workspace_size(H, Hkv, d, kk) bytes, 256-B aligned,
+ *           ZERO-FILLED before its first use: it starts with one counter per
+ *           KV head (chunks of that head done), which every call returns to
+ *           zero, also when a wait timed out; one call at a time per workspace
  *  dev_err  device int32 or NULL (KVC_DEV_ERR_TIMEOUT only)
  * head_dim in {64, 128}; at most 16 query heads per KV head.  fp32
- * arithmetic from the bf16 values; deterministic.
+ * accumulation from the bf16 values; deterministic.  At head_dim 128 with up
+ * to 8 query heads per KV head both contractions run on the tensor cores
+ * (the probabilities enter the second one as two bf16 terms, hi + lo, good
+ * to ~2^-17 of each) in one launch; otherwise on the CUDA cores, with a
+ * second launch that merges the chunk partials.
  */
 kvc_status kvc_decode_attention(const uint16_t* q, int64_t q_stride_h, const uint16_t* k_c, const uint16_t* v_c,
                                 int64_t kk, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, float scale,

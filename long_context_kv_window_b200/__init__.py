@@ -503,7 +503,8 @@ def kvc_decode_attention(q: torch.Tensor, k_c: torch.Tensor, v_c: torch.Tensor, 
                          out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
                          dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """One decode query per head, q [H][d], over the compacted cache
-    k_c, v_c [Hkv][kk][d] (every retained entry visible); returns fp32 [H][d]."""
+    k_c, v_c [Hkv][kk][d] (every retained entry visible); returns fp32 [H][d].
+    A caller's ws must have been zero-filled once (the call leaves it so)."""
     _bf16(q, "q", 2)
     _bf16(k_c, "k_c", 3)
     _bf16(v_c, "v_c", 3)
@@ -519,8 +520,8 @@ def kvc_decode_attention(q: torch.Tensor, k_c: torch.Tensor, v_c: torch.Tensor, 
         out = torch.empty((H, d), dtype=torch.float32, device=dev)
     _dense(out, "out", (H, d), torch.float32, dev)
     _err_word(dev_err, dev)
-    if ws is None:
-        ws = _workspace(decode_workspace_size(H, Hkv, d, kk), dev)
+    if ws is None:  # starts with per-KV-head counters, which must be zero before the first call
+        ws = torch.zeros(max(decode_workspace_size(H, Hkv, d, kk), 1), dtype=torch.uint8, device=dev)
     sc = float(1.0 / math.sqrt(d) if scale is None else scale)
     _check(_call(dev, lib().kvc_decode_attention, _ptr(q), q.stride(0), _ptr(k_c), _ptr(v_c), kk, H, Hkv, d, sc,
                  _ptr(out), _ptr(ws), _ws_bytes(ws, dev), _ptr(dev_err), _stream(stream, dev)),

@@ -26,6 +26,8 @@
 
 #include <algorithm>
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "tc.cuh"
 
@@ -51,6 +53,7 @@ struct DecArgs {
   float* part_m;      // [H][nchunks]: running max (log2 domain)
   float* part_l;      // [H][nchunks]: sum of 2^(s*c - max)
   float* part_o;      // [H][nchunks][d]: sum of 2^(s*c - max) * v
+  uint32_t* cnt;      // [Hkv]: chunks of the KV head done (tensor-core kernel; zero between calls)
   float* out;         // [H][d]
   int32_t* err;
 };
@@ -320,6 +323,422 @@ decode_partial_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
   }
 }
 
+// --------------------------------------------------------------------------
+// tcgen05 variant (head_dim 128, up to 8 query heads per KV head).  The two
+// contractions of a 128-entry tile run on the tensor cores, so the CUDA cores
+// only form the probabilities and the stream of Kc / Vc sets the pace:
+//   logits  S[entry][h] = Kc_tile (M = 128 entries, K = d) x q^T (N = 16: the
+//           group's heads, zero rows past G), fp32 in TMEM;
+//   output  O[dim][n]   = Vc_tile^T (M = d = 128, K = entries; the TMA tile of
+//           Vc read as an MN-major operand) x P (N = 16, K = entries), where
+//           P rows 0..7 hold bf16(p_h) and rows 8..15 the bf16 rounding
+//           residual p_h - bf16(p_h), so hi + lo carries p_h to ~2^-17.
+// Each epilogue warp owns 32 entries of a tile and a running reference per
+// head (the max logit its entries have shown, log2 domain), so no barrier
+// joins the warps inside the loop; the output MMA of a tile is split into the
+// four warps' 32-entry slices, each into its own TMEM accumulator, and every
+// epilogue thread (one output dimension) folds the four slices into its
+// registers with the four references.
+// Kc and Vc tiles stream through two rings: a Kc tile is released as soon as
+// its logits MMA has read it, a Vc tile only after the output MMA, which
+// waits for the probabilities.
+// Warp roles: 0 Kc producer, 1 TMEM allocator + MMA issuer, 2..5 epilogue
+// (TMEM lane quarter = warp & 3), 6 Vc producer.
+// --------------------------------------------------------------------------
+constexpr int kTcT = 128;        // entries per tile (MMA M of the logits)
+constexpr int kTcKStages = 1;    // 32 KB Kc tiles (held only until the logits MMA)
+constexpr int kTcVStages = 2;    // 32 KB Vc tiles (held until the output MMA)
+constexpr int kTcCtasPerSm = 2;  // 110 KB of shared memory and 256 TMEM columns each
+constexpr float kTcSlack = 8.f;  // log2 units a logit may pass a warp's reference by
+constexpr int kTcMaxG = 8;
+constexpr int kTcBlock = 224;
+constexpr uint32_t kTcCols = 256;  // S: 2 x 16 columns, O: 2 buffers x 4 slices x 16
+constexpr uint32_t kTcO = 32;      // first O column
+
+struct TcSmem {
+  static constexpr int kTile = kTcT * 128;           // one 64-column block of a tile (16 KB)
+  static constexpr int kStage = 2 * kTile;           // a Kc or a Vc tile (two column blocks)
+  static constexpr int kQ = 2 * 16 * 128;            // q: 2 column blocks x 16 rows x 128 B
+  static constexpr int kP = 2 * 16 * 128;            // one P buffer: 2 entry blocks x 16 rows x 128 B
+  static constexpr int kVOff = kTcKStages * kStage;  // the Vc ring follows the Kc ring
+  static constexpr int kQOff = kVOff + kTcVStages * kStage;
+  static constexpr int kPOff = kQOff + kQ;
+  static constexpr int kBarOff = kPOff + 2 * kP;
+  static constexpr size_t kBytes = 1024 + (size_t)kBarOff + 1024;
+};
+
+struct TcBars {
+  uint64_t kfull[kTcKStages], kempty[kTcKStages], vfull[kTcVStages], vempty[kTcVStages];
+  uint64_t s_full[2], s_empty[2], p_full[2], o_full[2], o_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+  int last;  // this CTA took the KV head's last ticket: it merges the partials
+  // reference each warp used for the P rows of tile t, at [t & 3]: a warp can
+  // run at most two tiles ahead of the slowest one (the logits buffer of tile
+  // t + 2 is released only once every warp has read tile t's), so a slot is
+  // rewritten only after every warp has folded the tile it belonged to
+  float mref[4][4][kTcMaxG];
+  float wm[4][kTcMaxG], wl[4][kTcMaxG];
+};
+
+// Byte offset of bf16 element (row r, column k) in a K-major operand stored
+// as 64-column blocks of `rows` rows x 128 B with the 128-byte swizzle.
+__device__ __forceinline__ int kmaj_off(int r, int k, int rows) {
+  return (k >> 6) * rows * 128 + r * 128 + ((((k & 63) >> 3) ^ (r & 7)) << 4) + ((k & 7) << 1);
+}
+
+// MN-major operand descriptor, 128-byte swizzle: 64 MN-consecutive elements per
+// 128-byte row, K rows at 128 B; `lbo` bytes between 64-element MN blocks,
+// 1024 B between 8-row K groups.
+__device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t smem_addr, uint32_t lbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr & 0x3FFFFu) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)2 << 61;
+  return d;
+}
+
+template <int KG>
+__global__ void __launch_bounds__(kTcBlock, kTcCtasPerSm)
+decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+                 const DecArgs a) {
+  using L = TcSmem;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* qb = sm + L::kQOff;
+  uint8_t* pb = sm + L::kPOff;
+  TcBars* bars = reinterpret_cast<TcBars*>(sm + L::kBarOff);
+  static_assert(sizeof(TcBars) <= 1024, "barrier block");
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g = blockIdx.y, chunk = blockIdx.x;
+  const int G = a.G;
+  const int64_t e0 = (int64_t)chunk * a.chunk;
+  const int64_t e1 = std::min<int64_t>(a.kk, e0 + a.chunk);
+  const int ntiles = (int)((e1 - e0 + kTcT - 1) / kTcT);
+  const int64_t row0 = (int64_t)g * a.kk + e0;
+
+  if (tid == 0) {
+    for (int s = 0; s < kTcKStages; ++s) {
+      tc::mbar_init(&bars->kfull[s], 1);
+      tc::mbar_init(&bars->kempty[s], 1);
+    }
+    for (int s = 0; s < kTcVStages; ++s) {
+      tc::mbar_init(&bars->vfull[s], 1);
+      tc::mbar_init(&bars->vempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&bars->s_full[b], 1);
+      tc::mbar_init(&bars->s_empty[b], 4);
+      tc::mbar_init(&bars->p_full[b], 4);
+      tc::mbar_init(&bars->o_full[b], 1);
+      tc::mbar_init(&bars->o_empty[b], 4);
+    }
+    tc::mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) tc::prefetch_tmap(&kmap);
+  if (warp == 6 && lane == 0) tc::prefetch_tmap(&vmap);
+  if (warp == 1) {
+    tc::tmem_alloc(&bars->tmem_base, kTcCols);
+    tc::tmem_relinquish();
+  }
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  pdl_wait();  // Kc / Vc / q may come from the previous kernel of the stream
+  pdl_trigger();
+  if (warp >= 1 && warp <= 5) {
+    // while the producers start the streams: both P buffers zero (rows past
+    // the group stay zero), and q of the group as the logits' B operand
+    // (rows = heads, zero past G; K = d)
+    constexpr int kN = 160;
+    for (int i = tid - 32; i < 2 * L::kP / 16; i += kN) reinterpret_cast<uint4*>(pb)[i] = make_uint4(0u, 0u, 0u, 0u);
+    for (int i = tid - 32; i < 16 * 128; i += kN) {
+      const int h = i >> 7, k = i & 127;
+      const uint16_t v = h < G ? a.q[(int64_t)(g * G + h) * a.q_sh + k] : (uint16_t)0;
+      *reinterpret_cast<uint16_t*>(qb + kmaj_off(h, k, 16)) = v;
+    }
+    tc::fence_proxy_async_smem();
+    tc::named_bar_sync(1, kN);
+  }
+  const uint32_t tmem = bars->tmem_base;
+  volatile int* abort_flag = &bars->abort;
+  float o_r[KG];  // epilogue: this thread's output dimension per head (relative to m_acc)
+#pragma unroll
+  for (int h = 0; h < KG; ++h) o_r[h] = 0.f;
+
+  if (warp == 0 || warp == 6) {
+    // ---- TMA producers: warp 0 the Kc tiles, warp 6 the Vc tiles
+    if (lane == 0) {
+      const bool is_k = warp == 0;
+      const int ns = is_k ? kTcKStages : kTcVStages;
+      uint64_t* fullb = is_k ? bars->kfull : bars->vfull;
+      uint64_t* emptyb = is_k ? bars->kempty : bars->vempty;
+      uint8_t* ring = sm + (is_k ? 0 : L::kVOff);
+      const CUtensorMap* map = is_k ? &kmap : &vmap;
+      int issued = 0;
+      for (int t = 0; t < ntiles; ++t) {
+        const int s = t % ns;
+        if (t >= ns && !tc::mbar_wait(&emptyb[s], ((t / ns) - 1) & 1, abort_flag)) break;
+        tc::mbar_arrive_expect_tx(&fullb[s], (uint32_t)L::kStage);
+        uint8_t* dst = ring + (size_t)s * L::kStage;
+        const int y = (int)(row0 + (int64_t)t * kTcT);
+        tc::tma_load_2d(dst, map, &fullb[s], 0, y);
+        tc::tma_load_2d(dst + L::kTile, map, &fullb[s], 64, y);
+        issued = t + 1;
+      }
+      if (*abort_flag)
+        for (int t = std::max(0, issued - ns); t < issued; ++t) tc::mbar_drain(&fullb[t % ns], (t / ns) & 1);
+    }
+  } else if (warp == 1) {
+    // ---- MMA issuer: logits of tile t, then the output of tile t - 1
+    if (lane == 0) {
+      const uint32_t id_s = tc::idesc_bf16_f32(128, 16);
+      const uint32_t id_o = tc::idesc_bf16_f32(128, 16) | (1u << 15);  // A (Vc^T) MN-major
+      const uint64_t q_desc = tc::desc_k_sw128(tc::smem_u32(qb));
+      const uint64_t k_desc = tc::desc_k_sw128(tc::smem_u32(sm));
+      const uint64_t v_desc = desc_mn_sw128(tc::smem_u32(sm + L::kVOff), (uint32_t)L::kTile);
+      const uint64_t p_desc = tc::desc_k_sw128(tc::smem_u32(pb));
+      auto logits = [&](int t) -> bool {
+        const int s = t % kTcKStages, b = t & 1;
+        if (!tc::mbar_wait(&bars->kfull[s], (t / kTcKStages) & 1, abort_flag)) return false;
+        if (t >= 2 && !tc::mbar_wait(&bars->s_empty[b], ((t >> 1) - 1) & 1, abort_flag)) return false;
+        tc::tc_fence_after();
+        const uint64_t kd = k_desc + (uint64_t)(((uint32_t)s * L::kStage) >> 4);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = (uint32_t)((ks >> 2) * L::kTile + (ks & 3) * 32) >> 4;  // K tile: 64-col block, 32 B step
+          const uint32_t qoff = (uint32_t)((ks >> 2) * 2048 + (ks & 3) * 32) >> 4;    // q: 16-row blocks of 2 KB
+          tc::mma_bf16(tmem + (uint32_t)(16 * b), kd + off, q_desc + qoff, id_s, ks != 0);
+        }
+        tc::mma_commit(&bars->s_full[b]);
+        tc::mma_commit(&bars->kempty[s]);  // the Kc tile is read
+        return true;
+      };
+      auto output = [&](int t) -> bool {
+        const int s = t % kTcVStages, b = t & 1;
+        if (!tc::mbar_wait(&bars->vfull[s], (t / kTcVStages) & 1, abort_flag)) return false;
+        if (!tc::mbar_wait(&bars->p_full[b], (t >> 1) & 1, abort_flag)) return false;
+        if (t >= 2 && !tc::mbar_wait(&bars->o_empty[b], ((t >> 1) - 1) & 1, abort_flag)) return false;
+        tc::tc_fence_after();
+        const uint64_t vd = v_desc + (uint64_t)(((uint32_t)s * L::kStage) >> 4);
+        const uint64_t pd = p_desc + (uint64_t)(((uint32_t)b * L::kP) >> 4);
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const int en = 32 * w + 16 * j;  // first entry of this K step
+            const uint32_t voff = (uint32_t)(en * 128) >> 4;                          // 16 Vc rows = 2 KB
+            const uint32_t poff = (uint32_t)((en >> 6) * 2048 + (en & 63) * 2) >> 4;  // P: 64-entry blocks
+            tc::mma_bf16(tmem + kTcO + (uint32_t)(64 * b + 16 * w), vd + voff, pd + poff, id_o, j != 0);
+          }
+        tc::mma_commit(&bars->o_full[b]);
+        tc::mma_commit(&bars->vempty[s]);  // the Vc tile is read
+        return true;
+      };
+      bool ok = true;
+      for (int t = 0; ok && t <= ntiles; ++t) {
+        if (t < ntiles) ok = logits(t);
+        if (ok && t >= 1) ok = output(t - 1);
+      }
+      tc::mma_commit(&bars->mma_done);  // every MMA issued above has completed before TMEM is freed
+      tc::mbar_drain(&bars->mma_done, 0);
+    }
+  } else {
+    // ---- epilogue: warp quarter wq owns entries 32 wq .. 32 wq + 31 of each
+    // tile (softmax role) and output dimension 32 wq + lane (output role)
+    const int wq = warp & 3;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * wq) << 16);
+    float m_w[KG], l_t[KG], m_acc[KG];
+#pragma unroll
+    for (int h = 0; h < KG; ++h) {
+      m_w[h] = -INFINITY;
+      l_t[h] = 0.f;
+      m_acc[h] = -INFINITY;
+    }
+    bool ok = true;
+    for (int t = 0; ok && t <= ntiles; ++t) {
+      if (t < ntiles) {
+        const int b = t & 1;
+        if (!tc::mbar_wait(&bars->s_full[b], (t >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc::tc_fence_after();
+        uint32_t x[32];
+        KVC_TMEM_LD16(lane_base + (uint32_t)(16 * b), x);
+        KVC_TMEM_WAIT_LD32(x);
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->s_empty[b]);
+        const int ent = 32 * wq + lane;
+        const bool valid = (int64_t)t * kTcT + ent < e1 - e0;
+        uint8_t* pbb = pb + b * L::kP;
+#pragma unroll
+        for (int h = 0; h < KG; ++h) {
+          const float sv = valid && h < G ? __uint_as_float(x[h]) * a.c : -INFINITY;
+          // the reference moves (to the warp's max) only when a logit passes it
+          // by more than kTcSlack: p <= 2^kTcSlack otherwise, which bf16 and the
+          // fp32 sums carry exactly as well as p <= 1 (warp-uniform vote)
+          if (__any_sync(0xffffffffu, sv > m_w[h] + kTcSlack)) {
+            float mx = sv;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            l_t[h] *= m_w[h] == -INFINITY ? 0.f : tc::ex2_approx(m_w[h] - mx);
+            m_w[h] = mx;
+          }
+          const float p = m_w[h] == -INFINITY ? 0.f : tc::ex2_approx(sv - m_w[h]);
+          l_t[h] += p;
+          const __nv_bfloat16 hi = __float2bfloat16_rn(p);
+          const __nv_bfloat16 lo = __float2bfloat16_rn(p - __bfloat162float(hi));
+          if (h < G) {
+            *reinterpret_cast<__nv_bfloat16*>(pbb + kmaj_off(h, ent, 16)) = hi;
+            *reinterpret_cast<__nv_bfloat16*>(pbb + kmaj_off(8 + h, ent, 16)) = lo;
+          }
+          if (lane == 0) bars->mref[t & 3][wq][h] = m_w[h];
+        }
+        tc::fence_proxy_async_smem();  // P visible to the tensor core
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->p_full[b]);
+      }
+      if (t >= 1) {
+        // fold the output slices of tile t - 1 into this thread's dimension
+        const int tp = t - 1, b = tp & 1;
+        // the slices' references: written by each warp before its P arrival
+        if (!tc::mbar_wait(&bars->p_full[b], (tp >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!tc::mbar_wait(&bars->o_full[b], (tp >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc::tc_fence_after();
+        uint32_t y[64];
+        KVC_TMEM_LD64(lane_base + kTcO + (uint32_t)(64 * b), y);
+        KVC_TMEM_WAIT_LD64(y);
+        tc::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bars->o_empty[b]);
+#pragma unroll
+        for (int h = 0; h < KG; ++h) {
+          if (h >= G) continue;
+          float mr[4], mt = m_acc[h];
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            mr[w] = bars->mref[tp & 3][w][h];
+            mt = fmaxf(mt, mr[w]);
+          }
+          if (mt == -INFINITY) continue;
+          float acc = m_acc[h] == -INFINITY ? 0.f : o_r[h] * tc::ex2_approx(m_acc[h] - mt);
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            if (mr[w] != -INFINITY)
+              acc += (__uint_as_float(y[16 * w + h]) + __uint_as_float(y[16 * w + 8 + h])) * tc::ex2_approx(mr[w] - mt);
+          o_r[h] = acc;
+          m_acc[h] = mt;
+        }
+      }
+    }
+    if (ok) {
+      // this warp's (reference, sum) per head for the CTA merge
+#pragma unroll
+      for (int h = 0; h < KG; ++h) {
+        float l = l_t[h];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+        if (lane == 0) {
+          bars->wm[wq][h] = m_w[h];
+          bars->wl[wq][h] = l;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (*abort_flag) {
+    if (tid == 0) set_dev_err(a.err, KVC_DEV_ERR_TIMEOUT);
+  } else if (warp >= 2 && warp <= 5) {
+    const int wq = warp & 3;
+    const int dim = 32 * wq + lane;
+#pragma unroll
+    for (int h = 0; h < KG; ++h) {
+      if (h >= G) break;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) M = fmaxf(M, bars->wm[w][h]);
+      float Lsum = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w)
+        if (bars->wm[w][h] != -INFINITY) Lsum += bars->wl[w][h] * tc::ex2_approx(bars->wm[w][h] - M);
+      const size_t slot = (size_t)(g * G + h) * a.nchunks + chunk;
+      a.part_o[slot * 128 + dim] = o_r[h];
+      if (dim == 0) {
+        a.part_m[slot] = M;
+        a.part_l[slot] = Lsum;
+      }
+    }
+  }
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, kTcCols);
+  }
+  // ---- the last CTA of the KV head to finish merges the chunk partials of
+  // its G heads (out_h = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c).  A CTA
+  // that gave up on a wait still takes its ticket, so the counter always
+  // returns to zero (the output is then flagged by the timeout bit).
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) bars->last = atomicAdd(&a.cnt[g], 1u) == (uint32_t)(a.nchunks - 1);
+  __syncthreads();
+  if (!bars->last) return;
+  __threadfence();
+  // chunk weights 2^(m_c - M) and the normaliser per head (one warp per head),
+  // in the stage memory, which no copy or MMA uses any more
+  const int nch = a.nchunks;
+  float* wv = reinterpret_cast<float*>(sm);  // [G][nch]
+  float* lv = wv + G * nch;                  // [G]
+  for (int hl = warp; hl < G; hl += kTcBlock / 32) {
+    const float* pm = a.part_m + (size_t)(g * G + hl) * nch;
+    const float* pl = a.part_l + (size_t)(g * G + hl) * nch;
+    float M = -INFINITY;
+    for (int c = lane; c < nch; c += 32) M = fmaxf(M, __ldcg(pm + c));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float Ls = 0.f;
+    for (int c = lane; c < nch; c += 32) {
+      const float mc = __ldcg(pm + c);
+      const float wc = mc == -INFINITY ? 0.f : tc::ex2_approx(mc - M);
+      wv[hl * nch + c] = wc;
+      Ls += wc * __ldcg(pl + c);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
+    if (lane == 0) lv[hl] = Ls;
+  }
+  __syncthreads();
+  // every thread sums four consecutive dimensions of one head over the chunks,
+  // sixteen 16-byte loads in flight
+  for (int i = tid; i < G * 32; i += kTcBlock) {
+    const int hl = i >> 5, d4 = (i & 31) * 4;
+    const float4* po = reinterpret_cast<const float4*>(a.part_o + (size_t)(g * G + hl) * nch * 128 + d4);
+    const float* wh = wv + hl * nch;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < nch; c0 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = c0 + u < nch ? __ldcg(po + (size_t)(c0 + u) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const float wc = c0 + u < nch ? wh[c0 + u] : 0.f;
+        acc.x += wc * v[u].x;
+        acc.y += wc * v[u].y;
+        acc.z += wc * v[u].z;
+        acc.w += wc * v[u].w;
+      }
+    }
+    const float ls = lv[hl];
+    *reinterpret_cast<float4*>(a.out + (size_t)(g * G + hl) * 128 + d4) =
+        make_float4(acc.x / ls, acc.y / ls, acc.z / ls, acc.w / ls);
+  }
+  if (tid == 0) a.cnt[g] = 0u;
+}
+
 // Merge the chunk partials of head h: out = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
 // The chunk weights are formed once (shared memory), then every thread sums
 // its dimension over the chunks with the loads of eight chunks in flight.
@@ -371,10 +790,20 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(const DecArgs a) {
   a.out[(size_t)h * D + e] = (((o[0] + o[1]) + (o[2] + o[3])) + ((o[4] + o[5]) + (o[6] + o[7]))) / L;
 }
 
-// Chunks per KV head: about two CTAs per SM in all, never more than one per tile.
-int decode_chunks(int64_t kk, int Hkv) {
-  const int64_t tiles = (kk + kT - 1) / kT;
-  const int64_t want = std::min<int64_t>(kMaxChunks, std::max<int64_t>(1, kDecCtaTarget / Hkv));
+// The tensor-core kernel serves head_dim 128 with up to 8 query heads per KV
+// head; the CUDA-core kernel everything else.
+bool decode_on_tc(int G, int d) { return d == 128 && G <= kTcMaxG; }
+
+// Entries per tile of the kernel that serves (G, d).
+int decode_tile(int G, int d) { return decode_on_tc(G, d) ? kTcT : kT; }
+
+// Chunks per KV head: about one wave of CTAs (one per SM for the tensor-core
+// kernel, two for the CUDA-core one), never more than one per tile.
+int decode_chunks(int64_t kk, int Hkv, int G, int d) {
+  const int tile = decode_tile(G, d);
+  const int target = decode_on_tc(G, d) ? kTcCtasPerSm * num_sms() : kDecCtaTarget;
+  const int64_t tiles = (kk + tile - 1) / tile;
+  const int64_t want = std::min<int64_t>(kMaxChunks, std::max<int64_t>(1, target / Hkv));
   const int64_t per = (tiles + std::min(tiles, want) - 1) / std::min(tiles, want);  // tiles per chunk
   return (int)((tiles + per - 1) / per);
 }
@@ -396,6 +825,19 @@ kvc_status launch_decode_g(const Launch& l, const CUtensorMap (&maps)[2], const 
   });
   if (s != KVC_OK) return s;
   KVC_CUDA_TRY(l.run(decode_partial_kernel<D, KG>, maps[0], maps[1], a));
+  return KVC_OK;
+}
+
+template <int KG>
+kvc_status launch_decode_tc(const Launch& l, const CUtensorMap (&maps)[2], const DecArgs& a) {
+  static ContextCache cache;
+  kvc_status s = once_per_context(cache, [] {
+    KVC_CUDA_TRY(cudaFuncSetAttribute(decode_tc_kernel<KG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)TcSmem::kBytes));
+    return KVC_OK;
+  });
+  if (s != KVC_OK) return s;
+  KVC_CUDA_TRY(l.run(decode_tc_kernel<KG>, maps[0], maps[1], a));
   return KVC_OK;
 }
 
@@ -422,8 +864,9 @@ kvc_status check_decode(int32_t H, int32_t Hkv, int32_t d, int64_t kk) {
 }
 
 size_t decode_ws_bytes(int32_t H, int32_t Hkv, int32_t d, int64_t kk) {
-  const size_t nch = (size_t)decode_chunks(kk, Hkv);
-  return round_up((size_t)H * nch * 4, kWsAlign) * 2 + round_up((size_t)H * nch * d * 4, kWsAlign);
+  const size_t nch = (size_t)decode_chunks(kk, Hkv, H / Hkv, d);
+  return round_up((size_t)Hkv * 4, kWsAlign) + round_up((size_t)H * nch * 4, kWsAlign) * 2 +
+         round_up((size_t)H * nch * d * 4, kWsAlign);
 }
 
 }  // namespace
@@ -449,7 +892,7 @@ extern "C" kvc_status kvc_decode_attention(const uint16_t* q, int64_t q_stride_h
   kvc_status s = check_decode(num_heads, num_kv_heads, head_dim, kk);
   if (s != KVC_OK) return s;
   KVC_CHECK_ARG(q && k_c && v_c && out, "q, k_c, v_c and out must be non-NULL");
-  KVC_CHECK_ARG(aligned(k_c, 16) && aligned(v_c, 16), "k_c and v_c must be 16-byte aligned");
+  KVC_CHECK_ARG(aligned(k_c, 16) && aligned(v_c, 16) && aligned(out, 16), "k_c, v_c and out must be 16-byte aligned");
   KVC_CHECK_ARG(q_stride_h >= head_dim, "q_stride_h must be >= head_dim");
   KVC_CHECK_ARG(scale > 0.f && scale < 1e30f, "scale must be positive and finite");
   const size_t need = decode_ws_bytes(num_heads, num_kv_heads, head_dim, kk);
@@ -466,13 +909,15 @@ extern "C" kvc_status kvc_decode_attention(const uint16_t* q, int64_t q_stride_h
       encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
   });
   if (!encode) return fail(KVC_ERR_CUDA, "cuTensorMapEncodeTiled is unavailable");
-  const int d = head_dim, Hkv = num_kv_heads;
+  const int d = head_dim, Hkv = num_kv_heads, G = num_heads / num_kv_heads;
+  const bool on_tc = decode_on_tc(G, d);
+  const int tile = decode_tile(G, d);
   CUtensorMap maps[2];
   const uint16_t* srcs[2] = {k_c, v_c};
   for (int i = 0; i < 2; ++i) {
     cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)(kk * Hkv)};
     cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)kT};
+    cuuint32_t box[2] = {64u, (cuuint32_t)tile};
     cuuint32_t es[2] = {1u, 1u};
     if (encode(&maps[i], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(srcs[i]), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -486,11 +931,12 @@ extern "C" kvc_status kvc_decode_attention(const uint16_t* q, int64_t q_stride_h
   a.H = num_heads;
   a.Hkv = Hkv;
   a.G = num_heads / Hkv;
-  a.nchunks = decode_chunks(kk, Hkv);
-  const int64_t tiles = (kk + kT - 1) / kT;
-  a.chunk = (int)(((tiles + a.nchunks - 1) / a.nchunks) * kT);
+  a.nchunks = decode_chunks(kk, Hkv, G, d);
+  const int64_t tiles = (kk + tile - 1) / tile;
+  a.chunk = (int)(((tiles + a.nchunks - 1) / a.nchunks) * tile);
   a.c = (float)((double)scale * kLog2e);
   WsCursor wc{static_cast<char*>(ws), ws_bytes};
+  a.cnt = wc.take<uint32_t>((size_t)Hkv);
   a.part_m = wc.take<float>((size_t)num_heads * a.nchunks);
   a.part_l = wc.take<float>((size_t)num_heads * a.nchunks);
   a.part_o = wc.take<float>((size_t)num_heads * a.nchunks * d);
@@ -500,7 +946,13 @@ extern "C" kvc_status kvc_decode_attention(const uint16_t* q, int64_t q_stride_h
 
   const int kg = decode_group_slots(a.G);
   const cudaStream_t st = (cudaStream_t)stream;
-  {
+  if (on_tc) {  // one launch: the last CTA of each KV head merges
+    const Launch l(dim3((unsigned)a.nchunks, (unsigned)Hkv), dim3(kTcBlock), TcSmem::kBytes, st);
+    s = G <= 4 ? launch_decode_tc<4>(l, maps, a) : launch_decode_tc<8>(l, maps, a);
+    if (s != KVC_OK) return s;
+    count_launch(1);
+    return KVC_OK;
+  } else {
     const size_t smem = d == 128 ? DecSmem<128>::kBytes : DecSmem<64>::kBytes;
     const Launch l(dim3((unsigned)a.nchunks, (unsigned)Hkv), dim3(kDecBlock), smem, st);
     s = d == 128 ? launch_decode<128>(l, kg, maps, a) : launch_decode<64>(l, kg, maps, a);

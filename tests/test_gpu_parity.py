@@ -448,12 +448,14 @@ def test_kv_head_split_reproduces_the_layer():
 # decode attention over the compacted cache
 # --------------------------------------------------------------------------- #
 @pytest.mark.parametrize("H,Hkv,d,kk", [(32, 8, 128, 13107), (32, 8, 128, 1), (32, 8, 128, 63), (8, 8, 64, 64),
-                                        (40, 8, 128, 4096), (16, 1, 128, 2000), (8, 2, 64, 65), (6, 3, 128, 777)])
+                                        (40, 8, 128, 4096), (16, 1, 128, 2000), (8, 2, 64, 65), (6, 3, 128, 777),
+                                        (64, 8, 128, 300), (8, 8, 128, 2305)])
 def test_decode_attention_matches_oracle(H, Hkv, d, kk):
     """One decode query per head over [Hkv][kk][d] retained entries: the
-    128K layer's 13107 entries per head, single and ragged tiles, G = 1, 5
-    and 16 query heads per KV head, head_dim 64; a few planted entries carry
-    most of the attention."""
+    128K layer's 13107 entries per head, single and ragged tiles, G = 1, 2,
+    4, 5, 8 (the tensor-core kernel) and 16 query heads per KV head and
+    head_dim 64 (the CUDA-core kernel); a few planted entries carry most of
+    the attention, so the running reference of a warp jumps mid-chunk."""
     rng = np.random.default_rng(H * 1000 + kk + d)
     q = workloads.f32_to_bf16_bits(rng.standard_normal((H, d)).astype(np.float32))
     kc = workloads.f32_to_bf16_bits(rng.standard_normal((Hkv, kk, d)).astype(np.float32))
@@ -471,6 +473,27 @@ def test_decode_attention_matches_oracle(H, Hkv, d, kk):
     assert err.item() == 0
     ref = oracle.get().decode_attention(q, kc, vc, H, Hkv, 1 / math.sqrt(d))
     parity.assert_decode_close(out.cpu().numpy(), ref, what=f"decode H={H} Hkv={Hkv} d={d} kk={kk}")
+
+
+def test_decode_workspace_reused_across_calls():
+    """The tensor-core decode keeps one ticket counter per KV head in its
+    workspace and returns it to zero: consecutive calls on one zero-filled
+    workspace -- different queries, then a smaller cache with fewer chunks --
+    all match the oracle."""
+    rng = np.random.default_rng(77)
+    H, Hkv, d = 32, 8, 128
+    kc = workloads.f32_to_bf16_bits(rng.standard_normal((Hkv, 5000, d)).astype(np.float32))
+    vc = workloads.f32_to_bf16_bits(rng.standard_normal((Hkv, 5000, d)).astype(np.float32))
+    ws = torch.zeros(kvc.decode_workspace_size(H, Hkv, d, 5000), dtype=torch.uint8, device="cuda")
+    orc = oracle.get()
+    for call, kk in enumerate([5000, 5000, 5000, 700]):
+        q = workloads.f32_to_bf16_bits(rng.standard_normal((H, d)).astype(np.float32))
+        kcc, vcc = np.ascontiguousarray(kc[:, :kk]), np.ascontiguousarray(vc[:, :kk])
+        out = kvc.kvc_decode_attention(dev_bf16(q), dev_bf16(kcc), dev_bf16(vcc), ws=ws)
+        torch.cuda.synchronize()
+        ref = orc.decode_attention(q, kcc, vcc, H, Hkv, 1 / math.sqrt(d))
+        parity.assert_decode_close(out.cpu().numpy(), ref, what=f"call {call} (kk={kk}) on a reused workspace")
+    assert int(ws[:Hkv * 4].view(torch.int32).abs().sum().item()) == 0, "ticket counters not returned to zero"
 
 
 def test_decode_over_the_layers_compacted_cache():
