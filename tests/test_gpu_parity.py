@@ -541,6 +541,44 @@ def test_rvq_encode_matches_oracle(n, d, S, M):
     np.testing.assert_allclose(residual.cpu().numpy(), xf - rec, rtol=0, atol=1e-5)
 
 
+def test_rvq_encode_strided_rows():
+    """Rows read through a row stride that is not a multiple of 8 elements
+    (the element-wise load path) give the same codes and residual as the
+    same rows stored contiguously (the 16-byte load path)."""
+    rng = np.random.default_rng(515)
+    n, d, S, M = 333, 128, 3, 128
+    x = workloads.f32_to_bf16_bits(rng.standard_normal((n, d)).astype(np.float32))
+    C = torch.from_numpy(workloads.make_codebooks(S, M, d, seed=12)).cuda()
+    wide = torch.zeros((n, d + 4), dtype=torch.bfloat16, device="cuda")
+    wide[:, :d] = dev_bf16(x)
+    strided = wide[:, :d]
+    assert strided.stride(0) == d + 4
+    r1 = torch.empty((n, d), dtype=torch.float32, device="cuda")
+    r2 = torch.empty((n, d), dtype=torch.float32, device="cuda")
+    c1, _ = kvc.kvc_rvq_encode(dev_bf16(x), C, residual=r1)
+    c2, _ = kvc.kvc_rvq_encode(strided, C, residual=r2)
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2) and torch.equal(r1, r2)
+
+
+def test_rvq_encode_crowded_codebook():
+    """A codebook of 256 near-copies of one vector puts every codeword inside
+    the candidate band of every row (more candidates than the parallel
+    re-scoring list holds): the per-warp re-scoring path decides, against the
+    oracle under the near-tie rule; a second, ordinary stage follows."""
+    rng = np.random.default_rng(616)
+    n, d, M = 300, 128, 256
+    x = workloads.f32_to_bf16_bits(rng.standard_normal((n, d)).astype(np.float32))
+    base = rng.standard_normal(d)
+    C0 = base[None, :] + 1e-3 * rng.standard_normal((M, d))
+    C1 = 0.5 * rng.standard_normal((M, d))
+    C = np.stack([C0, C1]).astype(np.float32)
+    codes, _ = kvc.kvc_rvq_encode(dev_bf16(x), torch.from_numpy(C).cuda())
+    torch.cuda.synchronize()
+    ref_codes, gap = oracle.get().rvq_encode(x, C)
+    parity.check_rvq_codes(codes.cpu().numpy(), ref_codes, gap, x, C, what="rvq, crowded codebook")
+
+
 def test_rvq_encode_planted_codes_and_ties():
     """Rows built as one codeword per stage (codebooks of entries +-8^-s,
     exact in bf16) come back with exactly those codes and a zero residual;
