@@ -75,6 +75,8 @@ class Oracle:
         lib.oracle_pivot_layer.restype = _I32
         lib.oracle_decode_attention.argtypes = [_P, _P, _P, _I32, _I32, _I64, _I32, ctypes.c_double, _P]
         lib.oracle_decode_attention.restype = _I32
+        lib.oracle_prefill_attention.argtypes = [_P, _P, _P, _I64, _I32, _I32, _I32, ctypes.c_double, _P, _P]
+        lib.oracle_prefill_attention.restype = _I32
         lib.oracle_rvq_encode.argtypes = [_P, _I64, _I64, _I32, _P, _I32, _I32, _P, _P]
         lib.oracle_rvq_encode.restype = _I32
         lib.oracle_max_threads.restype = _I32
@@ -181,6 +183,20 @@ class Oracle:
                                             float(scale), out.ctypes.data) != 0:
             raise ValueError("oracle_decode_attention: bad arguments")
         return out
+
+    def prefill_attention(self, q: np.ndarray, k: np.ndarray, v: np.ndarray, H: int, Hkv: int,
+                          scale: float):
+        """Causal attention of one sequence: (out [N][H][d], lse [N][H]) in
+        float64 from bf16 bits q [N][H][d], k and v [N][Hkv][d]."""
+        q, k, v = (np.ascontiguousarray(a, dtype=np.uint16) for a in (q, k, v))
+        N, Hq, d = q.shape
+        assert Hq == H and k.shape == (N, Hkv, d) and v.shape == k.shape
+        out = np.empty((N, H, d), dtype=np.float64)
+        lse = np.empty((N, H), dtype=np.float64)
+        if self.lib.oracle_prefill_attention(q.ctypes.data, k.ctypes.data, v.ctypes.data, N, H, Hkv, d,
+                                             float(scale), out.ctypes.data, lse.ctypes.data) != 0:
+            raise ValueError("oracle_prefill_attention: bad arguments")
+        return out, lse
 
     def rvq_encode(self, x: np.ndarray, C: np.ndarray):
         """Residual VQ codes [n][S] int32 and per-stage gaps [n][S] float64 of

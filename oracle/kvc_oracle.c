@@ -447,6 +447,72 @@ int oracle_decode_attention(const uint16_t* q, const uint16_t* kc, const uint16_
 }
 
 /*
+ * Causal prefill attention of one sequence, with each query row's
+ * log-sum-exp  [FastKV (gist.science 2502.01068) section 1: every layer runs
+ * full (quadratic) attention over the prompt during prefill; section 2.A: the
+ * TSP layer does so over the whole prompt, which is where the window rows'
+ * normalisers come from; FastKV abstract: grouped-query heads].  Query i sees
+ * keys j <= i:
+ *   s_ij       = scale * q[i,h] . k[j,g],   g = h / G
+ *   lse[i,h]   = ln sum_{j<=i} exp(s_ij)
+ *   out[i,h,:] = sum_{j<=i} exp(s_ij - lse[i,h]) v[j,g,:]
+ * q [N][H][d], k and v [N][Hkv][d], contiguous bf16 bits; out [N][H][d] and
+ * lse [N][H] float64.  Returns 0, or -1 on bad arguments.
+ */
+int oracle_prefill_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t N, int H,
+                             int Hkv, int d, double scale, double* out, double* lse) {
+  if (!q || !k || !v || !out || !lse || N < 1 || H <= 0 || Hkv <= 0 || H % Hkv || d <= 0) return -1;
+  double* kd = (double*)malloc(sizeof(double) * (size_t)N * Hkv * d);
+  double* vd = (double*)malloc(sizeof(double) * (size_t)N * Hkv * d);
+  if (!kd || !vd) {
+    free(kd); free(vd);
+    return -1;
+  }
+  for (int64_t e = 0; e < N * Hkv * d; ++e) {
+    kd[e] = bf16_to_f64(k[e]);
+    vd[e] = bf16_to_f64(v[e]);
+  }
+  int bad = 0;
+#pragma omp parallel for schedule(dynamic, 4) reduction(| : bad)
+  for (int64_t ih = 0; ih < N * H; ++ih) {
+    const int64_t i = ih / H;
+    const int h = (int)(ih % H);
+    const int g = kv_head_of(h, H, Hkv);
+#if ORACLE_MUTANT == 9
+    const int64_t last = i - 1 < 0 ? 0 : i - 1; /* mutant: the query's own key dropped */
+#else
+    const int64_t last = i;
+#endif
+    double* qd = (double*)malloc(sizeof(double) * (size_t)d);
+    double* sv = (double*)malloc(sizeof(double) * (size_t)(last + 1));
+    if (!qd || !sv) {
+      free(qd); free(sv);
+      bad = 1;
+      continue;
+    }
+    for (int c = 0; c < d; ++c) qd[c] = bf16_to_f64(q[ih * d + c]);
+    double mx = -INFINITY;
+    for (int64_t j = 0; j <= last; ++j) {
+      sv[j] = logit(qd, kd + (j * Hkv + g) * d, d, scale);
+      if (sv[j] > mx) mx = sv[j];
+    }
+    double z = 0.0;
+    for (int64_t j = 0; j <= last; ++j) z += exp(sv[j] - mx);
+    lse[ih] = mx + log(z);
+    double* o = out + ih * d;
+    for (int c = 0; c < d; ++c) o[c] = 0.0;
+    for (int64_t j = 0; j <= last; ++j) {
+      const double pj = exp(sv[j] - mx) / z;
+      const double* vr = vd + (j * Hkv + g) * d;
+      for (int c = 0; c < d; ++c) o[c] += pj * vr[c];
+    }
+    free(qd); free(sv);
+  }
+  free(kd); free(vd);
+  return bad ? -1 : 0;
+}
+
+/*
  * Residual vector quantisation of retained K or V rows  [VQKV (gist.science
  * 2603.16435) section 2: each cached vector is mapped to nearest codewords
  * stage by stage, the first codebook taking the main approximation and every

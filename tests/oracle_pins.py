@@ -541,7 +541,78 @@ def pin_rvq_tie_to_lowest_index(orc):
     return None
 
 
+# --------------------------------------------------------------------------- #
+# causal prefill attention with the rows' log-sum-exp
+# --------------------------------------------------------------------------- #
+def pin_prefill_sdpa(orc):
+    """Against torch SDPA in float64 (causal, GQA by repeating the KV heads)
+    for the outputs, and scipy's logsumexp of the masked logits the test
+    forms itself for the log-sum-exp."""
+    import torch
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(53)
+    for (N, H, Hkv, d) in [(37, 4, 2, 64), (9, 6, 3, 128), (1, 2, 1, 64)]:
+        q = _bf16(rng.standard_normal((N, H, d)) * 1.5)
+        k = _bf16(rng.standard_normal((N, Hkv, d)))
+        v = _bf16(rng.standard_normal((N, Hkv, d)))
+        scale = 1 / math.sqrt(d)
+        out, lse = orc.prefill_attention(q, k, v, H, Hkv, scale)
+        G = H // Hkv
+        qt = torch.from_numpy(_widen(q)).permute(1, 0, 2)                              # [H][N][d]
+        kt = torch.from_numpy(_widen(k)).permute(1, 0, 2).repeat_interleave(G, dim=0)  # [H][N][d]
+        vt = torch.from_numpy(_widen(v)).permute(1, 0, 2).repeat_interleave(G, dim=0)
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True, scale=scale)
+        ref = ref.permute(1, 0, 2).numpy()
+        err = np.max(np.abs(out - ref)) / max(np.max(np.abs(ref)), 1e-300)
+        if err > 1e-12:
+            return f"prefill attention != causal SDPA (N={N}, H={H}, Hkv={Hkv}): err {err:.3e}"
+        s = np.einsum("nhd,mhd->hnm", _widen(q), np.repeat(_widen(k), G, axis=1)) * scale    # [H][N][N]
+        s = np.where(np.tril(np.ones((N, N), dtype=bool))[None], s, -np.inf)
+        ref_lse = logsumexp(s, axis=2).T                                                       # [N][H]
+        if np.max(np.abs(lse - ref_lse)) > 1e-12 * max(1.0, np.max(np.abs(ref_lse))):
+            return f"prefill log-sum-exp != scipy logsumexp (N={N}, H={H})"
+    return None
+
+
+def pin_prefill_closed_forms(orc):
+    """K = 0: query i is uniform over keys 0..i, so its output is the mean of
+    V rows 0..i and its log-sum-exp is ln(i + 1); query 0 returns V row 0."""
+    rng = np.random.default_rng(59)
+    N, H, Hkv, d = 20, 4, 2, 64
+    q = _bf16(rng.standard_normal((N, H, d)))
+    v = _bf16(rng.standard_normal((N, Hkv, d)))
+    out, lse = orc.prefill_attention(q, np.zeros((N, Hkv, d), dtype=np.uint16), v, H, Hkv, 0.125)
+    vm = np.cumsum(_widen(v), axis=0) / np.arange(1, N + 1)[:, None, None]     # running means [N][Hkv][d]
+    ref = np.repeat(vm, H // Hkv, axis=1)
+    if np.max(np.abs(out - ref)) > 1e-13:
+        return "prefill attention with K = 0 is not the running mean of V"
+    if np.max(np.abs(lse - np.log(np.arange(1, N + 1))[:, None])) > 1e-13:
+        return "prefill log-sum-exp with K = 0 is not ln(i + 1)"
+    out1, _ = orc.prefill_attention(q, _bf16(rng.standard_normal((N, Hkv, d))), v, H, Hkv, 0.125)
+    if not np.array_equal(out1[0], np.repeat(_widen(v[0]), H // Hkv, axis=0)):
+        return "the first query's output is not V row 0"
+    return None
+
+
+def pin_prefill_lse_feeds_window_scores(orc):
+    """The window rows' log-sum-exp from the prefill attention, handed to the
+    given-normaliser scores, reproduces the two-pass window scores (the
+    scoring normaliser is the attention's)."""
+    rng = np.random.default_rng(61)
+    N, H, Hkv, d, w = 60, 4, 2, 64, 5
+    qa = _bf16(rng.standard_normal((N, H, d)))
+    k = _bf16(rng.standard_normal((N, Hkv, d)))
+    _, lse = orc.prefill_attention(qa, k, np.zeros_like(k), H, Hkv, 0.125)
+    qw = qa[N - w:]
+    A2 = orc.window_scores(qw, k, H, Hkv, w, 0.125)
+    A1 = orc.window_scores_lse(qw, k, np.ascontiguousarray(lse[N - w:]), H, Hkv, w, 0.125)
+    if np.max(np.abs(A1 - A2)) > 1e-12 * max(1.0, np.max(np.abs(A2))):
+        return "window scores from the prefill log-sum-exp differ from the two-pass scores"
+    return None
+
+
 ALL_PINS = [pin_zero_keys, pin_sdpa, pin_mpmath, pin_mass, pin_dominant_key, pin_lse_sdpa, pin_lse_zero_keys,
             pin_lse_shift, pin_pool, pin_select, pin_gather, pin_stats, pin_pivot_hand_cases,
             pin_pivot_synthetic_phase_change, pin_decode_sdpa, pin_decode_closed_forms,
-            pin_rvq_nearest_and_residual, pin_rvq_planted_codes, pin_rvq_tie_to_lowest_index]
+            pin_rvq_nearest_and_residual, pin_rvq_planted_codes, pin_rvq_tie_to_lowest_index,
+            pin_prefill_sdpa, pin_prefill_closed_forms, pin_prefill_lse_feeds_window_scores]

@@ -14,7 +14,7 @@ def test_pin_holds(orc, pin):
     assert pin(orc) is None
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8, 9])
 def test_each_planted_mistake_is_caught(mutant):
     """Every deliberately broken oracle build violates at least one pin."""
     bad = oracle.mutant(mutant)
