@@ -140,6 +140,15 @@ def load_traffic(kernel: str):
         return None
 
 
+def tensor_peak_bf16():
+    """Dense bf16 tensor peak: the measured cuBLAS bf16 GEMM burst figure."""
+    try:
+        mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        return round(float(mp["bf16_tflops"]), 1), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def tensor_peak_tf32():
     """Dense tf32 tensor peak: the measured bf16 GEMM peak times the nominal
     tf32 / bf16 ratio (1.1 / 2.25 PFLOP/s)."""
@@ -672,6 +681,39 @@ def main() -> None:
     rvq_flop = 2 * rvq_rows * rvq_M * cfg.d * rvq_S
     tf32_peak, tf32_kind = tensor_peak_tf32()
 
+    # ---- causal prefill attention with the rows' log-sum-exp -----------------
+    # The producer of the window rows' normalisers (the TSP layer's attention
+    # over the prompt) and the later layers' attention over the propagated
+    # tokens: random queries over the layer's first n_pre keys and values.
+    pre = None
+    if cfg.d == 128:
+        n_pre = min(cfg.N, 32768)
+        gp = torch.Generator(device=dev)
+        gp.manual_seed(23)
+        q_pre = torch.randn(n_pre, cfg.H, cfg.d, device=dev, generator=gp).to(torch.bfloat16)
+        k_pre, v_pre = k[:n_pre], v[:n_pre]
+        out_pre = torch.empty((n_pre, cfg.H, cfg.d), dtype=torch.bfloat16, device=dev)
+        lse_pre = torch.empty((n_pre, cfg.H), dtype=torch.float32, device=dev)
+        kvc.kvc_prefill_attention(q_pre, k_pre, v_pre, out=out_pre, lse=lse_pre, dev_err=plan.dev_err, stream=st)
+        torch.cuda.synchronize(dev)
+        n_p = 3
+        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        p0.record(st)
+        for _ in range(n_p):
+            kvc.kvc_prefill_attention(q_pre, k_pre, v_pre, out=out_pre, lse=lse_pre, dev_err=plan.dev_err,
+                                      stream=st)
+        p1.record(st)
+        torch.cuda.synchronize(dev)
+        ms_pre = p0.elapsed_time(p1) / n_p
+        pre_flop = 4 * cfg.d * cfg.H * n_pre * (n_pre + 1) / 2  # QK^T and PV over the causal half
+        bf16_peak, bf16_kind = tensor_peak_bf16()
+        pre = {"ms": round(ms_pre, 4), "n": n_pre, "tflops": round(pre_flop / (ms_pre * 1e-3) / 1e12, 1),
+               "tflops_peak_bf16": bf16_peak, "peak_kind": bf16_kind,
+               "frac": round(pre_flop / (ms_pre * 1e-3) / 1e12 / bf16_peak, 4),
+               "note": f"kvc_prefill_attention: causal, {cfg.H}/{cfg.Hkv} heads, d {cfg.d}, over {n_pre} tokens, "
+                       "with every row's log-sum-exp; not part of the headline step"}
+        del q_pre, out_pre, lse_pre
+
     # ---- end to end through the public API with host buffers ------------------
     hq, hk, hv, hx = (workloads.torch_bf16(a).pin_memory() for a in (lay.q, lay.k, lay.v, lay.x))
     outs = [plan.idx_kv, plan.idx_tsp, plan.k_c, plan.v_c, plan.x_c]
@@ -739,6 +781,7 @@ def main() -> None:
                        "note": "kvc_decode_attention: one decode query per head over the compacted cache "
                                f"({cfg.Hkv} x {cfg.k_kv} entries, K and V), cache copies cycled past L2; "
                                "not part of the headline step"},
+            "prefill_attention": pre,
             "score_lse": {"ms": round(ms_lse, 5), "alg_bytes": alg["score"],
                           "gbs": round(alg["score"] / (ms_lse * 1e-3) / 1e9, 1),
                           "max_rel_diff_vs_two_pass": rel_lse,

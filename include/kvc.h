@@ -322,6 +322,36 @@ kvc_status kvc_decode_attention(const uint16_t* q, int64_t q_stride_h, const uin
                                 int64_t kk, int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
                                 float* out, void* ws, size_t ws_bytes, int32_t* dev_err, void* stream);
 
+/* Causal prefill attention with the rows' log-sum-exp ------------------- */
+
+/*
+ * Causal attention of one sequence over itself, returning every query row's
+ * log-sum-exp  [FastKV (gist.science 2502.01068) 1: during prefill every
+ * layer runs full attention over the prompt; 2.A: at the TSP layer this is
+ * the attention whose window rows' normalisers the token scores use --
+ * kvc_score_lse takes lse[n - w .. n) and reads K once; FastKV abstract:
+ * grouped-query heads, h reads KV head h / G].  Query i sees keys j <= i:
+ *     s_ij     = scale * q[i, h, :] . k[j, g, :]
+ *     lse[i,h] = ln sum_{j <= i} exp(s_ij)
+ *     out[i,h] = sum_{j <= i} exp(s_ij - lse[i,h]) v[j, g, :]
+ * The same call is the attention of the later layers over the TSP-propagated
+ * tokens (their positions ascend, so the causal order carries over).
+ *  q        [n][H][d] bf16, contiguous, 16-byte aligned
+ *  k, v     [n][Hkv][d] bf16, contiguous, 16-byte aligned
+ *  out      [n][H][d] bf16 out, 16-byte aligned, or NULL (log-sum-exp only)
+ *  lse      [n][H] fp32 out, or NULL
+ *  dev_err  device int32 or NULL (KVC_DEV_ERR_TIMEOUT only)
+ * head_dim 128; 1 <= n < 2^31.  Both contractions run on the tensor cores
+ * (bf16 operands, fp32 accumulation); the probabilities enter the output
+ * contraction as bf16 and the output is normalised by the sum of those
+ * rounded probabilities (a convex combination of V rows: |error| <= ~6e-3 of
+ * max |v|), while the log-sum-exp sums the fp32 probabilities in fp64
+ * (relative error ~1e-6).  Deterministic.
+ */
+kvc_status kvc_prefill_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v, int64_t n,
+                                 int32_t num_heads, int32_t num_kv_heads, int32_t head_dim, float scale,
+                                 uint16_t* out, float* lse, int32_t* dev_err, void* stream);
+
 /* Residual vector quantisation of retained rows --------------------------- */
 
 /*

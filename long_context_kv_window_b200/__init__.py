@@ -57,6 +57,7 @@ _SIGS = {
     "kvc_score_noalloc": ([_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P], _I32),
     "kvc_score_lse": ([_P, _I64, _I64, _P, _I64, _I64, _I64, _P, _P, _I64, _I64, _P, _P, _P, _P, _SZ, _P, _P],
                       _I32),
+    "kvc_prefill_attention": ([_P, _P, _P, _I64, _I32, _I32, _I32, ctypes.c_float, _P, _P, _P, _P], _I32),
     "kvc_select_workspace_size": ([_I32, _I32, _I64, _P], _I32),
     "kvc_select_topk": ([_P, _I32, _I64, _I32, _I64, _I32, _I32, _I64, _P, _I64, _P, _P, _SZ, _P], _I32),
     "kvc_select_topk_varlen": ([_P, _I32, _I64, _I32, _P, _I32, _I64, _I64, _I32, _I32, _I64, _P, _P, _P,
@@ -527,6 +528,38 @@ def kvc_decode_attention(q: torch.Tensor, k_c: torch.Tensor, v_c: torch.Tensor, 
                  _ptr(out), _ptr(ws), _ws_bytes(ws, dev), _ptr(dev_err), _stream(stream, dev)),
            "kvc_decode_attention")
     return out
+
+
+def kvc_prefill_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, scale: Optional[float] = None,
+                          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                          want_out: bool = True, dev_err: Optional[torch.Tensor] = None,
+                          stream=None) -> Tuple[Optional[torch.Tensor], torch.Tensor]:
+    """Causal attention of one sequence, q [n][H][d], k and v [n][Hkv][d]
+    (bf16, contiguous): returns (out bf16 [n][H][d] or None when want_out is
+    False and none was passed, lse fp32 [n][H], the rows' log-sum-exp)."""
+    _bf16(q, "q", 3)
+    _bf16(k, "k", 3)
+    _bf16(v, "v", 3)
+    dev = q.device
+    _same_device(dev, k=k, v=v)
+    n, H, d = q.shape
+    if tuple(k.shape[::2]) != (n, d) or tuple(v.shape) != tuple(k.shape):
+        raise ValueError("q [n][H][d], k and v [n][Hkv][d] must agree")
+    if not (q.is_contiguous() and k.is_contiguous() and v.is_contiguous()):
+        raise ValueError("q, k and v must be contiguous")
+    Hkv = k.shape[1]
+    if out is None and want_out:
+        out = torch.empty((n, H, d), dtype=torch.bfloat16, device=dev)
+    if out is not None:
+        _dense(out, "out", (n, H, d), _BF16_BITS, dev)
+    if lse is None:
+        lse = torch.empty((n, H), dtype=torch.float32, device=dev)
+    _dense(lse, "lse", (n, H), torch.float32, dev)
+    _err_word(dev_err, dev)
+    sc = float(1.0 / math.sqrt(d) if scale is None else scale)
+    _check(_call(dev, lib().kvc_prefill_attention, _ptr(q), _ptr(k), _ptr(v), n, H, Hkv, d, sc, _ptr(out),
+                 _ptr(lse), _ptr(dev_err), _stream(stream, dev)), "kvc_prefill_attention")
+    return out, lse
 
 
 # --------------------------------------------------------------------------- #

@@ -154,6 +154,20 @@ def test_decode_attention_rejects_bad_arguments(lib):
     assert kvc.launch_count() == before
 
 
+def test_prefill_attention_rejects_bad_arguments(lib):
+    dummy = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    before = kvc.launch_count()
+    assert lib.kvc_prefill_attention(None, dummy, dummy, 100, 32, 8, 128, 0.1, dummy, dummy, None, None) == 1
+    assert lib.kvc_prefill_attention(dummy, dummy, dummy, 100, 32, 8, 64, 0.1, dummy, dummy, None, None) == 2  # d 64
+    assert lib.kvc_prefill_attention(dummy, dummy, dummy, 100, 30, 8, 128, 0.1, dummy, dummy, None, None) == 1
+    assert lib.kvc_prefill_attention(dummy, dummy, dummy, 0, 32, 8, 128, 0.1, dummy, dummy, None, None) == 1
+    assert lib.kvc_prefill_attention(dummy, dummy, dummy, 100, 32, 8, 128, 0.0, dummy, dummy, None, None) == 1
+    assert lib.kvc_prefill_attention(dummy, ctypes.c_void_p(264), dummy, 100, 32, 8, 128, 0.1, dummy, dummy,
+                                     None, None) == 1  # misaligned k
+    assert kvc.last_error() != ""
+    assert kvc.launch_count() == before
+
+
 def test_rvq_encode_rejects_bad_arguments(lib):
     dummy = ctypes.c_void_p(256)  # never dereferenced: validation fails first
     before = kvc.launch_count()

@@ -515,6 +515,102 @@ def test_decode_over_the_layers_compacted_cache():
 
 
 # --------------------------------------------------------------------------- #
+# causal prefill attention with the rows' log-sum-exp
+# --------------------------------------------------------------------------- #
+def _prefill_inputs(rng, N, H, Hkv, d=128, planted=0):
+    q = rng.standard_normal((N, H, d)).astype(np.float32)
+    k = rng.standard_normal((N, Hkv, d)).astype(np.float32)
+    v = rng.standard_normal((N, Hkv, d)).astype(np.float32)
+    if planted:  # keys aligned with the queries of their group: logits far above the rest, mid-sequence
+        G = H // Hkv
+        for pos in rng.choice(N, size=min(planted, N), replace=False):
+            for g in range(Hkv):
+                u = q[min(N - 1, pos + 3), g * G].copy()
+                k[pos, g] = 4.0 * u / np.linalg.norm(u) * np.sqrt(d)
+    return tuple(workloads.f32_to_bf16_bits(a) for a in (q, k, v))
+
+
+def assert_prefill_close(out, lse, ref_out, ref_lse, v_bits, H, Hkv, what):
+    """Outputs within 6e-3 of max |v| of the KV head (the bf16 probabilities
+    and the bf16 output each round by <= 2^-9: a convex combination of V rows
+    whose weights move by <= 2^-8 relative, plus the output rounding); the
+    log-sum-exp within 2e-5 of max(1, |lse|) (fp32 logits, fp64 sums)."""
+    G = H // Hkv
+    vmax = np.abs(workloads.bf16_bits_to_f32(v_bits)).max(axis=(0, 2))          # [Hkv]
+    bound = 6e-3 * np.repeat(vmax, G)[None, :, None]
+    err = np.abs(out - ref_out)
+    assert np.all(err <= bound), f"{what}: output error {float((err / bound).max()):.2f} x the bound"
+    lerr = np.abs(lse - ref_lse) / np.maximum(1.0, np.abs(ref_lse))
+    assert lerr.max() <= 2e-5, f"{what}: log-sum-exp error {lerr.max():.2e}"
+
+
+@pytest.mark.parametrize("N,H,Hkv,planted", [(1, 4, 2, 0), (100, 4, 1, 3), (128, 8, 2, 0), (129, 4, 4, 2),
+                                             (300, 6, 3, 5), (700, 32, 8, 8), (1000, 4, 2, 0)])
+def test_prefill_attention_matches_oracle(N, H, Hkv, planted):
+    """Causal attention with grouped heads against the float64 oracle: single
+    and ragged query blocks, G = 1, 2, 4; planted keys make some rows' maxima
+    jump by far more than the reference slack mid-sequence (the output
+    rescale in TMEM).  The log-sum-exp only mode (no output) gives the same
+    log-sum-exp."""
+    rng = np.random.default_rng(N * 7 + H + planted)
+    q, k, v = _prefill_inputs(rng, N, H, Hkv, planted=planted)
+    err = _err_word()
+    out, lse = kvc.kvc_prefill_attention(dev_bf16(q), dev_bf16(k), dev_bf16(v), dev_err=err)
+    _, lse2 = kvc.kvc_prefill_attention(dev_bf16(q), dev_bf16(k), dev_bf16(v), want_out=False)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+    assert torch.equal(lse, lse2)
+    ref_out, ref_lse = oracle.get().prefill_attention(q, k, v, H, Hkv, 1 / math.sqrt(128))
+    assert_prefill_close(out.float().cpu().numpy(), lse.cpu().numpy(), ref_out, ref_lse, v, H, Hkv,
+                         f"prefill N={N} H={H} Hkv={Hkv}")
+
+
+def test_prefill_log_sum_exp_scores_the_window_in_one_read():
+    """The TSP layer's chain with the prefill attention as the producer: its
+    window rows' log-sum-exp handed to kvc_score_lse (one read of K) gives the
+    two-pass scores within 1e-3 of the oracle and, ranked, the oracle's TSP and
+    K/V sets under the near-tie rule."""
+    cfg = workloads.shrink(workloads.C3, N=4096, k_kv=410, k_tsp=819, n_hitters=16, seed=64)
+    rng = np.random.default_rng(64)
+    N, H, Hkv, w = cfg.N, cfg.H, cfg.Hkv, cfg.w
+    q, k, v = _prefill_inputs(rng, N, H, Hkv)
+    qd, kd, vd = dev_bf16(q), dev_bf16(k), dev_bf16(v)
+    _, lse = kvc.kvc_prefill_attention(qd, kd, vd, want_out=False)
+    S1 = kvc.kvc_score_lse(qd[N - w:], kd, lse[N - w:])
+    S2 = kvc.kvc_score(qd[N - w:], kd)
+    torch.cuda.synchronize()
+    qw = np.ascontiguousarray(q[N - w:])
+    res = oracle.layer(qw, k, H, Hkv, w, 1 / math.sqrt(128), cfg.pool, cfg.k_kv, k_tsp=cfg.k_tsp)
+    parity.assert_scores_close(S1.cpu().numpy(), res.A, what="scores from the prefill log-sum-exp")
+    parity.assert_scores_close(S2.cpu().numpy(), res.A, what="two-pass scores")
+    ik = kvc.kvc_select_topk(S1, w, cfg.pool, cfg.k_kv).cpu().numpy()
+    it = kvc.kvc_select_topk(S1, w, cfg.pool, cfg.k_tsp, row_group=Hkv).cpu().numpy()[0]
+    for g in range(Hkv):
+        parity.assert_selection_matches(ik[g], res.idx_kv[g], res.pooled[g], N, w, cfg.k_kv, what=f"K/V set {g}")
+    parity.assert_selection_matches(it, res.idx_tsp, res.pooled_tsp, N, w, cfg.k_tsp, what="TSP set")
+
+
+def test_prefill_over_the_propagated_tokens():
+    """The later layers' attention over the TSP-propagated tokens: the query,
+    key and value rows of the selected positions (gathered as hidden rows,
+    ascending) attend causally among themselves, against the oracle on the
+    same compacted rows."""
+    rng = np.random.default_rng(71)
+    N, H, Hkv = 2048, 8, 2
+    q, k, v = _prefill_inputs(rng, N, H, Hkv)
+    idx = np.sort(rng.choice(N, size=600, replace=False)).astype(np.int32)
+    it = torch.from_numpy(idx).cuda()
+    qc = kvc.kvc_gather_hidden(dev_bf16(q).view(N, H * 128), it).view(-1, H, 128)
+    kc = kvc.kvc_gather_hidden(dev_bf16(k).view(N, Hkv * 128), it).view(-1, Hkv, 128)
+    vc = kvc.kvc_gather_hidden(dev_bf16(v).view(N, Hkv * 128), it).view(-1, Hkv, 128)
+    out, lse = kvc.kvc_prefill_attention(qc, kc, vc)
+    torch.cuda.synchronize()
+    ref_out, ref_lse = oracle.get().prefill_attention(q[idx], k[idx], v[idx], H, Hkv, 1 / math.sqrt(128))
+    assert_prefill_close(out.float().cpu().numpy(), lse.cpu().numpy(), ref_out, ref_lse, v[idx], H, Hkv,
+                         "prefill over the propagated tokens")
+
+
+# --------------------------------------------------------------------------- #
 # residual vector quantisation
 # --------------------------------------------------------------------------- #
 @pytest.mark.parametrize("n,d,S,M", [(1000, 128, 4, 256), (129, 128, 2, 256), (300, 64, 3, 64), (77, 128, 1, 16),
