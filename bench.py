@@ -502,6 +502,8 @@ def main() -> None:
     st = torch.cuda.current_stream(dev)
     side = plan.side
     calls = ["score", "select_kv", "gather_kv", "select_tsp", "gather_hidden"]
+    given_lse = [None]  # the window rows' log-sum-exp, for the one-read variant of the step
+
     def step(evs=None, main=None):
         """One layer: the K/V chain on a side stream, the TSP chain on the main
         stream (as LayerPlan.run), with optional per-call timing events
@@ -516,8 +518,12 @@ def main() -> None:
             fn()
             if evs is not None:
                 evs[name][1].record(call_stream[name])
-        timed("score", lambda: kvc.kvc_score(q, k, scores=plan.scores, ws=plan.ws_score, dev_err=plan.dev_err,
-                                             stream=st))
+        if given_lse[0] is None:
+            timed("score", lambda: kvc.kvc_score(q, k, scores=plan.scores, ws=plan.ws_score, dev_err=plan.dev_err,
+                                                 stream=st))
+        else:
+            timed("score", lambda: kvc.kvc_score_lse(q, k, given_lse[0], scores=plan.scores, ws=plan.ws_score,
+                                                     dev_err=plan.dev_err, stream=st))
         ev_scores.record(st)
         timed("select_tsp", lambda: kvc.kvc_select_topk(plan.scores, cfg.w, cfg.pool, cfg.k_tsp, row_group=cfg.Hkv,
                                                         idx=plan.idx_tsp, ws=plan.ws_sel_tsp, stream=st))
@@ -620,6 +626,13 @@ def main() -> None:
     ms_lse = l0.elapsed_time(l1) / n_lse
     rel_lse = float(((lse_scores - plan.scores).abs() / plan.scores.abs().clamp_min(1e-30)).max())
     del lse_scores
+    # the whole step with those normalisers given (one read of K): what the
+    # layer costs when its prefill attention supplies them (not the headline)
+    given_lse[0] = lse
+    for _ in range(3):
+        step()
+    ms_step_lse, _, _ = timed_run(with_events=False)
+    given_lse[0] = None
 
     # ---- decode over the compacted cache (the consumer of the K/V retention) ----
     # One decode query per head over the retained entries.  The cache (K_c +
@@ -782,6 +795,13 @@ def main() -> None:
                                f"({cfg.Hkv} x {cfg.k_kv} entries, K and V), cache copies cycled past L2; "
                                "not part of the headline step"},
             "prefill_attention": pre,
+            "step_with_given_normalisers": {
+                "ms_per_step": round(ms_step_lse, 5), "value": world * cfg.N / (ms_step_lse * 1e-3),
+                "unit": "tokens/s", "hbm_gbs": round(layer_bytes(cfg) / (ms_step_lse * 1e-3) / 1e9, 1),
+                "frac": round(layer_bytes(cfg) / (ms_step_lse * 1e-3) / 1e9 / peak, 4),
+                "note": "the same layer step with the window rows' log-sum-exp supplied (as the layer's "
+                        "prefill attention, kvc_prefill_attention, returns it) and kvc_score_lse in place of "
+                        "kvc_score: one read of K; not the headline"},
             "score_lse": {"ms": round(ms_lse, 5), "alg_bytes": alg["score"],
                           "gbs": round(alg["score"] / (ms_lse * 1e-3) / 1e9, 1),
                           "max_rel_diff_vs_two_pass": rel_lse,

@@ -682,9 +682,11 @@ class LayerPlan:
         self._ev_scores = torch.cuda.Event()
         self._ev_side = torch.cuda.Event()
 
-    def run(self, q_win, k, v=None, x=None, stream=None) -> LayerOutputs:
+    def run(self, q_win, k, v=None, x=None, stream=None, lse=None) -> LayerOutputs:
         """Score -> per-KV-head top-k -> K/V gather; with a TSP budget also the
-        all-head top-k -> hidden-state gather.
+        all-head top-k -> hidden-state gather.  With lse (the window rows'
+        log-sum-exp [w][H], as kvc_prefill_attention returns it for the last w
+        rows) the scores come from kvc_score_lse: one read of K.
 
         The TSP selection ranks the sum of the KV-head score rows, formed as it
         stages them (heads in order, the same fp32 sum as the scoring call's
@@ -696,8 +698,12 @@ class LayerPlan:
         synchronised with the host; inputs must stay alive until the work
         completes."""
         main = stream if stream is not None else torch.cuda.current_stream(self.scores.device)
-        kvc_score(q_win, k, scores=self.scores, tsp=self.tsp, ws=self.ws_score, dev_err=self.dev_err,
-                  stream=main)
+        if lse is None:
+            kvc_score(q_win, k, scores=self.scores, tsp=self.tsp, ws=self.ws_score, dev_err=self.dev_err,
+                      stream=main)
+        else:
+            kvc_score_lse(q_win, k, lse, scores=self.scores, tsp=self.tsp, ws=self.ws_score, dev_err=self.dev_err,
+                          stream=main)
         out = LayerOutputs(self.scores, self.idx_kv, self.k_c, self.v_c)
         if self.k_tsp is None:
             self._kv_chain(k, v, main)

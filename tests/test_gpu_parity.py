@@ -583,11 +583,17 @@ def test_prefill_log_sum_exp_scores_the_window_in_one_read():
     res = oracle.layer(qw, k, H, Hkv, w, 1 / math.sqrt(128), cfg.pool, cfg.k_kv, k_tsp=cfg.k_tsp)
     parity.assert_scores_close(S1.cpu().numpy(), res.A, what="scores from the prefill log-sum-exp")
     parity.assert_scores_close(S2.cpu().numpy(), res.A, what="two-pass scores")
+    # the layer plan with the same normalisers: the same scores and sets as the direct calls
+    plan = kvc.LayerPlan(N, H, Hkv, 128, w, cfg.k_kv, cfg.k_tsp, None, False, "cuda", pool_kernel=cfg.pool)
+    outp = plan.run(qd[N - w:], kd, lse=lse[N - w:])
+    torch.cuda.synchronize()
+    assert torch.equal(outp.scores, S1)
     ik = kvc.kvc_select_topk(S1, w, cfg.pool, cfg.k_kv).cpu().numpy()
     it = kvc.kvc_select_topk(S1, w, cfg.pool, cfg.k_tsp, row_group=Hkv).cpu().numpy()[0]
     for g in range(Hkv):
         parity.assert_selection_matches(ik[g], res.idx_kv[g], res.pooled[g], N, w, cfg.k_kv, what=f"K/V set {g}")
     parity.assert_selection_matches(it, res.idx_tsp, res.pooled_tsp, N, w, cfg.k_tsp, what="TSP set")
+    assert np.array_equal(outp.idx_kv.cpu().numpy(), ik) and np.array_equal(outp.idx_tsp.cpu().numpy()[0], it)
 
 
 def test_prefill_over_the_propagated_tokens():
