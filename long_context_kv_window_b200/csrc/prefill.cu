@@ -291,26 +291,31 @@ prefill_attention_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_
       }
       // P buffer b was last read by the output MMA of tile t - 2
       if (t >= 2 && !tc::mbar_wait(&bars->o_done[b], ((t >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
-      const float nm = -m_ref;
-      float se = 0.f, sr = 0.f;
+      // p in packed pairs, its bf16 copy into P, and both row sums on two
+      // accumulators each (short dependency chains)
+      const float2 c2 = make_float2(a.c, a.c), nm2 = make_float2(-m_ref, -m_ref);
+      float2 se2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+      float2 sr2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       uint8_t* pb = prow + b * L::kTile;
 #pragma unroll
       for (int c8 = 0; c8 < kPT; c8 += 8) {
         uint32_t w[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const float p0 = tc::ex2_approx(fmaf(__uint_as_float(x[c8 + 2 * u]), a.c, nm));
-          const float p1 = tc::ex2_approx(fmaf(__uint_as_float(x[c8 + 2 * u + 1]), a.c, nm));
-          const __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
-          se += p0 + p1;
-          sr += __low2float(hp) + __high2float(hp);
+          const float2 t2 =
+              tc::fma2(make_float2(__uint_as_float(x[c8 + 2 * u]), __uint_as_float(x[c8 + 2 * u + 1])), c2, nm2);
+          const float2 p2 = make_float2(tc::ex2_approx(t2.x), tc::ex2_approx(t2.y));
+          const __nv_bfloat162 hp = __floats2bfloat162_rn(p2.x, p2.y);
+          se2[u & 1] = tc::add2(se2[u & 1], p2);
+          sr2[u & 1] = tc::add2(sr2[u & 1], __bfloat1622float2(hp));
           w[u] = *reinterpret_cast<const uint32_t*>(&hp);
         }
         const int blk = c8 >> 6, ch = ((c8 & 63) >> 3) ^ (r & 7);
         *reinterpret_cast<uint4*>(pb + blk * L::kBlk + (ch << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      l_round += sr;
-      l_exact += (double)se;
+      const float2 se = tc::add2(se2[0], se2[1]), sr = tc::add2(sr2[0], sr2[1]);
+      l_round += sr.x + sr.y;
+      l_exact += (double)(se.x + se.y);
       tc::fence_proxy_async_smem();  // P visible to the tensor core
       tc::tc_fence_before();         // (and the O rescale stores)
       __syncwarp();
