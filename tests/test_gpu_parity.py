@@ -596,6 +596,35 @@ def test_prefill_log_sum_exp_scores_the_window_in_one_read():
     assert np.array_equal(outp.idx_kv.cpu().numpy(), ik) and np.array_equal(outp.idx_tsp.cpu().numpy()[0], it)
 
 
+def test_new_kernels_are_deterministic_under_repetition():
+    """Repeated calls give bit-identical results: the decode's last-CTA merge
+    (ticket counters), the residual-VQ candidate list and per-row atomic
+    minimum, and the prefill's warp-local references and TMEM rescales
+    depend on no arrival order."""
+    rng = np.random.default_rng(97)
+    H, Hkv, d, kk = 32, 8, 128, 3000
+    q = dev_bf16(workloads.f32_to_bf16_bits(rng.standard_normal((H, d)).astype(np.float32)))
+    kc = dev_bf16(workloads.f32_to_bf16_bits(rng.standard_normal((Hkv, kk, d)).astype(np.float32)))
+    vc = dev_bf16(workloads.f32_to_bf16_bits(rng.standard_normal((Hkv, kk, d)).astype(np.float32)))
+    ws = torch.zeros(kvc.decode_workspace_size(H, Hkv, d, kk), dtype=torch.uint8, device="cuda")
+    ref = kvc.kvc_decode_attention(q, kc, vc, ws=ws).clone()
+    for _ in range(20):
+        assert torch.equal(kvc.kvc_decode_attention(q, kc, vc, ws=ws), ref)
+    C = torch.from_numpy(workloads.make_codebooks(4, 256, d, seed=5)).cuda()
+    rows = kc.view(-1, d)
+    rc, _ = kvc.kvc_rvq_encode(rows, C)
+    rc = rc.clone()
+    for _ in range(10):
+        assert torch.equal(kvc.kvc_rvq_encode(rows, C)[0], rc)
+    qp, kp, vp = (dev_bf16(a) for a in _prefill_inputs(rng, 1500, 8, 2, planted=4))
+    o0, l0 = kvc.kvc_prefill_attention(qp, kp, vp)
+    o0, l0 = o0.clone(), l0.clone()
+    for _ in range(10):
+        o1, l1 = kvc.kvc_prefill_attention(qp, kp, vp)
+        assert torch.equal(o1, o0) and torch.equal(l1, l0)
+    torch.cuda.synchronize()
+
+
 def test_prefill_over_the_propagated_tokens():
     """The later layers' attention over the TSP-propagated tokens: the query,
     key and value rows of the selected positions (gathered as hidden rows,
