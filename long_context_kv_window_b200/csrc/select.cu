@@ -134,22 +134,56 @@ __device__ __forceinline__ int4 ld_dsmem_v4(uint32_t local, uint32_t rank) {
 template <int CS>
 __device__ void cluster_find_bucket(cg::cluster_group& cluster, RadixShared& sh, int buf, int nbins,
                                     uint32_t want) {
-  // 16-byte loads of every rank's histogram, all issued before the sum: one
-  // round trip through distributed shared memory
-  for (int v4 = threadIdx.x; v4 < nbins / 4; v4 += kThreads) {
-    int4 part[CS];
-    const uint32_t local = (uint32_t)__cvta_generic_to_shared(&sh.hist[buf][4 * v4]);
+  if constexpr (CS <= 8) {
+    // 16-byte loads of every rank's histogram, all issued before the sum: one
+    // round trip through distributed shared memory
+    for (int v4 = threadIdx.x; v4 < nbins / 4; v4 += kThreads) {
+      int4 part[CS];
+      const uint32_t local = (uint32_t)__cvta_generic_to_shared(&sh.hist[buf][4 * v4]);
 #pragma unroll
-    for (int c = 0; c < CS; ++c) part[c] = ld_dsmem_v4(local, (uint32_t)c);
-    int4 acc = part[0];
+      for (int c = 0; c < CS; ++c) part[c] = ld_dsmem_v4(local, (uint32_t)c);
+      int4 acc = part[0];
 #pragma unroll
-    for (int c = 1; c < CS; ++c) {
-      acc.x += part[c].x;
-      acc.y += part[c].y;
-      acc.z += part[c].z;
-      acc.w += part[c].w;
+      for (int c = 1; c < CS; ++c) {
+        acc.x += part[c].x;
+        acc.y += part[c].y;
+        acc.z += part[c].z;
+        acc.w += part[c].w;
+      }
+      reinterpret_cast<int4*>(sh.tot)[v4] = acc;
     }
-    reinterpret_cast<int4*>(sh.tot)[v4] = acc;
+  } else {
+    // Larger clusters: every rank reading every histogram moves CS^2
+    // histograms through the cluster.  Instead each rank sums its own slice
+    // of the bins over all ranks (a reduce-scatter), and after a cluster
+    // barrier collects the CS summed slices: 2 x CS slices per rank.
+    const int slice = nbins / CS;  // a multiple of 4
+    const uint32_t me = cluster.block_rank();
+    for (int v4 = threadIdx.x; v4 < slice / 4; v4 += kThreads) {
+      const int bin = (int)me * slice + 4 * v4;
+      int4 part[CS];
+      const uint32_t local = (uint32_t)__cvta_generic_to_shared(&sh.hist[buf][bin]);
+#pragma unroll
+      for (int c = 0; c < CS; ++c) part[c] = ld_dsmem_v4(local, (uint32_t)c);
+      int4 acc = part[0];
+#pragma unroll
+      for (int c = 1; c < CS; ++c) {
+        acc.x += part[c].x;
+        acc.y += part[c].y;
+        acc.z += part[c].z;
+        acc.w += part[c].w;
+      }
+      *reinterpret_cast<int4*>(&sh.tot[bin]) = acc;
+    }
+    cluster.sync();
+    // other ranks' slices (this rank's own slice is in place); a rank writes
+    // only slices it does not own, and reads only the owners' slices
+    for (int v4 = threadIdx.x; v4 < nbins / 4; v4 += kThreads) {
+      const uint32_t owner = (uint32_t)(4 * v4 / slice);
+      if (owner == me) continue;
+      const uint32_t local = (uint32_t)__cvta_generic_to_shared(&sh.tot[4 * v4]);
+      reinterpret_cast<int4*>(sh.tot)[v4] = ld_dsmem_v4(local, owner);
+    }
   }
   __syncthreads();
   scan_find(sh, sh.tot, nbins, want);
@@ -277,6 +311,58 @@ inline size_t sel_stage_words(int64_t seg, int half) { return round4(seg) + 2 * 
 // Positions per CTA: a multiple of 4, so that segments start 16-byte aligned.
 __host__ __device__ inline int64_t sel_segment(int64_t L, int cs) { return ((L + cs - 1) / cs + 3) & ~int64_t(3); }
 
+// Row sums of `row_group` score rows over stage positions [p0, p0 + 4*n4)
+// into st4, zero outside [0, L), with 16-byte loads: RU rows x PU positions
+// of loads in flight per thread before any of them is summed (a row-group sum
+// of eight rows then costs one round trip to L2 per position, not eight).
+// Every position is summed in row order starting from +0, whatever RU is.
+template <int RU, int PU>
+__device__ __forceinline__ void stage_row_sums(float4* st4, int n4, const float* rows0, int64_t row_stride,
+                                               int row_group, int64_t p0, int64_t L) {
+  for (int i0 = threadIdx.x; i0 < n4; i0 += kThreads * PU) {
+    float4 acc[PU];
+#pragma unroll
+    for (int u = 0; u < PU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r0 = 0; r0 < row_group; r0 += RU) {
+      float4 x[RU][PU];
+#pragma unroll
+      for (int ru = 0; ru < RU; ++ru) {
+        const float* row = rows0 + (int64_t)(r0 + ru) * row_stride;
+#pragma unroll
+        for (int u = 0; u < PU; ++u) {
+          const int i = i0 + u * kThreads;
+          const int64_t pos = p0 + 4 * (int64_t)i;
+          x[ru][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (r0 + ru < row_group && i < n4) {
+            if (pos >= 0 && pos + 4 <= L) {
+              x[ru][u] = *reinterpret_cast<const float4*>(row + pos);
+            } else {
+              if (pos + 0 >= 0 && pos + 0 < L) x[ru][u].x = row[pos + 0];
+              if (pos + 1 >= 0 && pos + 1 < L) x[ru][u].y = row[pos + 1];
+              if (pos + 2 >= 0 && pos + 2 < L) x[ru][u].z = row[pos + 2];
+              if (pos + 3 >= 0 && pos + 3 < L) x[ru][u].w = row[pos + 3];
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int ru = 0; ru < RU; ++ru) {
+        if (r0 + ru >= row_group) break;
+#pragma unroll
+        for (int u = 0; u < PU; ++u) {
+          acc[u].x += x[ru][u].x;
+          acc[u].y += x[ru][u].y;
+          acc[u].z += x[ru][u].z;
+          acc[u].w += x[ru][u].w;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < PU; ++u)
+      if (i0 + u * kThreads < n4) st4[i0 + u * kThreads] = acc[u];
+  }
+}
+
 template <int CS>
 __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
   pdl_wait();
@@ -354,43 +440,16 @@ __global__ void __launch_bounds__(kThreads, 1) select_kernel(const SelArgs a) {
     const int span = nseg4 + 2 * hs + 4;
     const bool vec_in = ((reinterpret_cast<uintptr_t>(rows0) & 15) == 0) && (a.row_stride & 3) == 0 && (p0 & 3) == 0;
     if (vec_in) {
-      // 16-byte loads, four per thread and row in flight
       float4* st4 = reinterpret_cast<float4*>(stage);
       const int n4 = span / 4;
-      constexpr int kU = 4;
-      for (int i0 = threadIdx.x; i0 < n4; i0 += kThreads * kU) {
-        float4 acc[kU];
-#pragma unroll
-        for (int u = 0; u < kU; ++u) acc[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int r = 0; r < a.row_group; ++r) {
-          const float* row = rows0 + (int64_t)r * a.row_stride;
-          float4 x[kU];
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            const int i = i0 + u * kThreads;
-            const int64_t pos = p0 + 4 * (int64_t)i;
-            x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < n4 && pos >= 0 && pos + 4 <= L) {
-              x[u] = *reinterpret_cast<const float4*>(row + pos);
-            } else if (i < n4) {
-              if (pos + 0 >= 0 && pos + 0 < L) x[u].x = row[pos + 0];
-              if (pos + 1 >= 0 && pos + 1 < L) x[u].y = row[pos + 1];
-              if (pos + 2 >= 0 && pos + 2 < L) x[u].z = row[pos + 2];
-              if (pos + 3 >= 0 && pos + 3 < L) x[u].w = row[pos + 3];
-            }
-          }
-#pragma unroll
-          for (int u = 0; u < kU; ++u) {
-            acc[u].x += x[u].x;
-            acc[u].y += x[u].y;
-            acc[u].z += x[u].z;
-            acc[u].w += x[u].w;
-          }
-        }
-#pragma unroll
-        for (int u = 0; u < kU; ++u)
-          if (i0 + u * kThreads < n4) st4[i0 + u * kThreads] = acc[u];
-      }
+      if (a.row_group >= 8)
+        stage_row_sums<8, 1>(st4, n4, rows0, a.row_stride, a.row_group, p0, L);
+      else if (a.row_group >= 4)
+        stage_row_sums<4, 2>(st4, n4, rows0, a.row_stride, a.row_group, p0, L);
+      else if (a.row_group >= 2)
+        stage_row_sums<2, 2>(st4, n4, rows0, a.row_stride, a.row_group, p0, L);
+      else
+        stage_row_sums<1, 4>(st4, n4, rows0, a.row_stride, a.row_group, p0, L);
     } else {
       // unaligned rows: coalesced 4-byte loads, eight positions per thread in flight
       constexpr int kU = 8;
