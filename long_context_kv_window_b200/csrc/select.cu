@@ -6,7 +6,11 @@
 // StructKV (gist.science 2604.06746) section 2.B: attention entropy, sparsity
 // (here: mass of the top 1 % keys) and variance per layer.
 //
-// Design: one thread-block cluster of kCS CTAs per ranking row.  Each CTA owns a contiguous segment of the row and keeps its pooled values in
+// Design: one thread-block cluster per ranking row -- kCS = 8 CTAs, or
+// kCSWide = 16 for a lone long row (the all-head TSP row) when the device can
+// place such a cluster.  Each CTA owns a contiguous segment of the row; it
+// stages the segment's row sums (a row group, e.g. the eight KV-head rows of
+// the TSP ranking, is summed while staging) and keeps its pooled values in
 // shared memory.  Keys are an order-preserving uint32 image of the fp32 score.
 // The exact k-th largest key is found in three cluster steps:
 //   1. every CTA samples its pooled keys; the cluster's sorted sample brackets
