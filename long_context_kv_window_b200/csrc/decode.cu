@@ -688,41 +688,50 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
   __syncthreads();
   if (!bars->last) return;
   __threadfence();
-  // chunk weights 2^(m_c - M) and the normaliser per head (one warp per head),
-  // in the stage memory, which no copy or MMA uses any more
+  // One warp per head of the group, lane l = output dimensions 4l .. 4l + 3.
+  // The rows of the first 16 chunks are requested together with the chunk
+  // references and sums (one round trip to L2), the weights 2^(m_c - M) and
+  // the normaliser are formed from those, and the remaining rows follow in
+  // batches of 16.  Chunk references and sums are staged in the stage memory,
+  // which no copy or MMA uses any more.  Sums run over the chunks in order.
   const int nch = a.nchunks;
-  float* wv = reinterpret_cast<float*>(sm);  // [G][nch]
-  float* lv = wv + G * nch;                  // [G]
+  float* wv = reinterpret_cast<float*>(sm);  // [G][nch]: references, then weights
+  float* lsm = wv + G * nch;                 // [G][nch]: sums
   for (int hl = warp; hl < G; hl += kTcBlock / 32) {
     const float* pm = a.part_m + (size_t)(g * G + hl) * nch;
     const float* pl = a.part_l + (size_t)(g * G + hl) * nch;
+    const float4* po = reinterpret_cast<const float4*>(a.part_o + (size_t)(g * G + hl) * nch * 128) + lane;
+    float* wh = wv + hl * nch;
+    float* lh = lsm + hl * nch;
+    float4 v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) v[u] = u < nch ? __ldcg(po + (size_t)u * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
     float M = -INFINITY;
-    for (int c = lane; c < nch; c += 32) M = fmaxf(M, __ldcg(pm + c));
+    for (int c = lane; c < nch; c += 32) {
+      const float mc = __ldcg(pm + c);
+      wh[c] = mc;
+      lh[c] = __ldcg(pl + c);
+      M = fmaxf(M, mc);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Ls = 0.f;
     for (int c = lane; c < nch; c += 32) {
-      const float mc = __ldcg(pm + c);
+      const float mc = wh[c];
       const float wc = mc == -INFINITY ? 0.f : tc::ex2_approx(mc - M);
-      wv[hl * nch + c] = wc;
-      Ls += wc * __ldcg(pl + c);
+      wh[c] = wc;
+      Ls += wc * lh[c];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
-    if (lane == 0) lv[hl] = Ls;
-  }
-  __syncthreads();
-  // every thread sums four consecutive dimensions of one head over the chunks,
-  // sixteen 16-byte loads in flight
-  for (int i = tid; i < G * 32; i += kTcBlock) {
-    const int hl = i >> 5, d4 = (i & 31) * 4;
-    const float4* po = reinterpret_cast<const float4*>(a.part_o + (size_t)(g * G + hl) * nch * 128 + d4);
-    const float* wh = wv + hl * nch;
+    __syncwarp();  // every lane's weights are in shared memory
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int c0 = 0; c0 < nch; c0 += 16) {
-      float4 v[16];
+      if (c0 > 0) {
 #pragma unroll
-      for (int u = 0; u < 16; ++u) v[u] = c0 + u < nch ? __ldcg(po + (size_t)(c0 + u) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < 16; ++u)
+          v[u] = c0 + u < nch ? __ldcg(po + (size_t)(c0 + u) * 32) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const float wc = c0 + u < nch ? wh[c0 + u] : 0.f;
@@ -732,9 +741,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant
         acc.w += wc * v[u].w;
       }
     }
-    const float ls = lv[hl];
-    *reinterpret_cast<float4*>(a.out + (size_t)(g * G + hl) * 128 + d4) =
-        make_float4(acc.x / ls, acc.y / ls, acc.z / ls, acc.w / ls);
+    *reinterpret_cast<float4*>(a.out + (size_t)(g * G + hl) * 128 + 4 * lane) =
+        make_float4(acc.x / Ls, acc.y / Ls, acc.z / Ls, acc.w / Ls);
   }
   if (tid == 0) a.cnt[g] = 0u;
 }
