@@ -200,6 +200,26 @@ def test_select_pooled_and_grouped(pool):
         parity.assert_selection_matches(idx[o], ref, Sp, n, w, k)
 
 
+@pytest.mark.parametrize("grp", [2, 3, 5, 7, 8, 16])
+def test_select_row_groups_of_every_size(grp):
+    """Row-group sums formed while staging, for group sizes that take each
+    load-batching shape of the staging (8, 4 or 2 rows per batch of loads,
+    with a partial last batch for 3, 5 and 7 rows): two output rows, each
+    the pooled sum of its group, against the oracle's sums."""
+    rng = np.random.default_rng(100 + grp)
+    n, w, k, pool = 5000, 16, 400, 7
+    rows = 2 * grp
+    S = (rng.random((rows, n)) ** 4).astype(np.float32)
+    pooled = torch.empty((2, n - w), dtype=torch.float32, device="cuda")
+    idx = kvc.kvc_select_topk(torch.from_numpy(S).cuda(), w, pool, k, row_group=grp, pooled=pooled).cpu().numpy()
+    orc = oracle.get()
+    for o in range(2):
+        T = orc.sum_rows(S[o * grp:(o + 1) * grp].astype(np.float64))
+        Sp = orc.rank_scores(T, n, w, pool)
+        parity.assert_scores_close(pooled[o].cpu().numpy(), Sp, rtol=1e-6, what=f"pooled, groups of {grp}")
+        parity.assert_selection_matches(idx[o], orc.select_topk(Sp, n, w, k), Sp, n, w, k)
+
+
 # --------------------------------------------------------------------------- #
 # scoring + selection + gathers on the configurations
 # --------------------------------------------------------------------------- #
