@@ -273,3 +273,68 @@ def test_pivot_update_checks(lib):
             kvc.kvc_pivot_update(**args)
     assert lib.calls == ["kvc_pivot_update"]
 
+
+
+def test_decode_checks(lib):
+    H, Hkv, d, kk = 8, 2, 64, 50
+    q = torch.empty((H, d), dtype=bf)
+    kc, vc = torch.empty((Hkv, kk, d), dtype=bf), torch.empty((Hkv, kk, d), dtype=bf)
+    ok = dict(out=torch.empty((H, d), dtype=f32), ws=_ws(), dev_err=torch.zeros(1, dtype=i32))
+    out = kvc.kvc_decode_attention(q, kc, vc, **ok)
+    assert out is ok["out"] and lib.calls == ["kvc_decode_attention"]
+    bad_inputs = [(torch.empty((H, d + 8), dtype=bf), kc, vc),                       # head_dim differs
+                  (q, kc, torch.empty((Hkv, kk + 1, d), dtype=bf)),                  # V rows differ
+                  (q, torch.empty((Hkv, 2 * kk, d), dtype=bf)[:, ::2], vc),           # not contiguous
+                  (q.float(), kc, vc)]                                                # not bf16
+    for qq, kk_, vv in bad_inputs:
+        with pytest.raises((ValueError, TypeError)):
+            kvc.kvc_decode_attention(qq, kk_, vv, **ok)
+    for b in (dict(out=torch.empty((H, d), dtype=torch.float64)), dict(out=torch.empty((H + 1, d), dtype=f32)),
+              dict(dev_err=torch.zeros(1, dtype=torch.int64)), dict(ws=torch.empty(32, dtype=torch.uint8)[::2])):
+        with pytest.raises((ValueError, TypeError)):
+            kvc.kvc_decode_attention(q, kc, vc, **{**ok, **b})
+    assert lib.calls == ["kvc_decode_attention"]
+
+
+def test_prefill_checks(lib):
+    n, H, Hkv, d = 20, 8, 2, 64
+    q = torch.empty((n, H, d), dtype=bf)
+    k, v = torch.empty((n, Hkv, d), dtype=bf), torch.empty((n, Hkv, d), dtype=bf)
+    out, lse = kvc.kvc_prefill_attention(q, k, v, dev_err=torch.zeros(1, dtype=i32))
+    assert tuple(out.shape) == (n, H, d) and out.dtype == bf
+    assert tuple(lse.shape) == (n, H) and lse.dtype == f32
+    out2, _ = kvc.kvc_prefill_attention(q, k, v, want_out=False)
+    assert out2 is None and lib.calls == ["kvc_prefill_attention"] * 2
+    bad_inputs = [(q, torch.empty((n + 1, Hkv, d), dtype=bf), v),                   # rows differ
+                  (q, k, torch.empty((n, Hkv + 1, d), dtype=bf)),                    # V heads differ
+                  (q, torch.empty((n, Hkv, d + 8), dtype=bf), v),                    # head_dim differs
+                  (torch.empty((n, 2 * H, d), dtype=bf)[:, ::2], k, v)]              # not contiguous
+    for qq, kk_, vv in bad_inputs:
+        with pytest.raises((ValueError, TypeError)):
+            kvc.kvc_prefill_attention(qq, kk_, vv)
+    for b in (dict(out=torch.empty((n, H, d + 1), dtype=bf)), dict(out=torch.empty((n, H, d), dtype=f32)),
+              dict(lse=torch.empty((n, H), dtype=torch.float64)), dict(lse=torch.empty((H, n), dtype=f32)),
+              dict(dev_err=torch.zeros(1, dtype=torch.int64))):
+        with pytest.raises((ValueError, TypeError)):
+            kvc.kvc_prefill_attention(q, k, v, **b)
+    assert lib.calls == ["kvc_prefill_attention"] * 2
+
+
+def test_rvq_checks(lib):
+    n, d, S, M = 30, 64, 3, 16
+    x, cb = torch.empty((n, d), dtype=bf), torch.empty((S, M, d), dtype=f32)
+    codes, res = kvc.kvc_rvq_encode(x, cb, residual=torch.empty((n, d), dtype=f32))
+    assert tuple(codes.shape) == (n, S) and codes.dtype == i32 and tuple(res.shape) == (n, d)
+    codes, res = kvc.kvc_rvq_encode(x, cb)
+    assert res is None and lib.calls == ["kvc_rvq_encode"] * 2
+    for bad_cb in (torch.empty((S, M, d), dtype=torch.float64), torch.empty((S, M, d + 1), dtype=f32),
+                   torch.empty((S, d, M), dtype=f32).transpose(1, 2), torch.empty((M, d), dtype=f32)):
+        with pytest.raises((ValueError, TypeError)):
+            kvc.kvc_rvq_encode(x, bad_cb)
+    for b in (dict(codes=torch.empty((n, S + 1), dtype=i32)), dict(codes=torch.empty((n, S), dtype=torch.int64)),
+              dict(residual=torch.empty((n, d + 1), dtype=f32)), dict(dev_err=torch.zeros(1, dtype=torch.int64))):
+        with pytest.raises((ValueError, TypeError)):
+            kvc.kvc_rvq_encode(x, cb, **b)
+    with pytest.raises((ValueError, TypeError)):
+        kvc.kvc_rvq_encode(x.float(), cb)
+    assert lib.calls == ["kvc_rvq_encode"] * 2
